@@ -1,0 +1,221 @@
+/*
+ * fh.h -- C ABI of the B200 FlashHead retrieval head.
+ *
+ * FlashHead replaces the dense LM classification head z = E h (FlashHead
+ * write-up, www.framerc.cn/news/2430929, section 1.1) by a two-stage
+ * retrieval (section 2.2.2: h -> centroid_scores -> top_p_clusters ->
+ * token_scores):
+ *
+ *   1. centroid scores  s = C h over c balanced clusters (section 1.2.2),
+ *      C in bf16 or in INT4 with one bf16 scale per 32 elements
+ *      (selective quantisation, section 1.2.4);
+ *   2. probe selection: the p best clusters (multi-probe retrieval,
+ *      section 1.2.2), or p clusters drawn by multinomial sampling at
+ *      temperature T (section 1.2.3), realised as the top p of
+ *      s/T + g with Gumbel noise g = -ln(-ln u) from caller uniforms u;
+ *   3. gather of the b = v/c tokens of every chosen cluster through the
+ *      dense cluster-to-token map C2T (balanced clustering, section 1.2.1);
+ *   4. candidate logits z_t = E_t h for those p*b tokens (section 1.2.4,
+ *      stage 2 in full precision);
+ *   5. argmax, or a token drawn from softmax(z/T) over the candidates by
+ *      inverse CDF with a caller uniform (section 1.2.3).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers named as device pointers must be CUDA device memory of the
+ *   current device; the caller owns them. E, C / C_q / C_scales and C2T are
+ *   borrowed by fh_create and must outlive the handle.
+ * - bf16 data is passed as `const void*` (IEEE bfloat16, row-major).
+ * - Every call is asynchronous on `stream` (a cudaStream_t) unless stated
+ *   otherwise. Argument errors are detected on the host and returned at
+ *   once, before anything is enqueued. Errors found by a kernel (an
+ *   out-of-range cluster id, a bounded wait that ran out) are recorded in a
+ *   device status word and reported by fh_get_device_status().
+ * - Ties: a ranking of clusters breaks equal keys by the lower cluster id,
+ *   an argmax of logits by the lower token id.
+ * - The library allocates device memory only in fh_create (one workspace
+ *   sized by max_batch and max_probes) and frees it in fh_destroy.
+ *   Calls on one handle must be stream-ordered (they share the workspace).
+ * - Accumulation is fp32; results match an fp64 evaluation of the same
+ *   steps within 2e-3 * |row| * |h| (row = the centroid or token row).
+ */
+#ifndef FH_H_
+#define FH_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* fh_stream_t;
+
+typedef enum {
+  FH_OK = 0,
+  FH_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, size out of range, bad mode or T */
+  FH_ERR_INVALID_C2T = 2,   /* C2T is not a permutation of 0..v-1 */
+  FH_ERR_UNSUPPORTED = 3,   /* device is not sm_100, or a shape this build does not handle */
+  FH_ERR_OOM = 4,           /* workspace allocation failed */
+  FH_ERR_CUDA = 5,          /* a CUDA runtime call failed */
+  FH_ERR_OUT_OF_RANGE = 6,  /* (device) a cluster id outside [0, c) or repeated in a row */
+  FH_ERR_TIMEOUT = 7        /* (device) a bounded wait inside a kernel ran out */
+} fh_status;
+
+typedef enum {
+  FH_CENTROID_BF16 = 0,     /* C: bf16 [c, d] */
+  FH_CENTROID_INT4_G32 = 1  /* C_q: uint8 [c, d/2], C_scales: bf16 [c, d/32] */
+} fh_centroid_format;
+
+typedef enum {
+  FH_GREEDY = 0,            /* top-p clusters by score, argmax token */
+  FH_SAMPLE_GUMBEL = 1      /* Gumbel-top-p clusters at T, softmax(z/T) token */
+} fh_mode;
+
+/*
+ * Head description (balanced clustering, write-up section 1.2.1: every one of
+ * the c clusters holds exactly b = v/c tokens; C2T[k][j] is the j-th token of
+ * cluster k, so slot k*b + j of the flattened map names one token).
+ *
+ *  v, d, c, b   vocabulary, hidden size, clusters, tokens per cluster;
+ *               v == c*b, d % 8 == 0 (d % 32 == 0 for INT4), 1 <= c.
+ *  E            device bf16 [v, d], 16-byte aligned.
+ *  C            device bf16 [c, d], 16-byte aligned (BF16 format, else NULL).
+ *  C_q          device uint8 [c, d/2] (INT4 format): element 2i in the low
+ *               nibble of byte i, 2i+1 in the high nibble, two's complement.
+ *  C_scales     device bf16 [c, d/32] (INT4 format): value = code * scale.
+ *  C2T          device int32 [c, b].
+ *  fmt          fh_centroid_format.
+ *  max_batch    largest B any call will pass (>= 1).
+ *  max_probes   largest p any call will pass (1 <= max_probes <= c).
+ */
+typedef struct {
+  int32_t v, d, c, b;
+  const void* E;
+  const void* C;
+  const uint8_t* C_q;
+  const void* C_scales;
+  const int32_t* C2T;
+  int32_t fmt;
+  int32_t max_batch;
+  int32_t max_probes;
+} fh_head_desc;
+
+typedef struct fh_head fh_head;
+
+/*
+ * Create a head. Validates the description, checks on the device that C2T
+ * is a permutation of 0..v-1 (FH_ERR_INVALID_C2T otherwise), allocates the
+ * workspace, and for INT4 packs each centroid row with its scales into a
+ * library-owned copy (row = d/2 code bytes, then d/16 scale bytes, padded to
+ * 16 bytes) so that one bulk copy moves a row. Synchronises `stream` once.
+ * On success *out owns the workspace; release it with fh_destroy.
+ */
+fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out);
+
+/* Free the workspace and the handle. Waits for the device first. NULL is a no-op. */
+void fh_destroy(fh_head* head);
+
+/*
+ * Stage 1 (write-up section 1.2.2): scores[r][k] = sum_i C[k][i] * hidden[r][i]
+ * for r < B, k < c (INT4: C dequantised exactly, code * scale).
+ *  hidden  device bf16 [B, d], 16-byte aligned.
+ *  scores  device fp32 [B, c].
+ */
+fh_status fh_centroid_scores(fh_head* head, const void* hidden, int32_t B, float* scores,
+                             fh_stream_t stream);
+
+/*
+ * Probe selection (sections 1.2.2 and 1.2.3). For each row r the p clusters
+ * with the largest key, key = scores (FH_GREEDY) or scores/T - ln(-ln u)
+ * with u = u_clusters[r][k] clamped to [2^-126, 1 - 2^-24] (FH_SAMPLE_GUMBEL).
+ *  scores       device fp32 [B, c].
+ *  u_clusters   device fp32 [B, c]; only read in FH_SAMPLE_GUMBEL (else may be NULL).
+ *  cluster_ids  device int32 [B, p], written in ascending cluster-id order.
+ * T must be finite and > 0 in FH_SAMPLE_GUMBEL; 1 <= p <= max_probes.
+ */
+fh_status fh_select_clusters(fh_head* head, const float* scores, int32_t B, int32_t p,
+                             int32_t mode, float T, const float* u_clusters,
+                             int32_t* cluster_ids, fh_stream_t stream);
+
+/*
+ * Gather + stage 2 (sections 1.2.1 and 1.2.4). For row r, the candidates
+ * are the tokens of the clusters in cluster_ids[r] taken in canonical order
+ * (cluster id ascending, slot j ascending): for the q-th smallest chosen
+ * cluster k, position q*b + j holds token C2T[k][j] and its logit
+ * E[token] . hidden[r].
+ *  cluster_ids  device int32 [B, p], any order, distinct within a row.
+ *  token_ids    device int32 [B, p*b].
+ *  logits       device fp32  [B, p*b].
+ * A row with an id outside [0, c) or a repeated id is skipped (its outputs
+ * are left untouched) and FH_ERR_OUT_OF_RANGE is recorded on the device.
+ */
+fh_status fh_candidate_logits(fh_head* head, const void* hidden, int32_t B, int32_t p,
+                              const int32_t* cluster_ids, int32_t* token_ids, float* logits,
+                              fh_stream_t stream);
+
+/*
+ * The whole head (section 2.2.2): scores, selection, gather, candidate
+ * logits and the output token, fused so that intermediates stay on chip or
+ * in the workspace.
+ *  hidden           device bf16 [B, d], 16-byte aligned.
+ *  u_clusters       device fp32 [B, c]  (FH_SAMPLE_GUMBEL only, else NULL).
+ *  u_token          device fp32 [B]     (FH_SAMPLE_GUMBEL only, else NULL);
+ *                   clamped to [0, 1 - 2^-24]; the token is the first
+ *                   candidate, in canonical order, whose running sum of
+ *                   exp(z/T - max z/T) exceeds u_token * total.
+ *  out_tokens       device int32 [B].
+ *  out_cluster_ids  device int32 [B, p] ascending, or NULL.
+ *  out_max_logit    device fp32 [B] (largest candidate logit), or NULL.
+ */
+fh_status fh_decode(fh_head* head, const void* hidden, int32_t B, int32_t p, int32_t mode,
+                    float T, const float* u_clusters, const float* u_token,
+                    int32_t* out_tokens, int32_t* out_cluster_ids, float* out_max_logit,
+                    fh_stream_t stream);
+
+/*
+ * Dense comparison head (write-up section 1.1): z = E h over the whole
+ * vocabulary and its argmax.
+ *  logits      device fp32 [B, v], or NULL to skip writing them.
+ *  out_argmax  device int32 [B].
+ */
+fh_status fh_dense_head(fh_head* head, const void* hidden, int32_t B, float* logits,
+                        int32_t* out_argmax, fh_stream_t stream);
+
+/*
+ * Synchronise `stream`, then return and clear the device status word
+ * (FH_OK if no kernel recorded an error since the last read).
+ */
+fh_status fh_get_device_status(fh_head* head, fh_stream_t stream);
+
+/* Static description of a status code. */
+const char* fh_status_string(fh_status status);
+
+/*
+ * Clock-cycle budget of the device-wide waits inside fused kernels (default
+ * about one second). A wait that runs out records FH_ERR_TIMEOUT and its
+ * kernel returns early; 0 makes every such wait give up at once (used to
+ * exercise that path).
+ */
+fh_status fh_set_spin_budget(fh_head* head, int64_t cycles);
+
+/*
+ * Introspection: FH_QUERY_WORKSPACE_BYTES, FH_QUERY_LAST_UNION (number of
+ * distinct clusters gathered by the last batched fh_decode, after
+ * fh_get_device_status or a stream sync), FH_QUERY_NUM_SMS,
+ * FH_QUERY_FUSED_B1 (1 if B = 1 decodes run the single fused kernel).
+ */
+typedef enum {
+  FH_QUERY_WORKSPACE_BYTES = 0,
+  FH_QUERY_LAST_UNION = 1,
+  FH_QUERY_NUM_SMS = 2,
+  FH_QUERY_FUSED_B1 = 3
+} fh_query_key;
+fh_status fh_query(fh_head* head, int32_t key, int64_t* value);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FH_H_ */

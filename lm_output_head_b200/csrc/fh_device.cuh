@@ -1,0 +1,464 @@
+// Device building blocks shared by the FlashHead kernels (sm_100a).
+//
+//  * bulk global->shared copies (cp.async.bulk) completed on mbarriers, with
+//    bounded waits;
+//  * order-preserving float <-> uint32 keys and packed (logit, token) argmax
+//    words;
+//  * bf16 / INT4 unpacking into fp32;
+//  * block-wide scans and the block radix select that picks the p largest
+//    keys (ties to the lower id), used for probe selection (multi-probe
+//    retrieval, FlashHead write-up section 1.2.2).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "fh_internal.h"
+
+namespace fh {
+
+constexpr int kThreads = 512;           // threads per CTA of the streaming kernels
+constexpr int kWarps = kThreads / 32;
+
+// ---------------------------------------------------------------------------
+// status word
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void record_error(int* status, int code) {
+  atomicCAS(status, 0, code);
+}
+
+// ---------------------------------------------------------------------------
+// shared-memory addresses, mbarriers, bulk copies
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+// One contiguous global->shared copy; both addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for phase `parity` of `bar` for at most `budget` SM clock cycles.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, long long budget) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > budget) return false;
+  }
+  return true;
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint16_t lds16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+
+// ---------------------------------------------------------------------------
+// number formats
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+
+// Signed 4-bit code (two's complement) in bits [4i, 4i+4) of w, as an exact float.
+// (n ^ 8) maps -8..7 to 0..15; OR-ing it into the mantissa of 2^23 gives 2^23 + (n ^ 8)
+// exactly, and subtracting 2^23 + 8 leaves the signed code.
+__device__ __forceinline__ float nib(uint32_t w, int i) {
+  const uint32_t u = ((w >> (4 * i)) & 0xFu) ^ 0x8u;
+  return __uint_as_float(0x4B000000u | u) - 8388616.0f;
+}
+
+// Dot of 8 bf16 (one 16-byte chunk) with 8 fp32 values.
+__device__ __forceinline__ float dot8(const uint4 w, const float* h, float acc) {
+  acc = fmaf(bf16lo(w.x), h[0], acc);
+  acc = fmaf(bf16hi(w.x), h[1], acc);
+  acc = fmaf(bf16lo(w.y), h[2], acc);
+  acc = fmaf(bf16hi(w.y), h[3], acc);
+  acc = fmaf(bf16lo(w.z), h[4], acc);
+  acc = fmaf(bf16hi(w.z), h[5], acc);
+  acc = fmaf(bf16lo(w.w), h[6], acc);
+  acc = fmaf(bf16hi(w.w), h[7], acc);
+  return acc;
+}
+
+// Dot of 16 INT4 codes (8 bytes) with 16 fp32 values; the group scale is applied by the caller.
+__device__ __forceinline__ float dot16q(const uint2 q, const float* h) {
+  float a = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a = fmaf(nib(q.x, i), h[i], a);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a = fmaf(nib(q.y, i), h[8 + i], a);
+  return a;
+}
+
+// ---------------------------------------------------------------------------
+// keys
+// ---------------------------------------------------------------------------
+// Monotone map float -> uint32 (larger float => larger key).
+__device__ __forceinline__ uint32_t f2key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key2f(uint32_t k) {
+  const uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+  return __uint_as_float(u);
+}
+// (logit, token) packed so that a larger word = larger logit, then lower token id.
+__device__ __forceinline__ unsigned long long pack_best(float z, int32_t token) {
+  return (static_cast<unsigned long long>(f2key(z)) << 32) |
+         static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(token));
+}
+__device__ __forceinline__ int32_t best_token(unsigned long long w) {
+  return static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(w & 0xFFFFFFFFull));
+}
+__device__ __forceinline__ float best_logit(unsigned long long w) {
+  return key2f(static_cast<uint32_t>(w >> 32));
+}
+
+// Gumbel-perturbed key s/T - ln(-ln u), u clamped to [2^-126, 1 - 2^-24].
+__device__ __forceinline__ float gumbel_key(float s, float T, float u) {
+  u = fminf(fmaxf(u, 1.17549435e-38f), 0.99999994f);
+  return s / T - logf(-logf(u));
+}
+
+// ---------------------------------------------------------------------------
+// warp / block reductions and scans
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long w = __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    v = w > v ? w : v;
+  }
+  return v;
+}
+
+// Exclusive scan of one value per thread over the block (NT threads);
+// `scratch` holds NT/32 + 1 words. Returns the exclusive prefix; *total gets the sum.
+template <int NT, typename T>
+__device__ __forceinline__ T block_exclusive_scan(T v, T* scratch, T* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  T x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const T y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) scratch[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    const T t = lane < NT / 32 ? scratch[lane] : T(0);
+    T s = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const T y = __shfl_up_sync(0xFFFFFFFFu, s, o);
+      if (lane >= o) s += y;
+    }
+    if (lane < NT / 32) scratch[lane] = s - t;
+    if (lane == NT / 32 - 1) scratch[NT / 32] = s;
+  }
+  __syncthreads();
+  const T r = scratch[w] + x - v;
+  if (total) *total = scratch[NT / 32];
+  __syncthreads();
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// block top-p select
+// ---------------------------------------------------------------------------
+struct SelectSmem {
+  uint32_t hist[2048];
+  uint32_t scan[kWarps + 1];
+  uint32_t warp_gt[kWarps];
+  uint32_t warp_eq[kWarps];
+  uint32_t digit, above, bincount;
+};
+
+// Selects the p largest of n keys (order-preserving uint32) held in shared
+// memory; equal keys go to the lower id. Writes the chosen ids to `sel`
+// (shared or global) in ascending id order. All kThreads threads must call it.
+//
+// MSB-first radix select with 11/11/10-bit digits: each pass histograms the
+// keys that still agree with the decided prefix, finds the digit where the
+// count from the top reaches the remaining need, and stops early once that
+// digit's bin holds exactly the keys still needed.
+__device__ inline void block_select_top_p(const uint32_t* skey, int n, int p, int32_t* sel,
+                                          SelectSmem& sm) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t prefix = 0, mask = 0;
+  int need = p;
+  const int shifts[3] = {21, 10, 0};
+  const uint32_t digit_mask[3] = {0x7FFu, 0x7FFu, 0x3FFu};
+  const int iters = (n + kThreads - 1) / kThreads;
+
+  for (int pass = 0; pass < 3; ++pass) {
+    const int sh = shifts[pass];
+    const uint32_t dm = digit_mask[pass];
+    for (int i = tid; i < 2048; i += kThreads) sm.hist[i] = 0;
+    __syncthreads();
+    for (int it = 0; it < iters; ++it) {
+      const int k = it * kThreads + tid;
+      bool act = k < n;
+      const uint32_t key = act ? skey[k] : 0u;
+      act = act && ((key & mask) == prefix);
+      const uint32_t bin = (key >> sh) & dm;
+      const uint32_t grp = __match_any_sync(0xFFFFFFFFu, act ? bin : (0x10000u | lane));
+      if (act && lane == __ffs(grp) - 1) atomicAdd(&sm.hist[bin], static_cast<uint32_t>(__popc(grp)));
+    }
+    __syncthreads();
+    // thread t owns bins 2047-4t .. 2044-4t (descending), so the exclusive
+    // scan gives the number of keys in higher bins
+    constexpr int kBpt = 2048 / kThreads;
+    uint32_t loc = 0;
+#pragma unroll
+    for (int i = 0; i < kBpt; ++i) loc += sm.hist[2047 - kBpt * tid - i];
+    const uint32_t above = block_exclusive_scan<kThreads, uint32_t>(loc, sm.scan, nullptr);
+    uint32_t run = above;
+#pragma unroll
+    for (int i = 0; i < kBpt; ++i) {
+      const int dg = 2047 - kBpt * tid - i;
+      const uint32_t h = sm.hist[dg];
+      if (run < static_cast<uint32_t>(need) && run + h >= static_cast<uint32_t>(need)) {
+        sm.digit = static_cast<uint32_t>(dg);
+        sm.above = run;
+        sm.bincount = h;
+      }
+      run += h;
+    }
+    __syncthreads();
+    need -= static_cast<int>(sm.above);
+    prefix |= sm.digit << sh;
+    mask |= dm << sh;
+    const bool done = sm.bincount == static_cast<uint32_t>(need);
+    __syncthreads();
+    if (done) break;
+  }
+
+  // Compaction in ascending id order. Keys with (key & mask) > prefix are
+  // taken; of those equal to prefix under the mask, the first `need` ids.
+  const int per_warp = ((n + kWarps - 1) / kWarps + 31) & ~31;
+  const int w0 = warp * per_warp, w1 = min(n, w0 + per_warp);
+  uint32_t cgt = 0, ceq = 0;
+  for (int k0 = w0; k0 < w1; k0 += 32) {
+    const int k = k0 + lane;
+    const uint32_t mk = k < w1 ? (skey[k] & mask) : 0u;
+    const bool in = k < w1;
+    cgt += __popc(__ballot_sync(0xFFFFFFFFu, in && mk > prefix));
+    ceq += __popc(__ballot_sync(0xFFFFFFFFu, in && mk == prefix));
+  }
+  if (lane == 0) {
+    sm.warp_gt[warp] = cgt;
+    sm.warp_eq[warp] = ceq;
+  }
+  __syncthreads();
+  uint32_t gt_before = 0, eq_before = 0;
+  for (int w = 0; w < warp; ++w) {
+    gt_before += sm.warp_gt[w];
+    eq_before += sm.warp_eq[w];
+  }
+  uint32_t pos = gt_before + min(eq_before, static_cast<uint32_t>(need));
+  uint32_t eq_seen = eq_before;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int k0 = w0; k0 < w1; k0 += 32) {
+    const int k = k0 + lane;
+    const bool in = k < w1;
+    const uint32_t mk = in ? (skey[k] & mask) : 0u;
+    const bool gt = in && mk > prefix;
+    const bool eq = in && mk == prefix;
+    const uint32_t eqm = __ballot_sync(0xFFFFFFFFu, eq);
+    const bool take = gt || (eq && eq_seen + __popc(eqm & lt_mask) < static_cast<uint32_t>(need));
+    const uint32_t tm = __ballot_sync(0xFFFFFFFFu, take);
+    const uint32_t at = pos + __popc(tm & lt_mask);
+    if (take && at < static_cast<uint32_t>(p)) sel[at] = k;
+    pos += __popc(tm);
+    eq_seen += __popc(eqm);
+  }
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
+// per-warp streaming of rows through a ring of shared-memory slots
+// ---------------------------------------------------------------------------
+// Each warp owns `nslot` slots of `slot_bytes` and one mbarrier per slot.
+// Item i of the warp's n items is copied by one cp.async.bulk into slot
+// i % nslot; lane 0 issues, all lanes wait, `use(i, slot_addr)` consumes, and
+// the slot is refilled with item i + nslot. `src(i, ptr, bytes)` is evaluated
+// by all lanes (it may shuffle prefetched ids). A wait that exceeds `budget`
+// cycles makes the warp wait (bounded) for its copies still in flight and
+// return false.
+template <class Src, class Use>
+__device__ __forceinline__ bool warp_stream(int n, int nslot, uint32_t ring, uint32_t slot_bytes,
+                                            uint32_t bars, uint32_t& phase_bits, long long budget,
+                                            Src src, Use use) {
+  const int lane = threadIdx.x & 31;
+  const int pre = n < nslot ? n : nslot;
+  for (int s = 0; s < pre; ++s) {
+    const void* ptr;
+    uint32_t bytes;
+    src(s, ptr, bytes);
+    if (lane == 0) {
+      mbar_expect_tx(bars + 8u * s, bytes);
+      bulk_g2s(ring + s * slot_bytes, ptr, bytes, bars + 8u * s);
+    }
+  }
+  for (int i = 0; i < n; ++i) {
+    const int s = i % nslot;
+    const uint32_t bar = bars + 8u * s;
+    const bool got = mbar_wait_bounded(bar, (phase_bits >> s) & 1u, budget);
+    if (!__all_sync(0xFFFFFFFFu, got)) {
+      const int last = (i + nslot < n) ? i + nslot : n;
+      for (int j = i; j < last; ++j) {
+        const int sj = j % nslot;
+        mbar_wait_bounded(bars + 8u * sj, (phase_bits >> sj) & 1u, budget);
+      }
+      __syncwarp();
+      return false;
+    }
+    phase_bits ^= 1u << s;
+    use(i, ring + s * slot_bytes);
+    __syncwarp();
+    if (i + nslot < n) {
+      const void* ptr;
+      uint32_t bytes;
+      src(i + nslot, ptr, bytes);
+      if (lane == 0) {
+        fence_proxy_async_smem();
+        mbar_expect_tx(bar, bytes);
+        bulk_g2s(ring + s * slot_bytes, ptr, bytes, bar);
+      }
+    }
+  }
+  return true;
+}
+
+// Load this lane's slice of a bf16 vector into fp32 registers in the layout
+// of 16-byte chunks: chunk m covers elements (lane + 32 m) * 8 .. + 8.
+template <int NCH>
+__device__ __forceinline__ void load_h_chunks(const uint16_t* h, int d, float* hr) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int m = 0; m < NCH; ++m) {
+    const int e = (lane + 32 * m) * 8;
+    uint4 w = make_uint4(0, 0, 0, 0);
+    if (e < d) w = *reinterpret_cast<const uint4*>(h + e);
+    hr[8 * m + 0] = bf16lo(w.x); hr[8 * m + 1] = bf16hi(w.x);
+    hr[8 * m + 2] = bf16lo(w.y); hr[8 * m + 3] = bf16hi(w.y);
+    hr[8 * m + 4] = bf16lo(w.z); hr[8 * m + 5] = bf16hi(w.z);
+    hr[8 * m + 6] = bf16lo(w.w); hr[8 * m + 7] = bf16hi(w.w);
+  }
+}
+
+// Same for the INT4 layout: half-group g (16 elements) = (lane + 32 m), NQ of them.
+template <int NQ>
+__device__ __forceinline__ void load_h_halfgroups(const uint16_t* h, int d, float* hq) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int m = 0; m < NQ; ++m) {
+    const int e = (lane + 32 * m) * 16;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint4 w = make_uint4(0, 0, 0, 0);
+      if (e < d) w = *reinterpret_cast<const uint4*>(h + e + 8 * half);
+      float* o = hq + 16 * m + 8 * half;
+      o[0] = bf16lo(w.x); o[1] = bf16hi(w.x); o[2] = bf16lo(w.y); o[3] = bf16hi(w.y);
+      o[4] = bf16lo(w.z); o[5] = bf16hi(w.z); o[6] = bf16lo(w.w); o[7] = bf16hi(w.w);
+    }
+  }
+}
+
+// Dot of a bf16 row in shared memory with register-resident h (chunk layout), warp-reduced.
+template <int NCH>
+__device__ __forceinline__ float row_dot_bf16(uint32_t row, int d, const float* hr) {
+  const int lane = threadIdx.x & 31;
+  float acc = 0.f;
+#pragma unroll
+  for (int m = 0; m < NCH; ++m) {
+    const int e = (lane + 32 * m) * 8;
+    if (e < d) acc = dot8(lds128(row + 2u * e), hr + 8 * m, acc);
+  }
+  return warp_sum(acc);
+}
+
+// Dot of a packed INT4 row ([d/2 code bytes][d/16 scale bytes]) with h in the half-group layout.
+template <int NQ>
+__device__ __forceinline__ float row_dot_int4(uint32_t row, int d, const float* hq) {
+  const int lane = threadIdx.x & 31;
+  float acc = 0.f;
+#pragma unroll
+  for (int m = 0; m < NQ; ++m) {
+    const int g = lane + 32 * m;  // half-group
+    if (g * 16 < d) {
+      const uint2 q = lds64(row + 8u * g);
+      const float sc = bf16f(lds16(row + d / 2 + 2u * (g >> 1)));
+      acc = fmaf(sc, dot16q(q, hq + 16 * m), acc);
+    }
+  }
+  return warp_sum(acc);
+}
+
+}  // namespace fh

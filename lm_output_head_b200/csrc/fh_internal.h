@@ -1,0 +1,156 @@
+// Internal declarations shared by the host layer and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "fh.h"
+
+namespace fh {
+
+// Largest hidden size the register-resident kernels handle: each lane keeps
+// ceil(d/256) 16-byte chunks of h (8 fp32 each) in registers.
+constexpr int kMaxD = 2560;
+constexpr long long kWaitBudget = 4000000000LL;      // bulk-copy waits (~2 s)
+constexpr long long kDefaultSpinBudget = 2000000000LL;  // device-wide waits (~1 s)
+
+// Workspace words at the start of the workspace.
+struct SyncWords {
+  int32_t status;
+  uint32_t arrive;        // grid barrier arrivals
+  uint32_t ticket;        // kernel exit tickets (last CTA finalises)
+  uint32_t union_count;   // distinct clusters of the last batched decode
+  uint32_t pad[4];
+};
+
+struct B1Params {
+  const uint16_t* E;
+  const uint8_t* Crows;   // bf16 rows (d*2 bytes) or packed INT4 rows (rs bytes)
+  const int32_t* C2T;
+  const uint16_t* hidden;
+  const float* u_clusters;
+  const float* u_token;
+  int32_t* out_tokens;
+  int32_t* out_cluster_ids;
+  float* out_max_logit;
+  float* scores;          // workspace [c]
+  float* cand_logits;     // workspace [p*b]
+  unsigned long long* best;
+  SyncWords* sync;
+  int v, d, c, b, p;
+  int crow_bytes;         // bytes per centroid row in Crows
+  int mode;
+  float T;
+  int nslot, slot_bytes;
+  int off_h, off_bar, off_sel, off_misc, off_ring;
+  long long spin_budget;
+};
+
+struct ScoresParams {
+  const uint8_t* Crows;
+  const uint16_t* hidden;  // [B, d]
+  const float* u_clusters; // [B, c] (gumbel)
+  float* out;              // [B, c]
+  int*  status;
+  int d, c, crow_bytes;
+  int row0, rows;          // hidden rows [row0, row0+rows) in this launch
+  int mode;                // 0 raw scores, 1 Gumbel keys
+  float T;
+  int nslot, slot_bytes;
+  int off_h, off_bar, off_ring;
+};
+
+struct SelectParams {
+  const float* in;         // [B, c] scores or keys
+  const float* u_clusters; // [B, c] when perturb
+  const int32_t* ids_in;   // [B, p] explicit ids (sort mode) or null
+  const int32_t* C2T;
+  int32_t* sel;            // [B, p] ascending
+  int32_t* cand_tok;       // [B, p*b] canonical token ids, or null
+  int32_t* row_ok;         // [B] (sort mode) or null
+  int*  status;
+  int c, b, p;
+  int perturb;             // compute Gumbel keys from scores + u
+  float T;
+};
+
+struct CandParams {
+  const uint16_t* E;
+  const uint16_t* hidden;   // [B, d]
+  const int32_t* cand_tok;  // [B, p*b]
+  const int32_t* row_ok;    // [B] or null
+  float* logits;            // [B, p*b] or null
+  int32_t* token_out;       // [B, p*b] or null
+  unsigned long long* best; // [B] or null
+  int*  status;
+  int v, d, nc, B;
+  int nslot, slot_bytes;
+  int off_bar, off_ring;
+};
+
+struct EpilogueParams {
+  const float* logits;      // [B, nc]
+  const int32_t* cand_tok;  // [B, nc]
+  const float* u_token;
+  unsigned long long* best; // [B]
+  int32_t* out_tokens;
+  float* out_max_logit;
+  int nc, mode;
+  float T;
+};
+
+struct DenseParams {
+  const uint16_t* E;
+  const uint16_t* hidden;   // [B, d]
+  float* logits;            // [B, v] or null
+  int32_t* out_argmax;      // [B]
+  unsigned long long* best; // [B]
+  SyncWords* sync;
+  int v, d;
+  int row0, rows;
+  int nslot, slot_bytes;
+  int off_h, off_bar, off_ring;
+};
+
+struct C2TCheckParams {
+  const int32_t* C2T;
+  uint32_t* counts;         // [v]
+  int* bad;
+  long long n;
+  int v;
+};
+
+struct RepackParams {
+  const uint8_t* C_q;
+  const uint16_t* C_scales;
+  uint8_t* out;
+  int c, d, rs;
+};
+
+// Launchers (defined in the .cu files). Each returns the CUDA error of the launch.
+cudaError_t launch_decode_b1(const B1Params& P, int grid, size_t smem, int int4, int nch,
+                             cudaStream_t st);
+cudaError_t launch_scores(const ScoresParams& P, int grid, size_t smem, int int4, int nch,
+                          cudaStream_t st);
+cudaError_t launch_select(const SelectParams& P, int B, size_t smem, cudaStream_t st);
+cudaError_t launch_sort_ids(const SelectParams& P, int B, size_t smem, cudaStream_t st);
+cudaError_t launch_candidates(const CandParams& P, int grid, size_t smem, int nch, cudaStream_t st);
+cudaError_t launch_epilogue(const EpilogueParams& P, int B, cudaStream_t st);
+cudaError_t launch_dense(const DenseParams& P, int grid, size_t smem, int nch, cudaStream_t st);
+cudaError_t launch_c2t_check(const C2TCheckParams& P, cudaStream_t st);
+cudaError_t launch_repack_int4(const RepackParams& P, cudaStream_t st);
+
+// Opt-in shared memory attribute for every instantiation (called once per device).
+cudaError_t set_kernel_attributes(int max_smem);
+
+// Register-array width for a hidden size: chunks of 8 elements per lane.
+inline int nch_for(int d) {
+  const int n = (d + 255) / 256;
+  const int sizes[] = {1, 2, 3, 4, 5, 6, 8, 10};
+  for (int s : sizes)
+    if (n <= s) return s;
+  return -1;
+}
+
+}  // namespace fh
