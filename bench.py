@@ -1,0 +1,381 @@
+"""Benchmark of the B200 FlashHead retrieval head.
+
+Default workload (one GPU): the Llama-3.2-1B-shaped head -- v = 128256,
+d = 2048, c = 8016 balanced clusters of b = 16, p = 512 probes, bf16 E and C
+-- decoding one hidden state per step (B = 1, greedy), cycling through 1024
+seeded planted/flat hidden states. A step is one ``fh_decode`` call: centroid
+scores, top-p selection, C2T gather, candidate logits and argmax, all in the
+library's fused kernel. L2 is flushed (a 2 x L2 memset, outside the timed
+events) before every step, so C and E come from HBM each time.
+
+Reported: head tokens/s (whole job, all ranks), us/token, the HBM roofline of
+the fused kernel (algorithmic bytes = centroid bytes + p*b*d*2 + C2T rows + h +
+output), the dense-head kernel on the same E for comparison, an end-to-end
+number through the public API from pinned host memory, SM clocks sampled
+during the timed region, and the fp64 oracle timed on the host cores.
+
+``--impl reference`` times the fp64 CPU oracle on the same workload instead.
+Under torchrun every rank runs its own replica (the head does not shard:
+independent hidden states), timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "Llama-3.2-1B-shaped FlashHead: v128256 d2048 c8016 b16 p512 bf16, B=1 greedy"
+METRIC = "head tokens/s at B=1, p=512 (Llama-3.2-1B-shaped head)"
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+
+
+def algorithmic_bytes(v, d, c, b, p, B=1, crow_bytes=None):
+    """Bytes the method must move per call at batch 1: all centroid rows once,
+    the p*b selected token rows once, their C2T rows, h and the output token."""
+    cb = crow_bytes if crow_bytes is not None else d * 2
+    return c * cb + p * b * d * 2 + p * b * 4 + B * d * 2 + B * 4
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "lm_output_head_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh_:
+            h.update(f.encode())
+            h.update(fh_.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(name):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current kernels."""
+    path = os.path.join(PROFILE_DIR, f"{name}.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons while the benchmark runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 50):
+        self.gpu_index = gpu_index
+        self.period_ms = period_ms
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", f"-lms={self.period_ms}"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+
+    def summary(self, t0, t1):
+        win = [s for t, s in self.samples if t0 <= t <= t1]
+        if not win:  # short timed regions: use everything sampled around them
+            win = [s for _, s in self.samples]
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(s[1]) for s in win if num(s[1]) is not None]
+        mx = [num(s[2]) for s in win if num(s[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in win for i in range(4) if s[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(win)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing
+# ---------------------------------------------------------------------------
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def time_oracle(head, hid, p, budget_s, max_states):
+    import oracle
+    n = 0
+    t0 = time.perf_counter()
+    while n < max_states and (time.perf_counter() - t0) < budget_s:
+        oracle.decode(head, hid.H[n:n + 1], p)
+        n += 1
+    dt = time.perf_counter() - t0
+    return n, dt
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+    world, rank, local = dist_setup()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    import synth
+    import lm_output_head_b200 as fh
+    from lm_output_head_b200 import build as fhbuild
+    fhbuild.build()
+
+    cfg, head, hid, _ = synth.make_config(1)
+    E = fh.bf16_from_bits(head.E, dev)
+    C = fh.bf16_from_bits(head.C, dev)
+    C2T = torch.from_numpy(head.C2T).to(dev)
+    dh = fh.FlashHead(E, C2T, C=C, max_batch=1, max_probes=cfg.p)
+    assert dh.fused_b1, "fused B=1 path unavailable"
+    n_states = hid.H.shape[0]
+    # each rank decodes its own slice of states (replicas; independent rows)
+    Hdev = fh.bf16_from_bits(np.roll(hid.H, -rank * 37, axis=0), dev)
+    out = torch.empty(1, dtype=torch.int32, device=dev)
+
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        dh.decode(Hdev[i % n_states:i % n_states + 1], cfg.p, out_tokens=out, stream=stream)
+
+    def timed_loop(fn, K, W, flush_l2=True):
+        for i in range(W):
+            if flush_l2:
+                flush.zero_()
+            fn(i)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        torch.cuda.synchronize(dev)
+        wall0 = time.time()
+        for i in range(K):
+            if flush_l2:
+                flush.zero_()
+            starts[i].record(stream)
+            fn(W + i)
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+        wall1 = time.time()
+        if world > 1:
+            torch.distributed.barrier()
+        ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+        return ms, wall0, wall1
+
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    time.sleep(0.3)
+    ms, w0, w1 = timed_loop(step, args.steps, args.warmup)
+    status = dh.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed loop")
+    total_ms = sum(ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    mean_ms = total_ms / args.steps
+    value = world * args.steps / (total_ms / 1e3)
+
+    # dense comparison (same protocol, fewer steps)
+    kd = max(3, min(args.steps, 200))
+    dense_out = torch.empty(1, dtype=torch.int32, device=dev)
+    ms_d, _, _ = timed_loop(lambda i: dh.dense_head(Hdev[i % n_states:i % n_states + 1], out_argmax=dense_out,
+                                                    stream=stream), kd, 3)
+    dense_ms = statistics.mean(ms_d)
+
+    # end to end from pinned host memory through the public API
+    host = torch.from_numpy(hid.H.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hd = fh.HostDecoder(dh, 1, cfg.p)
+    ke = max(3, min(args.steps, 500))
+    e2e_ms = []
+    for i in range(ke + 3):
+        flush.zero_()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        hd(host[i % n_states:i % n_states + 1], stream=stream)   # H2D, decode, D2H, synchronize
+        s1.record(stream)
+        s1.synchronize()
+        if i >= 3:
+            e2e_ms.append(s0.elapsed_time(s1))
+    sampler.stop()
+    clocks = sampler.summary(w0, w1)
+
+    if world > 1:
+        torch.distributed.barrier()
+    if rank != 0:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    peak, peak_kind = load_peaks()
+    abytes = algorithmic_bytes(cfg.v, cfg.d, cfg.c, cfg.b, cfg.p)
+    achieved = abytes / (mean_ms * 1e-3) / 1e9
+    dense_bytes = cfg.v * cfg.d * 2 + cfg.d * 2 + 4
+    rec = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(mean_ms, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded planted-cluster head; 75% planted / 25% flat hidden states)",
+        "config": {"workload": WORKLOAD, "global_batch": world, "per_gpu_batch": 1,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed before every step (2 x L2 memset outside the timed events)",
+                   "states": n_states},
+        "us_per_token": round(mean_ms * 1e3, 3),
+        "latency_us": {"p50": round(statistics.median(ms) * 1e3, 3),
+                       "p90": round(float(np.percentile(ms, 90)) * 1e3, 3)},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                     "frac_of_8TBps": round(achieved / 8000.0, 4),
+                     "algorithmic_bytes": abytes, "kernel": "decode_b1_kernel<8,false>",
+                     "traffic": measured_traffic("decode_b1_llama1b")},
+        "dense": {"us_per_token": round(dense_ms * 1e3, 3), "tokens_per_s": round(1e3 / dense_ms, 1),
+                  "achieved_GBps": round(dense_bytes / (dense_ms * 1e-3) / 1e9, 1),
+                  "frac": round(dense_bytes / (dense_ms * 1e-3) / 1e9 / peak, 4),
+                  "speedup_flashhead_vs_dense": round(dense_ms / mean_ms, 3)},
+        "e2e": {"value": round(1e3 / statistics.mean(e2e_ms), 1), "unit": "tokens/s",
+                "us_per_token": round(statistics.mean(e2e_ms) * 1e3, 3),
+                "h2d_bytes_per_step": hd.h2d_bytes, "d2h_bytes_per_step": hd.d2h_bytes},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        n, dt = time_oracle(head, hid, cfg.p, args.cpu_seconds, n_states)
+        rec["cpu_baseline"] = {"value": round(n / dt, 3), "unit": "tokens/s", "cores": oracle_threads(),
+                               "kind": "oracle",
+                               "sample": f"{n} hidden states of the same workload, fp64 numpy oracle, "
+                                         f"{dt:.1f} s"}
+    print(json.dumps(rec), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the fp64 oracle on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return
+    import synth
+    cfg, head, hid, _ = synth.make_config(1)
+    import oracle
+    for i in range(min(args.warmup, 1)):
+        oracle.decode(head, hid.H[i:i + 1], cfg.p)
+    budget = args.cpu_seconds
+    n, dt = time_oracle(head, hid, cfg.p, budget, min(args.steps, hid.H.shape[0]))
+    value = n / dt
+    rec = {
+        "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+        "steps": n, "warmup": min(args.warmup, 1), "ms_per_step": round(dt / n * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded planted-cluster head)",
+        "config": {"workload": WORKLOAD, "global_batch": 1, "parallelism": "host cores"},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": oracle_threads(),
+                         "kind": "oracle",
+                         "sample": f"{n} of the {args.steps} requested steps (one hidden state each) "
+                                   f"within a {budget:.0f} s budget"},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(rec), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

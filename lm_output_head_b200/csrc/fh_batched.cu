@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1) candidates_kernel(const CandParam
   const int n = i0 < total ? static_cast<int>(i1 - i0) : 0;
 
   // tokens of items [32*q, 32*q + 32) of this warp live in lane registers
-  int tq = -1, tcur = 0, tnext = 0;
+  int tq = -2, tcur = 0, tnext = 0;  // -2: no batch loaded yet
   auto tok_batch = [&](int q) -> int {
     const long long it = i0 + 32LL * q + lane;
     return it < i1 ? __ldg(P.cand_tok + it) : 0;
@@ -282,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1) candidates_kernel(const CandParam
     return __shfl_sync(0xFFFFFFFFu, tcur, i & 31);
   };
   // src runs ahead of use by nslot (< 32) items, so keep a separate cursor for it
-  int sq = -1, scur = 0, snext = 0;
+  int sq = -2, scur = 0, snext = 0;
   auto src_token = [&](int i) -> int {
     const int q = i >> 5;
     if (q != sq && q != sq + 1) {

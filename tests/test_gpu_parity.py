@@ -45,6 +45,10 @@ def _to_dev(head, max_batch, max_probes, fh_mod, int4=None):
 
 
 def get_cfg(cfg_id, fh_mod, n_states=None, max_batch=None, max_probes=None):
+    if cfg_id == 0:  # one tiny head serves every tiny-case test (B up to 65, p up to c)
+        n_states, max_batch, max_probes = 65, 65, 256
+    elif cfg_id == 1:
+        max_batch = 8
     key = (cfg_id, n_states, max_batch, max_probes)
     if key not in _HEADS:
         cfg, head, hid, uni = synth.make_config(cfg_id, n_states=n_states)
