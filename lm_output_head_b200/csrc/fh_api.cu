@@ -34,6 +34,8 @@ struct fh_head {
   float* cand_logits = nullptr;        // [max_batch, max_probes * b]
   int32_t* row_ok = nullptr;           // [max_batch]
   uint32_t* c2t_counts = nullptr;      // [v]
+  uint32_t* ghist = nullptr;           // [2, 4096] fused B = 1 key histograms
+  uint32_t* hist = nullptr;            // [max_batch, 4096] batched key histograms
   const uint8_t* crows = nullptr;      // centroid rows (bf16 borrowed, or packed INT4 in ws)
   int crow_bytes = 0;
   int nch = 0;
@@ -52,6 +54,7 @@ inline size_t up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct B1MiscSize {
+  unsigned long long hbar;
   unsigned long long wbest[kWarps];
   float scan[kWarps + 1];
   int claim, lastpos, ok, last;
@@ -89,7 +92,7 @@ int ring_slots(size_t budget, size_t fixed, size_t slot) {
 }
 
 fh_status launch_scores_rows(fh_head* h, const void* hidden, int32_t B, int mode, float T,
-                             const float* u, float* out, cudaStream_t st) {
+                             const float* u, float* out, uint32_t* hist, cudaStream_t st) {
   const fh_head_desc& D = h->desc;
   const size_t slot = up(static_cast<size_t>(h->crow_bytes), 128);
   const int nslot = 2;
@@ -105,6 +108,7 @@ fh_status launch_scores_rows(fh_head* h, const void* hidden, int32_t B, int mode
     P.hidden = static_cast<const uint16_t*>(hidden);
     P.u_clusters = u;
     P.out = out;
+    P.hist = hist;
     P.status = &h->sync->status;
     P.d = D.d;
     P.c = D.c;
@@ -155,7 +159,7 @@ fh_status launch_candidates_rows(fh_head* h, const void* hidden, int32_t B, int3
 }
 
 size_t select_smem(const fh_head* h, int32_t p) {
-  return up(static_cast<size_t>(h->desc.c) * 4, 128) + up(static_cast<size_t>(p) * 4, 128) + sizeof(SelectSmem);
+  return up(static_cast<size_t>(p) * 4, 128) + hist_select_smem_bytes(h->desc.c);
 }
 
 }  // namespace
@@ -233,6 +237,8 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   const size_t o_log = take(mb * nc * 4);
   const size_t o_rok = take(mb * 4);
   const size_t o_cnt = take(static_cast<size_t>(D.v) * 4);
+  const size_t o_ghist = take(2 * kHistBins * 4);
+  const size_t o_hist = take(mb * kHistBins * 4);
   const size_t o_crow = D.fmt == FH_CENTROID_INT4_G32 ? take(static_cast<size_t>(D.c) * h->crow_bytes) : 0;
   h->ws_bytes = off;
 
@@ -254,6 +260,8 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   h->cand_logits = reinterpret_cast<float*>(h->ws + o_log);
   h->row_ok = reinterpret_cast<int32_t*>(h->ws + o_rok);
   h->c2t_counts = reinterpret_cast<uint32_t*>(h->ws + o_cnt);
+  h->ghist = reinterpret_cast<uint32_t*>(h->ws + o_ghist);
+  h->hist = reinterpret_cast<uint32_t*>(h->ws + o_hist);
   h->crows = D.fmt == FH_CENTROID_INT4_G32 ? h->ws + o_crow : static_cast<const uint8_t*>(D.C);
 
   fh_status status = FH_OK;
@@ -310,7 +318,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
     h->b1_off_ring = static_cast<int>(o);
     const int nslot = ring_slots(h->smem_budget, o, slot);
     const size_t ring = static_cast<size_t>(kWarps) * nslot * slot;
-    const size_t sel_scratch = up(static_cast<size_t>(D.c) * 4, 128) + sizeof(SelectSmem);
+    const size_t sel_scratch = hist_select_smem_bytes(D.c);
     h->b1_nslot = nslot;
     h->b1_slot = static_cast<int>(slot);
     h->b1_smem = o + ring;
@@ -376,7 +384,7 @@ fh_status fh_centroid_scores(fh_head* h, const void* hidden, int32_t B, float* s
   fh_status s = check_call(h, hidden, B);
   if (s != FH_OK) return s;
   if (!scores || !aligned(scores, 4)) return FH_ERR_INVALID_ARG;
-  return launch_scores_rows(h, hidden, B, 0, 1.f, nullptr, scores, reinterpret_cast<cudaStream_t>(stream));
+  return launch_scores_rows(h, hidden, B, 0, 1.f, nullptr, scores, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
 fh_status fh_select_clusters(fh_head* h, const float* scores, int32_t B, int32_t p, int32_t mode, float T,
@@ -454,6 +462,7 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
     P.out_max_logit = out_max_logit;
     P.scores = h->keys;
     P.cand_logits = h->cand_logits;
+    P.ghist = h->ghist;
     P.best = h->best;
     P.sync = h->sync;
     P.v = D.v;
@@ -477,10 +486,11 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
   }
 
   // batched path: keys -> per-row select -> candidates -> epilogue
-  s = launch_scores_rows(h, hidden, B, gumbel ? 1 : 0, gumbel ? T : 1.f, u_clusters, h->keys, st);
+  s = launch_scores_rows(h, hidden, B, gumbel ? 1 : 0, gumbel ? T : 1.f, u_clusters, h->keys, h->hist, st);
   if (s != FH_OK) return s;
   SelectParams SP{};
   SP.in = h->keys;
+  SP.hist = h->hist;
   SP.C2T = D.C2T;
   SP.sel = h->sel;
   SP.cand_tok = h->cand_tok;

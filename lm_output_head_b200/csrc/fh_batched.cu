@@ -38,8 +38,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_kernel(const ScoresParams 
 
   const uint4* hsrc = reinterpret_cast<const uint4*>(P.hidden + static_cast<size_t>(P.row0) * d);
   for (int i = tid; i < R * d / 8; i += kThreads) reinterpret_cast<uint4*>(sh)[i] = hsrc[i];
-  if (lane < P.nslot) mbar_init(bar_w + 8u * lane, 1);
-  fence_mbar_init();
+  warp_ring_init(bar_w, P.nslot);
   __syncthreads();
 
   const int n = gw < P.c ? (P.c - 1 - gw) / W + 1 : 0;
@@ -50,7 +49,9 @@ __global__ void __launch_bounds__(kThreads, 1) scores_kernel(const ScoresParams 
   };
   auto emit = [&](int r, int k, float s) {
     const size_t o = static_cast<size_t>(P.row0 + r) * P.c + k;
-    P.out[o] = P.mode == 1 ? gumbel_key(s, P.T, __ldg(P.u_clusters + o)) : s;
+    const float key = P.mode == 1 ? gumbel_key(s, P.T, __ldg(P.u_clusters + o)) : s;
+    P.out[o] = key;
+    if (P.hist) atomicAdd(P.hist + static_cast<size_t>(P.row0 + r) * kHistBins + (f2key(key) >> kHistShift), 1u);
   };
   bool ok;
   if constexpr (INT4) {
@@ -147,20 +148,14 @@ __device__ void write_candidates(const SelectParams& P, const int32_t* ssel, int
 __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelectParams P) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int row = blockIdx.x;
-  uint32_t* skey = reinterpret_cast<uint32_t*>(smem);
-  const size_t key_bytes = (static_cast<size_t>(P.c) * 4 + 127) & ~size_t(127);
-  int32_t* ssel = reinterpret_cast<int32_t*>(smem + key_bytes);
-  const size_t sel_bytes = (static_cast<size_t>(P.p) * 4 + 127) & ~size_t(127);
-  SelectSmem* ssm = reinterpret_cast<SelectSmem*>(smem + key_bytes + sel_bytes);
+  int32_t* ssel = reinterpret_cast<int32_t*>(smem);
+  uint8_t* scratch = smem + ((static_cast<size_t>(P.p) * 4 + 127) & ~size_t(127));
   const float* in = P.in + static_cast<size_t>(row) * P.c;
-  const float* u = P.u_clusters ? P.u_clusters + static_cast<size_t>(row) * P.c : nullptr;
-  for (int k = threadIdx.x; k < P.c; k += kThreads) {
-    float key = in[k];
-    if (P.perturb) key = gumbel_key(key, P.T, u[k]);
-    skey[k] = f2key(key);
-  }
-  __syncthreads();
-  block_select_top_p(skey, P.c, P.p, ssel, *ssm);
+  const float* u = P.perturb ? P.u_clusters + static_cast<size_t>(row) * P.c : nullptr;
+  uint32_t* hist = P.hist ? P.hist + static_cast<size_t>(row) * kHistBins : nullptr;
+  select_top_p_hist(in, u, P.T, P.c, P.p, hist, ssel, scratch);
+  if (hist)  // consumed: clear it for the next call
+    for (int i = threadIdx.x; i < kHistBins; i += kThreads) hist[i] = 0u;
   int32_t* gsel = P.sel + static_cast<size_t>(row) * P.p;
   for (int i = threadIdx.x; i < P.p; i += kThreads) gsel[i] = ssel[i];
   write_candidates(P, ssel, row);
@@ -251,8 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1) candidates_kernel(const CandParam
   const int d = P.d;
   const uint32_t ring_w = smem_addr(smem + P.off_ring) + static_cast<uint32_t>(warp * P.nslot * P.slot_bytes);
   const uint32_t bar_w = smem_addr(smem + P.off_bar) + static_cast<uint32_t>(warp * P.nslot * 8);
-  if (lane < P.nslot) mbar_init(bar_w + 8u * lane, 1);
-  fence_mbar_init();
+  warp_ring_init(bar_w, P.nslot);
   __syncthreads();
 
   // contiguous item range per warp: item = row * nc + r

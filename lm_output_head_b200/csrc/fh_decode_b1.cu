@@ -31,6 +31,7 @@ namespace fh {
 namespace {
 
 struct B1Misc {
+  unsigned long long hbar;
   unsigned long long wbest[kWarps];
   float scan[kWarps + 1];
   int claim, lastpos, ok, last;
@@ -75,25 +76,46 @@ __global__ void __launch_bounds__(kThreads, 1) decode_b1_kernel(const B1Params P
   const uint32_t ring_w = smem_addr(ring) + static_cast<uint32_t>(warp * P.nslot * P.slot_bytes);
   const uint32_t bar_w = smem_addr(smem + P.off_bar) + static_cast<uint32_t>(warp * P.nslot * 8);
 
-  for (int i = tid; i < d / 8; i += kThreads)
-    reinterpret_cast<uint4*>(sh)[i] = reinterpret_cast<const uint4*>(P.hidden)[i];
-  if (lane < P.nslot) mbar_init(bar_w + 8u * lane, 1);
-  fence_mbar_init();
-  __syncthreads();
-
   uint32_t phase_bits = 0;
   bool ok = true;
   const bool gumbel = P.mode == 1;
+  // histogram of this call's keys, and the other buffer to clear for the next call
+  const uint32_t epoch = P.sync->epoch;
+  uint32_t* hist_cur = P.ghist + (epoch & 1u) * kHistBins;
+  uint32_t* hist_next = P.ghist + ((epoch + 1u) & 1u) * kHistBins;
 
   // ---------------- phase 1: centroid scores ----------------
+  // h is staged by the first bulk copy of the CTA; the centroid rows follow
+  // at once (they do not depend on h).
+  const uint32_t hbar = smem_addr(&misc->hbar);
+  if (tid == 0) {
+    mbar_init(hbar, 1);
+    fence_mbar_init();
+    mbar_expect_tx(hbar, static_cast<uint32_t>(d * 2));
+    bulk_g2s(smem_addr(sh), P.hidden, static_cast<uint32_t>(d * 2), hbar);
+  }
+  warp_ring_init(bar_w, P.nslot);
+  const int n1 = gw < P.c ? (P.c - 1 - gw) / W + 1 : 0;
+  auto src1 = [&](int i, const void*& ptr, uint32_t& bytes) {
+    ptr = P.Crows + static_cast<size_t>(gw + i * W) * P.crow_bytes;
+    bytes = static_cast<uint32_t>(P.crow_bytes);
+  };
+  warp_stream_prologue(n1, P.nslot, ring_w, P.slot_bytes, bar_w, src1);
+  float ureg = 0.f;  // lane j holds u of item j (j < 32)
+  if (gumbel && lane < n1) ureg = __ldg(P.u_clusters + gw + lane * W);
   {
-    const int n1 = gw < P.c ? (P.c - 1 - gw) / W + 1 : 0;
-    float ureg = 0.f;  // lane j holds u of item j (j < 32)
-    if (gumbel && lane < n1) ureg = __ldg(P.u_clusters + gw + lane * W);
-    auto src = [&](int i, const void*& ptr, uint32_t& bytes) {
-      ptr = P.Crows + static_cast<size_t>(gw + i * W) * P.crow_bytes;
-      bytes = static_cast<uint32_t>(P.crow_bytes);
-    };
+    const int per = (kHistBins + G - 1) / G;
+    for (int i = tid; i < per; i += kThreads) {
+      const int b = blockIdx.x * per + i;
+      if (b < kHistBins) hist_next[b] = 0u;
+    }
+  }
+  __syncthreads();  // hbar initialised before anyone waits on it
+  if (!mbar_wait_bounded(hbar, 0u, kWaitBudget)) {
+    ok = false;
+    if (lane == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
+  }
+  {
     if constexpr (INT4) {
       constexpr int NQ = (NCH + 1) / 2;
       float hq[NQ * 16];
@@ -106,10 +128,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_b1_kernel(const B1Params P
           float key = s;
           if (gumbel) key = gumbel_key(s, P.T, i < 32 ? u : __ldg(P.u_clusters + k));
           P.scores[k] = key;
+          atomicAdd(hist_cur + (f2key(key) >> kHistShift), 1u);
           prefetch_l2(P.C2T + static_cast<size_t>(k) * P.b);
         }
       };
-      ok = warp_stream(n1, P.nslot, ring_w, P.slot_bytes, bar_w, phase_bits, kWaitBudget, src, use);
+      ok = warp_stream_run(n1, P.nslot, ring_w, P.slot_bytes, bar_w, phase_bits, kWaitBudget, src1, use);
     } else {
       float hr[NCH * 8];
       load_h_chunks<NCH>(sh, d, hr);
@@ -121,10 +144,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_b1_kernel(const B1Params P
           float key = s;
           if (gumbel) key = gumbel_key(s, P.T, i < 32 ? u : __ldg(P.u_clusters + k));
           P.scores[k] = key;
+          atomicAdd(hist_cur + (f2key(key) >> kHistShift), 1u);
           prefetch_l2(P.C2T + static_cast<size_t>(k) * P.b);
         }
       };
-      ok = warp_stream(n1, P.nslot, ring_w, P.slot_bytes, bar_w, phase_bits, kWaitBudget, src, use);
+      ok = warp_stream_run(n1, P.nslot, ring_w, P.slot_bytes, bar_w, phase_bits, kWaitBudget, src1, use);
     }
     if (!ok && lane == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
   }
@@ -134,11 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_b1_kernel(const B1Params P
   if (!passed) {
     if (tid == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
   } else {
-    uint32_t* skey = reinterpret_cast<uint32_t*>(ring);
-    SelectSmem* ssm = reinterpret_cast<SelectSmem*>(ring + ((static_cast<size_t>(P.c) * 4 + 127) & ~size_t(127)));
-    for (int k = tid; k < P.c; k += kThreads) skey[k] = f2key(__ldcg(P.scores + k));
-    __syncthreads();
-    block_select_top_p(skey, P.c, P.p, ssel, *ssm);
+    select_top_p_hist(P.scores, nullptr, 1.f, P.c, P.p, hist_cur, ssel, ring);
     if (blockIdx.x == 0 && P.out_cluster_ids)
       for (int i = tid; i < P.p; i += kThreads) P.out_cluster_ids[i] = ssel[i];
     fence_proxy_async_smem();  // generic writes to the ring before the next bulk copies
@@ -246,6 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_b1_kernel(const B1Params P
     *P.best = 0ull;
     P.sync->arrive = 0u;
     P.sync->ticket = 0u;
+    P.sync->epoch = epoch + 1u;
     __threadfence();
   }
 }

@@ -28,19 +28,19 @@ __global__ void __launch_bounds__(kThreads, 1) dense_kernel(const DenseParams P)
   const uint32_t ring_w = smem_addr(smem + P.off_ring) + static_cast<uint32_t>(warp * P.nslot * P.slot_bytes);
   const uint32_t bar_w = smem_addr(smem + P.off_bar) + static_cast<uint32_t>(warp * P.nslot * 8);
 
-  const uint4* hsrc = reinterpret_cast<const uint4*>(P.hidden + static_cast<size_t>(P.row0) * d);
-  for (int i = tid; i < R * d / 8; i += kThreads) reinterpret_cast<uint4*>(sh)[i] = hsrc[i];
-  for (int i = tid; i < kWarps * kDenseMaxRows; i += kThreads) (&wbest[0][0])[i] = 0ull;
-  if (lane < P.nslot) mbar_init(bar_w + 8u * lane, 1);
-  fence_mbar_init();
-  __syncthreads();
-
   const int n = gw < P.v ? (P.v - 1 - gw) / W + 1 : 0;
   uint32_t phase_bits = 0;
   auto src = [&](int i, const void*& ptr, uint32_t& bytes) {
     ptr = P.E + static_cast<size_t>(gw + i * W) * d;
     bytes = static_cast<uint32_t>(d * 2);
   };
+  // first copies go out before the hidden rows are staged
+  warp_ring_init(bar_w, P.nslot);
+  warp_stream_prologue(n, P.nslot, ring_w, P.slot_bytes, bar_w, src);
+  const uint4* hsrc = reinterpret_cast<const uint4*>(P.hidden + static_cast<size_t>(P.row0) * d);
+  for (int i = tid; i < R * d / 8; i += kThreads) reinterpret_cast<uint4*>(sh)[i] = hsrc[i];
+  for (int i = tid; i < kWarps * kDenseMaxRows; i += kThreads) (&wbest[0][0])[i] = 0ull;
+  __syncthreads();
   bool ok;
   if constexpr (ONE) {
     float hr[NCH * 8];
@@ -53,7 +53,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_kernel(const DenseParams P)
       best = pk > best ? pk : best;
       if (lane == 0 && P.logits) P.logits[static_cast<size_t>(P.row0) * P.v + t] = z;
     };
-    ok = warp_stream(n, P.nslot, ring_w, P.slot_bytes, bar_w, phase_bits, kWaitBudget, src, use);
+    ok = warp_stream_run(n, P.nslot, ring_w, P.slot_bytes, bar_w, phase_bits, kWaitBudget, src, use);
     if (lane == 0) wbest[warp][0] = best;
   } else {
     auto use = [&](int i, uint32_t slot) {
@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_kernel(const DenseParams P)
         }
       }
     };
-    ok = warp_stream(n, P.nslot, ring_w, P.slot_bytes, bar_w, phase_bits, kWaitBudget, src, use);
+    ok = warp_stream_run(n, P.nslot, ring_w, P.slot_bytes, bar_w, phase_bits, kWaitBudget, src, use);
   }
   if (!ok && lane == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
   __syncthreads();

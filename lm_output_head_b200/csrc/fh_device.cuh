@@ -342,19 +342,203 @@ __device__ inline void block_select_top_p(const uint32_t* skey, int n, int p, in
 }
 
 // ---------------------------------------------------------------------------
+// histogram-driven top-p select
+// ---------------------------------------------------------------------------
+// A 4096-bin histogram of the top 12 key bits (sign, exponent, 3 mantissa
+// bits) locates the bin holding the p-th largest key; every key above that
+// bin is taken, and the keys inside it are ranked exactly (key desc, id asc)
+// against each other -- a few hundred at most for real score distributions,
+// so the exact step is a small all-pairs count rather than more radix passes.
+// The histogram either arrives precomputed in global memory (built with
+// fire-and-forget atomics by the kernel that produced the scores) or is
+// built here in shared memory.
+constexpr int kHistBins = 4096;
+constexpr int kHistShift = 20;
+constexpr int kKeysPerThreadMax = 32;          // keys held in registers: c <= 16384
+constexpr int kBoundaryMax = 2048;              // exact all-pairs ranking up to this many ties-in-bin
+
+struct HistSelectSmem {
+  uint32_t hist[kHistBins];
+  uint32_t ckey[kBoundaryMax];
+  int32_t cid[kBoundaryMax];
+  uint32_t scan[kWarps + 1];
+  uint32_t wcount[kWarps];
+  uint32_t t1, above, m1, ncand;
+};
+
+// Bytes of shared scratch the select needs for c keys: the struct, a c-byte
+// flag array, and c keys for the radix fallback.
+__host__ __device__ inline size_t hist_select_smem_bytes(int c) {
+  return ((sizeof(HistSelectSmem) + 127) & ~size_t(127)) + ((static_cast<size_t>(c) + 127) & ~size_t(127)) +
+         ((static_cast<size_t>(c) * 4 + 127) & ~size_t(127)) + sizeof(SelectSmem);
+}
+
+// Top-p of the c keys derived from `scores` (global, read through L2):
+// key = scores[k], or the Gumbel key scores[k]/T - ln(-ln u[k]) when u != null.
+// `hist_g` (global, 4096 bins of key >> 20) may be null. Writes the chosen
+// ids in ascending order to `sel`. All kThreads threads must call it.
+__device__ inline void select_top_p_hist(const float* scores, const float* u, float T, int c, int p,
+                                         const uint32_t* hist_g, int32_t* sel, uint8_t* scratch) {
+  HistSelectSmem& sm = *reinterpret_cast<HistSelectSmem*>(scratch);
+  uint8_t* flag = scratch + ((sizeof(HistSelectSmem) + 127) & ~size_t(127));
+  uint32_t* skey = reinterpret_cast<uint32_t*>(flag + ((static_cast<size_t>(c) + 127) & ~size_t(127)));
+  SelectSmem* fsm = reinterpret_cast<SelectSmem*>(reinterpret_cast<uint8_t*>(skey) +
+                                                   ((static_cast<size_t>(c) * 4 + 127) & ~size_t(127)));
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+
+  if (c > kWarps * 32 * kKeysPerThreadMax) {  // too many keys for registers: radix select in smem
+    for (int k = tid; k < c; k += kThreads)
+      skey[k] = f2key(u ? gumbel_key(__ldcg(scores + k), T, __ldcg(u + k)) : __ldcg(scores + k));
+    __syncthreads();
+    block_select_top_p(skey, c, p, sel, *fsm);
+    return;
+  }
+
+  // keys in registers, warp-block layout: warp w holds ids [w*kpt*32, (w+1)*kpt*32)
+  const int kpt = (c + kWarps * 32 - 1) / (kWarps * 32);
+  const int wbase = warp * kpt * 32;
+  uint32_t key[kKeysPerThreadMax];
+#pragma unroll
+  for (int i = 0; i < kKeysPerThreadMax; ++i) {
+    const int id = wbase + i * 32 + lane;
+    float v = 0.f;
+    if (i < kpt && id < c) {
+      v = __ldcg(scores + id);
+      if (u) v = gumbel_key(v, T, __ldcg(u + id));
+    }
+    key[i] = f2key(v);
+  }
+  for (int i = tid; i < (c + 15) / 16; i += kThreads) reinterpret_cast<uint4*>(flag)[i] = make_uint4(0, 0, 0, 0);
+  if (hist_g == nullptr) {
+    for (int i = tid; i < kHistBins; i += kThreads) sm.hist[i] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kKeysPerThreadMax; ++i) {
+      const int id = wbase + i * 32 + lane;
+      if (i < kpt && id < c) atomicAdd(&sm.hist[key[i] >> kHistShift], 1u);
+    }
+  } else {
+    for (int i = tid; i < kHistBins; i += kThreads) sm.hist[i] = __ldcg(hist_g + i);
+  }
+  if (tid == 0) sm.ncand = 0u;
+  __syncthreads();
+
+  // bin t1 holding the p-th largest key: thread t owns bins 4095-8t .. 4088-8t
+  constexpr int kBpt = kHistBins / kThreads;
+  uint32_t loc = 0;
+#pragma unroll
+  for (int i = 0; i < kBpt; ++i) loc += sm.hist[kHistBins - 1 - kBpt * tid - i];
+  const uint32_t above = block_exclusive_scan<kThreads, uint32_t>(loc, sm.scan, nullptr);
+  uint32_t run = above;
+#pragma unroll
+  for (int i = 0; i < kBpt; ++i) {
+    const int b = kHistBins - 1 - kBpt * tid - i;
+    const uint32_t h = sm.hist[b];
+    if (run < static_cast<uint32_t>(p) && run + h >= static_cast<uint32_t>(p)) {
+      sm.t1 = static_cast<uint32_t>(b);
+      sm.above = run;
+      sm.m1 = h;
+    }
+    run += h;
+  }
+  __syncthreads();
+  const uint32_t t1 = sm.t1, m1 = sm.m1;
+  const uint32_t need = static_cast<uint32_t>(p) - sm.above;
+  const bool all_in_bin = (m1 == need);
+
+  if (!all_in_bin && m1 > static_cast<uint32_t>(kBoundaryMax)) {  // pathological ties: radix fallback
+#pragma unroll
+    for (int i = 0; i < kKeysPerThreadMax; ++i) {
+      const int id = wbase + i * 32 + lane;
+      if (i < kpt && id < c) skey[id] = key[i];
+    }
+    __syncthreads();
+    block_select_top_p(skey, c, p, sel, *fsm);
+    return;
+  }
+  if (!all_in_bin) {
+    // gather the boundary bin, rank it exactly, flag the chosen ids
+#pragma unroll
+    for (int i = 0; i < kKeysPerThreadMax; ++i) {
+      const int id = wbase + i * 32 + lane;
+      const bool in = i < kpt && id < c && (key[i] >> kHistShift) == t1;
+      const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
+      if (m) {
+        uint32_t base = 0;
+        if (lane == 0) base = atomicAdd(&sm.ncand, static_cast<uint32_t>(__popc(m)));
+        base = __shfl_sync(0xFFFFFFFFu, base, 0);
+        const uint32_t at = base + __popc(m & lt_mask);
+        if (in && at < static_cast<uint32_t>(kBoundaryMax)) {
+          sm.ckey[at] = key[i];
+          sm.cid[at] = id;
+        }
+      }
+    }
+    __syncthreads();
+    const uint32_t nb = min(sm.ncand, static_cast<uint32_t>(kBoundaryMax));  // == m1 for a consistent histogram
+    for (uint32_t a = tid; a < nb; a += kThreads) {
+      const uint32_t ka = sm.ckey[a];
+      const int ia = sm.cid[a];
+      uint32_t r = 0;
+      for (uint32_t b = 0; b < nb; ++b) {
+        const uint32_t kb = sm.ckey[b];
+        r += (kb > ka) || (kb == ka && sm.cid[b] < ia);
+      }
+      if (r < need) flag[ia] = 1;
+    }
+    __syncthreads();
+  }
+
+  // ascending-id compaction with ballots
+  uint32_t cnt = 0;
+#pragma unroll
+  for (int i = 0; i < kKeysPerThreadMax; ++i) {
+    const int id = wbase + i * 32 + lane;
+    const uint32_t dg = key[i] >> kHistShift;
+    const bool take = i < kpt && id < c && (dg > t1 || (dg == t1 && (all_in_bin || flag[id])));
+    cnt += __popc(__ballot_sync(0xFFFFFFFFu, take));
+  }
+  if (lane == 0) sm.wcount[warp] = cnt;
+  __syncthreads();
+  uint32_t pos = 0;
+  for (int w = 0; w < warp; ++w) pos += sm.wcount[w];
+#pragma unroll
+  for (int i = 0; i < kKeysPerThreadMax; ++i) {
+    const int id = wbase + i * 32 + lane;
+    const uint32_t dg = key[i] >> kHistShift;
+    const bool take = i < kpt && id < c && (dg > t1 || (dg == t1 && (all_in_bin || flag[id])));
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, take);
+    const uint32_t at = pos + __popc(m & lt_mask);
+    if (take && at < static_cast<uint32_t>(p)) sel[at] = id;
+    pos += __popc(m);
+  }
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
 // per-warp streaming of rows through a ring of shared-memory slots
 // ---------------------------------------------------------------------------
 // Each warp owns `nslot` slots of `slot_bytes` and one mbarrier per slot.
 // Item i of the warp's n items is copied by one cp.async.bulk into slot
 // i % nslot; lane 0 issues, all lanes wait, `use(i, slot_addr)` consumes, and
 // the slot is refilled with item i + nslot. `src(i, ptr, bytes)` is evaluated
-// by all lanes (it may shuffle prefetched ids). A wait that exceeds `budget`
+// by all lanes (it may shuffle prefetched ids). The first min(n, nslot)
+// copies can be issued early (warp_stream_prologue) so that they overlap
+// whatever the warp does before consuming. A wait that exceeds `budget`
 // cycles makes the warp wait (bounded) for its copies still in flight and
 // return false.
-template <class Src, class Use>
-__device__ __forceinline__ bool warp_stream(int n, int nslot, uint32_t ring, uint32_t slot_bytes,
-                                            uint32_t bars, uint32_t& phase_bits, long long budget,
-                                            Src src, Use use) {
+__device__ __forceinline__ void warp_ring_init(uint32_t bars, int nslot) {
+  if ((threadIdx.x & 31) == 0) {
+    for (int s = 0; s < nslot; ++s) mbar_init(bars + 8u * s, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+}
+
+template <class Src>
+__device__ __forceinline__ void warp_stream_prologue(int n, int nslot, uint32_t ring, uint32_t slot_bytes,
+                                                     uint32_t bars, Src src) {
   const int lane = threadIdx.x & 31;
   const int pre = n < nslot ? n : nslot;
   for (int s = 0; s < pre; ++s) {
@@ -366,6 +550,13 @@ __device__ __forceinline__ bool warp_stream(int n, int nslot, uint32_t ring, uin
       bulk_g2s(ring + s * slot_bytes, ptr, bytes, bars + 8u * s);
     }
   }
+}
+
+template <class Src, class Use>
+__device__ __forceinline__ bool warp_stream_run(int n, int nslot, uint32_t ring, uint32_t slot_bytes,
+                                                uint32_t bars, uint32_t& phase_bits, long long budget,
+                                                Src src, Use use) {
+  const int lane = threadIdx.x & 31;
   for (int i = 0; i < n; ++i) {
     const int s = i % nslot;
     const uint32_t bar = bars + 8u * s;
@@ -394,6 +585,34 @@ __device__ __forceinline__ bool warp_stream(int n, int nslot, uint32_t ring, uin
     }
   }
   return true;
+}
+
+template <class Src, class Use>
+__device__ __forceinline__ bool warp_stream(int n, int nslot, uint32_t ring, uint32_t slot_bytes,
+                                            uint32_t bars, uint32_t& phase_bits, long long budget,
+                                            Src src, Use use) {
+  warp_stream_prologue(n, nslot, ring, slot_bytes, bars, src);
+  return warp_stream_run(n, nslot, ring, slot_bytes, bars, phase_bits, budget, src, use);
+}
+
+// Load n fp32 values from global memory (L2, bypassing L1) and store their
+// order-preserving keys to shared memory; 16 loads per thread are in flight
+// together instead of one L2 round trip per element.
+__device__ __forceinline__ void load_keys_l2(const float* src, int n, uint32_t* skey) {
+  constexpr int KPT = 16;
+  for (int base = 0; base < n; base += KPT * kThreads) {
+    float v[KPT];
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+      const int k = base + j * kThreads + threadIdx.x;
+      v[j] = k < n ? __ldcg(src + k) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+      const int k = base + j * kThreads + threadIdx.x;
+      if (k < n) skey[k] = f2key(v[j]);
+    }
+  }
 }
 
 // Load this lane's slice of a bf16 vector into fp32 registers in the layout

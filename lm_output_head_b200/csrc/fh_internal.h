@@ -21,7 +21,8 @@ struct SyncWords {
   uint32_t arrive;        // grid barrier arrivals
   uint32_t ticket;        // kernel exit tickets (last CTA finalises)
   uint32_t union_count;   // distinct clusters of the last batched decode
-  uint32_t pad[4];
+  uint32_t epoch;         // fused B = 1 calls so far (selects the histogram buffer)
+  uint32_t pad[3];
 };
 
 struct B1Params {
@@ -36,6 +37,7 @@ struct B1Params {
   float* out_max_logit;
   float* scores;          // workspace [c]
   float* cand_logits;     // workspace [p*b]
+  uint32_t* ghist;        // workspace [2][4096] key histograms, used by alternate calls
   unsigned long long* best;
   SyncWords* sync;
   int v, d, c, b, p;
@@ -52,6 +54,7 @@ struct ScoresParams {
   const uint16_t* hidden;  // [B, d]
   const float* u_clusters; // [B, c] (gumbel)
   float* out;              // [B, c]
+  uint32_t* hist;          // [B, 4096] key histograms (accumulated), or null
   int*  status;
   int d, c, crow_bytes;
   int row0, rows;          // hidden rows [row0, row0+rows) in this launch
@@ -63,6 +66,7 @@ struct ScoresParams {
 
 struct SelectParams {
   const float* in;         // [B, c] scores or keys
+  uint32_t* hist;          // [B, 4096] key histograms of `in` (cleared after use), or null
   const float* u_clusters; // [B, c] when perturb
   const int32_t* ids_in;   // [B, p] explicit ids (sort mode) or null
   const int32_t* C2T;
