@@ -15,6 +15,7 @@ cudaError_t set_attrs_batched(int max_smem);
 cudaError_t set_attrs_dense(int max_smem);
 int dense_max_rows();
 cudaError_t occupancy_decode_b1(int int4, int nch, size_t smem, int* blocks);
+size_t decode_b1_misc_bytes();
 }  // namespace fh
 
 using namespace fh;
@@ -34,7 +35,13 @@ struct fh_head {
   float* cand_logits = nullptr;        // [max_batch, max_probes * b]
   int32_t* row_ok = nullptr;           // [max_batch]
   uint32_t* c2t_counts = nullptr;      // [v]
-  uint32_t* ghist = nullptr;           // [2, 4096] fused B = 1 key histograms
+  uint32_t* b1_hist_hi = nullptr;      // fused B = 1 per-call state (two buffers each)
+  uint32_t* b1_hist_lo = nullptr;
+  uint32_t* b1_bitmap = nullptr;
+  unsigned long long* b1_bnd = nullptr;
+  uint32_t* b1_bnd_count = nullptr;
+  float* z_slot = nullptr;             // [v]
+  int words = 0;
   uint32_t* hist = nullptr;            // [max_batch, 4096] batched key histograms
   const uint8_t* crows = nullptr;      // centroid rows (bf16 borrowed, or packed INT4 in ws)
   int crow_bytes = 0;
@@ -53,12 +60,6 @@ constexpr size_t kAlign = 256;
 inline size_t up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-struct B1MiscSize {
-  unsigned long long hbar;
-  unsigned long long wbest[kWarps];
-  float scan[kWarps + 1];
-  int claim, lastpos, ok, last;
-};
 
 std::mutex g_attr_mu;
 bool g_attr_done[64] = {};
@@ -237,7 +238,13 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   const size_t o_log = take(mb * nc * 4);
   const size_t o_rok = take(mb * 4);
   const size_t o_cnt = take(static_cast<size_t>(D.v) * 4);
-  const size_t o_ghist = take(2 * kHistBins * 4);
+  const int words = (D.c + 31) / 32;
+  const size_t o_hhi = take(2 * 256 * 4);
+  const size_t o_hlo = take(2 * kHistBins * 4);
+  const size_t o_bmp = take(2 * static_cast<size_t>(words) * 4);
+  const size_t o_bnd = take(2 * kBoundaryMax * 8);
+  const size_t o_bnc = take(2 * 4);
+  const size_t o_zs = take(static_cast<size_t>(D.v) * 4);
   const size_t o_hist = take(mb * kHistBins * 4);
   const size_t o_crow = D.fmt == FH_CENTROID_INT4_G32 ? take(static_cast<size_t>(D.c) * h->crow_bytes) : 0;
   h->ws_bytes = off;
@@ -260,7 +267,13 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   h->cand_logits = reinterpret_cast<float*>(h->ws + o_log);
   h->row_ok = reinterpret_cast<int32_t*>(h->ws + o_rok);
   h->c2t_counts = reinterpret_cast<uint32_t*>(h->ws + o_cnt);
-  h->ghist = reinterpret_cast<uint32_t*>(h->ws + o_ghist);
+  h->b1_hist_hi = reinterpret_cast<uint32_t*>(h->ws + o_hhi);
+  h->b1_hist_lo = reinterpret_cast<uint32_t*>(h->ws + o_hlo);
+  h->b1_bitmap = reinterpret_cast<uint32_t*>(h->ws + o_bmp);
+  h->b1_bnd = reinterpret_cast<unsigned long long*>(h->ws + o_bnd);
+  h->b1_bnd_count = reinterpret_cast<uint32_t*>(h->ws + o_bnc);
+  h->z_slot = reinterpret_cast<float*>(h->ws + o_zs);
+  h->words = words;
   h->hist = reinterpret_cast<uint32_t*>(h->ws + o_hist);
   h->crows = D.fmt == FH_CENTROID_INT4_G32 ? h->ws + o_crow : static_cast<const uint8_t*>(D.C);
 
@@ -313,7 +326,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
     h->b1_off_sel = static_cast<int>(o);
     o += up(static_cast<size_t>(D.max_probes) * 4, 128);
     h->b1_off_misc = static_cast<int>(o);
-    o += up(sizeof(B1MiscSize), 128);
+    o += up(decode_b1_misc_bytes(), 128);
     o = up(o, 1024);
     h->b1_off_ring = static_cast<int>(o);
     const int nslot = ring_slots(h->smem_budget, o, slot);
@@ -322,7 +335,10 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
     h->b1_nslot = nslot;
     h->b1_slot = static_cast<int>(slot);
     h->b1_smem = o + ring;
-    h->fused_ok = nslot >= 2 && sel_scratch <= ring;
+    // each warp owns at most 32 clusters (one per lane register)
+    const long long warps = static_cast<long long>(h->num_sms) * kWarps;
+    h->fused_ok = nslot >= 2 && sel_scratch <= ring && D.c <= 32 * warps &&
+                  static_cast<size_t>(kBoundaryMax) * 8 <= ring;
     if (h->fused_ok) {
       // the cooperative launch needs one resident CTA per SM
       int blocks = 0;
@@ -461,8 +477,13 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
     P.out_cluster_ids = out_cluster_ids;
     P.out_max_logit = out_max_logit;
     P.scores = h->keys;
-    P.cand_logits = h->cand_logits;
-    P.ghist = h->ghist;
+    P.z_slot = h->z_slot;
+    P.hist_hi = h->b1_hist_hi;
+    P.hist_lo = h->b1_hist_lo;
+    P.bitmap = h->b1_bitmap;
+    P.bnd_list = h->b1_bnd;
+    P.bnd_count = h->b1_bnd_count;
+    P.words = h->words;
     P.best = h->best;
     P.sync = h->sync;
     P.v = D.v;

@@ -21,8 +21,9 @@ struct SyncWords {
   uint32_t arrive;        // grid barrier arrivals
   uint32_t ticket;        // kernel exit tickets (last CTA finalises)
   uint32_t union_count;   // distinct clusters of the last batched decode
-  uint32_t epoch;         // fused B = 1 calls so far (selects the histogram buffer)
-  uint32_t pad[3];
+  uint32_t epoch;         // fused B = 1 calls so far (selects the per-call buffers)
+  uint32_t arrive2;       // second barrier (boundary list complete)
+  uint32_t pad[2];
 };
 
 struct B1Params {
@@ -35,12 +36,17 @@ struct B1Params {
   int32_t* out_tokens;
   int32_t* out_cluster_ids;
   float* out_max_logit;
-  float* scores;          // workspace [c]
-  float* cand_logits;     // workspace [p*b]
-  uint32_t* ghist;        // workspace [2][4096] key histograms, used by alternate calls
+  float* scores;          // workspace [c] keys (read only by the tie fallback)
+  float* z_slot;          // workspace [v]: logit of slot k*b + j (sampling)
+  // per-call state, two buffers used by alternate calls
+  uint32_t* hist_hi;      // [2][256]   histogram of key >> 24
+  uint32_t* hist_lo;      // [2][4096]  histogram of key >> 20
+  uint32_t* bitmap;       // [2][words] selected clusters
+  unsigned long long* bnd_list;  // [2][2048] boundary (key << 32 | id)
+  uint32_t* bnd_count;    // [2]
   unsigned long long* best;
   SyncWords* sync;
-  int v, d, c, b, p;
+  int v, d, c, b, p, words;
   int crow_bytes;         // bytes per centroid row in Crows
   int mode;
   float T;
