@@ -16,6 +16,7 @@ cudaError_t set_attrs_dense(int max_smem);
 int dense_max_rows();
 cudaError_t occupancy_decode_b1(int int4, int nch, size_t smem, int* blocks);
 size_t decode_b1_misc_bytes();
+cudaError_t occupancy_dense(int nch, size_t smem, int* blocks);
 }  // namespace fh
 
 using namespace fh;
@@ -35,13 +36,17 @@ struct fh_head {
   float* cand_logits = nullptr;        // [max_batch, max_probes * b]
   int32_t* row_ok = nullptr;           // [max_batch]
   uint32_t* c2t_counts = nullptr;      // [v]
-  uint32_t* b1_hist_hi = nullptr;      // fused B = 1 per-call state (two buffers each)
+  uint32_t* b1_keys = nullptr;         // fused B = 1 state
+  float* b1_z_tok = nullptr;
+  uint32_t* b1_hist_hi = nullptr;
   uint32_t* b1_hist_lo = nullptr;
   uint32_t* b1_bitmap = nullptr;
   unsigned long long* b1_bnd = nullptr;
-  uint32_t* b1_bnd_count = nullptr;
-  float* z_slot = nullptr;             // [v]
+  uint32_t* b1_counts = nullptr;
+  int32_t* b1_queue = nullptr;
   int words = 0;
+  int b1_grid = 0;
+  int dense_grid = 0;
   uint32_t* hist = nullptr;            // [max_batch, 4096] batched key histograms
   const uint8_t* crows = nullptr;      // centroid rows (bf16 borrowed, or packed INT4 in ws)
   int crow_bytes = 0;
@@ -49,8 +54,7 @@ struct fh_head {
   long long spin_budget = kDefaultSpinBudget;
   // fused B = 1 plan
   bool fused_ok = false;
-  int b1_nslot = 0, b1_slot = 0, b1_off_h = 0, b1_off_bar = 0, b1_off_sel = 0, b1_off_misc = 0,
-      b1_off_ring = 0;
+  int b1_off_h = 0, b1_off_sel = 0, b1_off_misc = 0, b1_off_scratch = 0;
   size_t b1_smem = 0;
 };
 
@@ -238,14 +242,16 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   const size_t o_log = take(mb * nc * 4);
   const size_t o_rok = take(mb * 4);
   const size_t o_cnt = take(static_cast<size_t>(D.v) * 4);
+  const size_t o_hist = take(mb * kHistBins * 4);
   const int words = (D.c + 31) / 32;
+  const size_t o_keys1 = take(static_cast<size_t>(D.c) * 4);
+  const size_t o_ztok = take(static_cast<size_t>(D.v) * 4);
   const size_t o_hhi = take(2 * 256 * 4);
   const size_t o_hlo = take(2 * kHistBins * 4);
   const size_t o_bmp = take(2 * static_cast<size_t>(words) * 4);
   const size_t o_bnd = take(2 * kBoundaryMax * 8);
-  const size_t o_bnc = take(2 * 4);
-  const size_t o_zs = take(static_cast<size_t>(D.v) * 4);
-  const size_t o_hist = take(mb * kHistBins * 4);
+  const size_t o_bcnt = take(4 * 4);
+  const size_t o_queue = take(2 * nc * 4);
   const size_t o_crow = D.fmt == FH_CENTROID_INT4_G32 ? take(static_cast<size_t>(D.c) * h->crow_bytes) : 0;
   h->ws_bytes = off;
 
@@ -267,12 +273,14 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   h->cand_logits = reinterpret_cast<float*>(h->ws + o_log);
   h->row_ok = reinterpret_cast<int32_t*>(h->ws + o_rok);
   h->c2t_counts = reinterpret_cast<uint32_t*>(h->ws + o_cnt);
+  h->b1_keys = reinterpret_cast<uint32_t*>(h->ws + o_keys1);
+  h->b1_z_tok = reinterpret_cast<float*>(h->ws + o_ztok);
   h->b1_hist_hi = reinterpret_cast<uint32_t*>(h->ws + o_hhi);
   h->b1_hist_lo = reinterpret_cast<uint32_t*>(h->ws + o_hlo);
   h->b1_bitmap = reinterpret_cast<uint32_t*>(h->ws + o_bmp);
   h->b1_bnd = reinterpret_cast<unsigned long long*>(h->ws + o_bnd);
-  h->b1_bnd_count = reinterpret_cast<uint32_t*>(h->ws + o_bnc);
-  h->z_slot = reinterpret_cast<float*>(h->ws + o_zs);
+  h->b1_counts = reinterpret_cast<uint32_t*>(h->ws + o_bcnt);
+  h->b1_queue = reinterpret_cast<int32_t*>(h->ws + o_queue);
   h->words = words;
   h->hist = reinterpret_cast<uint32_t*>(h->ws + o_hist);
   h->crows = D.fmt == FH_CENTROID_INT4_G32 ? h->ws + o_crow : static_cast<const uint8_t*>(D.C);
@@ -294,6 +302,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
       }
     }
     e = cudaMemsetAsync(h->ws, 0, h->ws_bytes, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(h->b1_queue, 0xFF, 2 * nc * 4, st);  // empty row-queue slots are -1
     if (e != cudaSuccess) { status = cuda_fail(e); break; }
     C2TCheckParams cp{D.C2T, h->c2t_counts, &h->sync->status, static_cast<long long>(D.v), D.v};
     e = launch_c2t_check(cp, st);
@@ -315,37 +324,32 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
     return status;
   }
 
-  // ---- fused B = 1 plan ----
+  // ---- fused B = 1 plan: h (fp32), selection list, misc, scratch ----
   {
-    const size_t slot = up(std::max(static_cast<size_t>(D.d) * 2, static_cast<size_t>(h->crow_bytes)), 128);
     size_t o = 0;
     h->b1_off_h = static_cast<int>(o);
-    o += up(static_cast<size_t>(D.d) * 2, 128);
-    h->b1_off_bar = static_cast<int>(o);
-    o += up(static_cast<size_t>(kWarps) * 8 * 8, 128);
+    o += up(static_cast<size_t>(D.d) * 4, 128);
     h->b1_off_sel = static_cast<int>(o);
     o += up(static_cast<size_t>(D.max_probes) * 4, 128);
     h->b1_off_misc = static_cast<int>(o);
     o += up(decode_b1_misc_bytes(), 128);
-    o = up(o, 1024);
-    h->b1_off_ring = static_cast<int>(o);
-    const int nslot = ring_slots(h->smem_budget, o, slot);
-    const size_t ring = static_cast<size_t>(kWarps) * nslot * slot;
-    const size_t sel_scratch = hist_select_smem_bytes(D.c);
-    h->b1_nslot = nslot;
-    h->b1_slot = static_cast<int>(slot);
-    h->b1_smem = o + ring;
-    // each warp owns at most 32 clusters (one per lane register)
-    const long long warps = static_cast<long long>(h->num_sms) * kWarps;
-    h->fused_ok = nslot >= 2 && sel_scratch <= ring && D.c <= 32 * warps &&
-                  static_cast<size_t>(kBoundaryMax) * 8 <= ring;
-    if (h->fused_ok) {
-      // the cooperative launch needs one resident CTA per SM
-      int blocks = 0;
-      e = occupancy_decode_b1(D.fmt == FH_CENTROID_INT4_G32, h->nch, h->b1_smem, &blocks);
-      h->fused_ok = e == cudaSuccess && blocks >= 1;
-      (void)cudaGetLastError();
-    }
+    h->b1_off_scratch = static_cast<int>(o);
+    o += up(std::max(std::max(static_cast<size_t>(kHistBins) * 4, static_cast<size_t>(kBoundaryMax) * 8),
+                     sizeof(SelectSmem)), 128);
+    h->b1_smem = o;
+    int blocks = 0;
+    e = occupancy_decode_b1(D.fmt == FH_CENTROID_INT4_G32, h->nch, h->b1_smem, &blocks);
+    (void)cudaGetLastError();
+    const int per_sm = e == cudaSuccess ? std::min(blocks, 2) : 0;
+    h->b1_grid = per_sm * h->num_sms;
+    // each warp owns at most 32 clusters (one key per lane register)
+    h->fused_ok = per_sm >= 1 && D.c <= 32LL * h->b1_grid * kWarps;
+  }
+  {
+    int blocks = 0;
+    e = occupancy_dense(h->nch, static_cast<size_t>(dense_max_rows()) * D.d * 4, &blocks);
+    (void)cudaGetLastError();
+    h->dense_grid = (e == cudaSuccess && blocks >= 1 ? std::min(blocks, 2) : 1) * h->num_sms;
   }
   *out = h;
   return FH_OK;
@@ -476,14 +480,14 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
     P.out_tokens = out_tokens;
     P.out_cluster_ids = out_cluster_ids;
     P.out_max_logit = out_max_logit;
-    P.scores = h->keys;
-    P.z_slot = h->z_slot;
+    P.keys = h->b1_keys;
+    P.z_tok = h->b1_z_tok;
     P.hist_hi = h->b1_hist_hi;
     P.hist_lo = h->b1_hist_lo;
     P.bitmap = h->b1_bitmap;
     P.bnd_list = h->b1_bnd;
-    P.bnd_count = h->b1_bnd_count;
-    P.words = h->words;
+    P.counts = h->b1_counts;
+    P.row_queue = h->b1_queue;
     P.best = h->best;
     P.sync = h->sync;
     P.v = D.v;
@@ -491,18 +495,17 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
     P.c = D.c;
     P.b = D.b;
     P.p = p;
+    P.words = h->words;
+    P.nc_max = D.max_probes * D.b;
     P.crow_bytes = h->crow_bytes;
     P.mode = mode;
     P.T = gumbel ? T : 1.f;
-    P.nslot = h->b1_nslot;
-    P.slot_bytes = h->b1_slot;
     P.off_h = h->b1_off_h;
-    P.off_bar = h->b1_off_bar;
     P.off_sel = h->b1_off_sel;
     P.off_misc = h->b1_off_misc;
-    P.off_ring = h->b1_off_ring;
+    P.off_scratch = h->b1_off_scratch;
     P.spin_budget = h->spin_budget;
-    cudaError_t e = launch_decode_b1(P, h->num_sms, h->b1_smem, D.fmt == FH_CENTROID_INT4_G32, h->nch, st);
+    cudaError_t e = launch_decode_b1(P, h->b1_grid, h->b1_smem, D.fmt == FH_CENTROID_INT4_G32, h->nch, st);
     return e == cudaSuccess ? FH_OK : cuda_fail(e);
   }
 
@@ -552,15 +555,9 @@ fh_status fh_dense_head(fh_head* h, const void* hidden, int32_t B, float* logits
   if (!out_argmax) return FH_ERR_INVALID_ARG;
   const fh_head_desc& D = h->desc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const size_t slot = up(static_cast<size_t>(D.d) * 2, 128);
-  const size_t row_bytes = static_cast<size_t>(D.d) * 2;
-  const int rmax_cfg = dense_max_rows();
-  for (int r0 = 0; r0 < B; r0 += rmax_cfg) {
-    const int rows = B - r0 < rmax_cfg ? B - r0 : rmax_cfg;
-    const size_t hbytes = up(rows * row_bytes, 128);
-    const size_t off_ring = 1024;
-    const int nslot = ring_slots(h->smem_budget, off_ring + hbytes, slot);
-    if (nslot < 1) return FH_ERR_UNSUPPORTED;
+  const int rmax = dense_max_rows();
+  for (int r0 = 0; r0 < B; r0 += rmax) {
+    const int rows = B - r0 < rmax ? B - r0 : rmax;
     DenseParams P{};
     P.E = static_cast<const uint16_t*>(D.E);
     P.hidden = static_cast<const uint16_t*>(hidden);
@@ -572,13 +569,8 @@ fh_status fh_dense_head(fh_head* h, const void* hidden, int32_t B, float* logits
     P.d = D.d;
     P.row0 = r0;
     P.rows = rows;
-    P.nslot = nslot;
-    P.slot_bytes = static_cast<int>(slot);
-    P.off_bar = 0;
-    P.off_ring = static_cast<int>(off_ring);
-    P.off_h = static_cast<int>(off_ring + static_cast<size_t>(kWarps) * nslot * slot);
-    const size_t smem = P.off_h + hbytes;
-    cudaError_t e = launch_dense(P, h->num_sms, smem, h->nch, st);
+    const size_t smem = static_cast<size_t>(rows) * D.d * 4;
+    cudaError_t e = launch_dense(P, h->dense_grid, smem, h->nch, st);
     if (e != cudaSuccess) return cuda_fail(e);
   }
   return FH_OK;

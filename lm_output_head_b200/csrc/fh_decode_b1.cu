@@ -1,36 +1,37 @@
 // Fused FlashHead decode for one hidden state (B = 1): one persistent
-// cooperative launch of one 512-thread CTA per SM.
+// cooperative launch, two 512-thread CTAs per SM, every row streamed HBM ->
+// registers with non-allocating 16-byte loads and dotted with h staged once
+// per CTA in shared memory (fp32).
 //
 // The pages' pipeline (FlashHead write-up, section 2.2.2: h -> centroid_scores
 // -> top_p_clusters -> token_scores) runs as phases of one kernel:
 //
-//  1. centroid scores (section 1.2.2; INT4 centroids per section 1.2.4): the
-//     c centroid rows are spread round-robin over every warp of the grid
-//     (cluster k belongs to global warp k mod W); each warp streams its rows
-//     HBM -> shared memory with cp.async.bulk into a private ring of slots and
-//     dots them with h held in registers. The key (the score, or when sampling
-//     the Gumbel key s/T - ln(-ln u), section 1.2.3) stays in a lane register
-//     of the owning warp and is counted into two device-wide histograms of its
-//     top 8 and top 12 bits (fire-and-forget atomics).
-//  2. device-wide barrier; one warp per CTA reads the two small histograms and
-//     finds the 12-bit bin t1 holding the p-th largest key. Every key above t1
-//     is selected; the keys inside t1 are the boundary. Each CTA classifies
-//     only the clusters it owns -- no CTA ever reads all c keys.
-//  3. each CTA streams the token rows of its own surely-selected clusters
-//     (gather through C2T, section 1.2.1: slot k*b + j holds token C2T[k][j]),
-//     dots them with h and keeps a packed (logit, token) maximum.
+//  1. centroid scores (section 1.2.2; INT4 centroids per section 1.2.4):
+//     cluster k belongs to global warp k mod W, which streams its centroid
+//     row and computes the key -- the score, or when sampling the Gumbel key
+//     s/T - ln(-ln u) (section 1.2.3). The key stays in a lane register of the
+//     owning warp and is counted into two device-wide histograms of its top 8
+//     and top 12 bits (fire-and-forget atomics).
+//  2. device-wide barrier; each CTA reads the histograms once and finds the
+//     12-bit bin t1 holding the p-th largest key. Keys above t1 are selected;
+//     keys inside t1 form the boundary. Owners publish the b token ids of
+//     each selected cluster (the C2T row, section 1.2.1: slot k*b + j holds
+//     token C2T[k][j]) into a device-wide row queue.
+//  3. the candidate rows are spread round-robin over every warp of the grid:
+//     a warp polls its queue slot for the token id, streams the token row and
+//     keeps a packed (logit, token) maximum (section 1.2.4, stage 2).
 //  4. only when the boundary bin is split (some but not all of its keys are
-//     needed): the boundary keys were published to a small global list, a
-//     second barrier (whose wait overlaps step 3) completes it, and each CTA
-//     ranks its own boundary keys exactly (key desc, id asc) and streams the
-//     ones that are in.
-//  5. the CTA maxima meet in one 64-bit atomicMax; the last CTA to finish
-//     (exit ticket) writes the token: the argmax, or, when sampling, the
-//     inverse-CDF draw over softmax(z/T) in canonical order (cluster asc, slot
-//     asc), walking a bitmap of the selected clusters.
+//     needed): owners published their boundary keys to a small list; after a
+//     second barrier each owner ranks its boundary keys exactly (key desc, id
+//     asc) against the list and queues the chosen clusters' rows, which the
+//     consumers pick up as in step 3.
+//  5. CTA maxima meet in one 64-bit atomicMax; the last CTA to finish (exit
+//     ticket) writes the token: the argmax, or, when sampling, the inverse-CDF
+//     draw over softmax(z/T) in canonical order (cluster asc, slot asc),
+//     walking a bitmap of the selected clusters.
 //
-// HBM traffic is the algorithmic minimum: each centroid row once, each
-// selected token row once, plus the C2T rows and h.
+// No CTA ever reads all c keys, and HBM traffic is the algorithmic minimum:
+// each centroid row once, each selected token row once, plus C2T rows and h.
 #include <climits>
 
 #include "fh_device.cuh"
@@ -39,31 +40,23 @@ namespace fh {
 namespace {
 
 constexpr int kHiBins = 256;
-constexpr int kMaxOwn = kWarps * 32;  // clusters a CTA can own (32 per warp)
 
 struct B1Misc {
-  unsigned long long hbar;
   unsigned long long wbest[kWarps];
   float scan[kWarps + 1];
   uint32_t uscan[kWarps + 1];
   int claim, lastpos, ok, last;
-  uint32_t t1, need, split, fallback;
-  uint32_t n_sure, n_bnd, n_bsel;
-  int32_t sure[kMaxOwn];
-  int32_t bnd[kMaxOwn];
-  uint32_t bnd_key[kMaxOwn];
+  uint32_t t1, need, split, fallback, n_sure;
 };
 
 // Device-wide barrier over the cooperative grid; false if `budget` cycles pass first.
-__device__ bool grid_barrier(uint32_t* arrive, uint32_t G, long long budget, B1Misc* misc) {
+__device__ bool grid_wait(uint32_t* counter, uint32_t target, long long budget, int* flag) {
   __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(arrive, 1u);
     int ok = 1;
-    if (ld_acquire_u32(arrive) < G) {
+    if (ld_acquire_u32(counter) < target) {
       const long long t0 = clock64();
-      while (ld_acquire_u32(arrive) < G) {
+      while (ld_acquire_u32(counter) < target) {
         if (clock64() - t0 > budget) {
           ok = 0;
           break;
@@ -71,13 +64,20 @@ __device__ bool grid_barrier(uint32_t* arrive, uint32_t G, long long budget, B1M
       }
     }
     __threadfence();
-    misc->ok = ok;
+    *flag = ok;
   }
   __syncthreads();
-  return misc->ok != 0;
+  return *flag != 0;
 }
 
-// Warp-inclusive prefix sum over lanes.
+__device__ __forceinline__ void grid_arrive(uint32_t* counter) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(counter, 1u);
+  }
+}
+
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
@@ -88,46 +88,61 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x) {
   return x;
 }
 
-// Stream the rows of `n_items` candidate slots of this CTA (item q -> cluster
-// list[q / b], slot q % b) through the warp rings; items go round-robin over
-// the CTA's warps. Updates `best` and, when sampling, the per-slot logits.
-template <int NCH>
-__device__ __forceinline__ bool stream_candidates(const B1Params& P, const int32_t* list, int n_items,
-                                                  const float* hr, uint32_t ring_w, uint32_t bar_w,
-                                                  uint32_t& phase_bits, unsigned long long& best,
-                                                  bool gumbel) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int n = warp < n_items ? (n_items - 1 - warp) / kWarps + 1 : 0;
-  const int b = P.b;
-  auto slot_of = [&](int i) -> int {  // flat index k*b + j of the warp's item i
-    const int q = warp + i * kWarps;
-    return list[q / b] * b + q % b;
-  };
-  int tok0 = 0, tok1 = 0;  // lane j: tokens of items j and 32 + j
-  if (lane < n) tok0 = __ldg(P.C2T + slot_of(lane));
-  if (32 + lane < n) tok1 = __ldg(P.C2T + slot_of(32 + lane));
-  auto token_of = [&](int i) -> int {
-    const int a = __shfl_sync(0xFFFFFFFFu, tok0, i & 31);
-    const int c1 = __shfl_sync(0xFFFFFFFFu, tok1, i & 31);
-    if (i < 32) return a;
-    if (i < 64) return c1;
-    return __ldg(P.C2T + slot_of(i));
-  };
-  auto src = [&](int i, const void*& ptr, uint32_t& bytes) {
-    ptr = P.E + static_cast<size_t>(token_of(i)) * P.d;
-    bytes = static_cast<uint32_t>(P.d * 2);
-  };
-  auto use = [&](int i, uint32_t slot) {
-    const int t = token_of(i);
-    const float z = row_dot_bf16<NCH>(slot, P.d, hr);
-    const unsigned long long pk = pack_best(z, t);
-    best = pk > best ? pk : best;
-    if (gumbel && lane == 0) P.z_slot[slot_of(i)] = z;
-  };
-  return warp_stream(n, P.nslot, ring_w, P.slot_bytes, bar_w, phase_bits, kWaitBudget, src, use);
+// Poll a row-queue slot until an owner has written the token id (bounded).
+__device__ __forceinline__ int poll_token(const int32_t* slot, long long budget) {
+  int t = static_cast<int>(ld_acquire_u32(reinterpret_cast<const unsigned*>(slot)));
+  if (t >= 0) return t;
+  const long long t0 = clock64();
+  while ((t = static_cast<int>(ld_acquire_u32(reinterpret_cast<const unsigned*>(slot)))) < 0) {
+    if (clock64() - t0 > budget) return -1;
+  }
+  return t;
 }
 
-// Ascending list of the clusters set in `bitmap` (words of 32 ids) into `sel`.
+// Queue the b token rows of cluster k (one warp): slots pos*b .. pos*b + b - 1.
+__device__ __forceinline__ void publish_cluster(const B1Params& P, int32_t* rq, uint32_t* qcount, uint32_t* bitmap,
+                                                int k) {
+  const int lane = threadIdx.x & 31;
+  uint32_t pos = 0;
+  if (lane == 0) {
+    pos = atomicAdd(qcount, 1u);
+    atomicOr(bitmap + (k >> 5), 1u << (k & 31));
+  }
+  pos = __shfl_sync(0xFFFFFFFFu, pos, 0);
+  if (pos >= static_cast<uint32_t>(P.p)) return;  // only an inconsistent histogram could overfill the queue
+  for (int j = lane; j < P.b; j += 32)
+    rq[static_cast<size_t>(pos) * P.b + j] = __ldg(P.C2T + static_cast<size_t>(k) * P.b + j);
+}
+
+// Consume candidate rows r = r0 + gw + i*W (< r1) of the row queue.
+template <int NCH>
+__device__ __forceinline__ void consume_rows(const B1Params& P, const int32_t* rq, const int32_t* ssel, bool direct,
+                                             int r0, int r1, int gw, int W, const float* hs,
+                                             unsigned long long& best, bool gumbel, bool& ok) {
+  const int lane = threadIdx.x & 31;
+  for (int r = r0 + gw; r < r1; r += W) {
+    int t;
+    if (direct) {
+      t = __ldg(P.C2T + static_cast<size_t>(ssel[r / P.b]) * P.b + r % P.b);
+    } else {
+      t = 0;
+      if (lane == 0) t = poll_token(rq + r, P.spin_budget);
+      t = __shfl_sync(0xFFFFFFFFu, t, 0);
+      if (t < 0) {
+        ok = false;
+        continue;
+      }
+    }
+    uint4 w[NCH];
+    row_load_bf16<NCH>(P.E + static_cast<size_t>(t) * P.d, P.d, w);
+    const float z = row_dot_bf16_hs<NCH>(w, hs, P.d);
+    const unsigned long long pk = pack_best(z, t);
+    best = pk > best ? pk : best;
+    if (gumbel && lane == 0) P.z_tok[t] = z;
+  }
+}
+
+// Ascending list of the clusters set in `bitmap` into `sel` (at most cap).
 __device__ void bitmap_to_list(const uint32_t* bitmap, int words, int32_t* sel, int cap, B1Misc* misc) {
   const int tid = threadIdx.x;
   uint32_t base = 0;
@@ -150,119 +165,107 @@ __device__ void bitmap_to_list(const uint32_t* bitmap, int words, int32_t* sel, 
 }
 
 template <int NCH, bool INT4>
-__global__ void __launch_bounds__(kThreads, 1) decode_b1_kernel(const B1Params P) {
+__global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = gridDim.x;
   const int W = G * kWarps;
   const int gw = blockIdx.x * kWarps + warp;
-  const int d = P.d;
+  const int d = P.d, b = P.b;
+  const bool gumbel = P.mode == 1;
 
-  uint16_t* sh = reinterpret_cast<uint16_t*>(smem + P.off_h);
+  float* hs = reinterpret_cast<float*>(smem + P.off_h);
   int32_t* ssel = reinterpret_cast<int32_t*>(smem + P.off_sel);
   B1Misc* misc = reinterpret_cast<B1Misc*>(smem + P.off_misc);
-  uint8_t* ring = smem + P.off_ring;
-  const uint32_t ring_w = smem_addr(ring) + static_cast<uint32_t>(warp * P.nslot * P.slot_bytes);
-  const uint32_t bar_w = smem_addr(smem + P.off_bar) + static_cast<uint32_t>(warp * P.nslot * 8);
+  uint8_t* scratch = smem + P.off_scratch;  // histogram copy, boundary list, or fallback select state
 
-  uint32_t phase_bits = 0;
-  bool ok = true;
-  const bool gumbel = P.mode == 1;
-  // per-call state lives in two buffers used by alternate calls; this call
-  // clears the other buffer for the next one
+  // per-call state: two buffers used by alternate calls; this call clears the other one
   const uint32_t epoch = P.sync->epoch;
   const uint32_t par = epoch & 1u, nxt = par ^ 1u;
   uint32_t* hist_hi = P.hist_hi + par * kHiBins;
   uint32_t* hist_lo = P.hist_lo + par * kHistBins;
   uint32_t* bitmap = P.bitmap + par * P.words;
   unsigned long long* bnd_list = P.bnd_list + par * kBoundaryMax;
-  uint32_t* bnd_count = P.bnd_count + par;
+  uint32_t* bnd_count = P.counts + 2 * par;
+  uint32_t* qcount = P.counts + 2 * par + 1;
+  int32_t* rq = P.row_queue + static_cast<size_t>(par) * P.nc_max;
 
   // ---------------- phase 1: centroid scores ----------------
-  // h is staged by the first bulk copy of the CTA; the centroid rows follow
-  // at once (they do not depend on h).
-  const uint32_t hbar = smem_addr(&misc->hbar);
-  if (tid == 0) {
-    mbar_init(hbar, 1);
-    fence_mbar_init();
-    mbar_expect_tx(hbar, static_cast<uint32_t>(d * 2));
-    bulk_g2s(smem_addr(sh), P.hidden, static_cast<uint32_t>(d * 2), hbar);
-  }
-  warp_ring_init(bar_w, P.nslot);
   const int n1 = gw < P.c ? (P.c - 1 - gw) / W + 1 : 0;  // <= 32 (host-checked)
-  auto src1 = [&](int i, const void*& ptr, uint32_t& bytes) {
-    ptr = P.Crows + static_cast<size_t>(gw + i * W) * P.crow_bytes;
-    bytes = static_cast<uint32_t>(P.crow_bytes);
-  };
-  warp_stream_prologue(n1, P.nslot, ring_w, P.slot_bytes, bar_w, src1);
+  constexpr int NQ = (NCH + 1) / 2;
+  uint4 w[NCH];
+  uint2 q[NQ];
+  uint32_t sc[NQ];
+  if (n1 > 0) {  // the first centroid row goes out before anything else
+    if constexpr (INT4) row_load_int4<NQ>(P.Crows + static_cast<size_t>(gw) * P.crow_bytes, d, q, sc);
+    else row_load_bf16<NCH>(reinterpret_cast<const uint16_t*>(P.Crows + static_cast<size_t>(gw) * P.crow_bytes), d, w);
+  }
   float ureg = 0.f;  // lane j holds u of item j
   if (gumbel && lane < n1) ureg = __ldg(P.u_clusters + gw + lane * W);
+  stage_h_f32(P.hidden, d, hs);
   {
-    const int nz = kHiBins + kHistBins + P.words + 1;
+    const int nz = kHiBins + kHistBins + P.words + 2 + P.nc_max;
     const int per = (nz + G - 1) / G;
     for (int i = tid; i < per; i += kThreads) {
-      const int z = blockIdx.x * per + i;
-      if (z < kHiBins) P.hist_hi[nxt * kHiBins + z] = 0u;
-      else if (z < kHiBins + kHistBins) P.hist_lo[nxt * kHistBins + (z - kHiBins)] = 0u;
-      else if (z < kHiBins + kHistBins + P.words) P.bitmap[nxt * P.words + (z - kHiBins - kHistBins)] = 0u;
-      else if (z == nz - 1) P.bnd_count[nxt] = 0u;
+      int z = blockIdx.x * per + i;
+      if (z < kHiBins) { P.hist_hi[nxt * kHiBins + z] = 0u; continue; }
+      z -= kHiBins;
+      if (z < kHistBins) { P.hist_lo[nxt * kHistBins + z] = 0u; continue; }
+      z -= kHistBins;
+      if (z < P.words) { P.bitmap[nxt * P.words + z] = 0u; continue; }
+      z -= P.words;
+      if (z < 2) { P.counts[2 * nxt + z] = 0u; continue; }
+      z -= 2;
+      if (z < P.nc_max) P.row_queue[static_cast<size_t>(nxt) * P.nc_max + z] = -1;
     }
   }
-  if (tid == 0) {
-    misc->n_sure = 0u;
-    misc->n_bnd = 0u;
-    misc->n_bsel = 0u;
-  }
-  __syncthreads();  // hbar initialised before anyone waits on it
-  if (!mbar_wait_bounded(hbar, 0u, kWaitBudget)) {
-    ok = false;
-    if (lane == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
-  }
+  __syncthreads();
+
   uint32_t own_key = 0u;  // lane j: key of the warp's item j
-  {
-    auto finish = [&](int i, float s) {
-      const int k = gw + i * W;
-      const float u = __shfl_sync(0xFFFFFFFFu, ureg, i & 31);
-      const float key = gumbel ? gumbel_key(s, P.T, u) : s;
-      const uint32_t kk = f2key(key);
-      if (lane == (i & 31)) own_key = kk;
-      if (lane == 0) {
-        P.scores[k] = key;
-        atomicAdd(hist_hi + (kk >> 24), 1u);
-        atomicAdd(hist_lo + (kk >> kHistShift), 1u);
-        prefetch_l2(P.C2T + static_cast<size_t>(k) * P.b);
-      }
-    };
+  for (int i = 0; i < n1; ++i) {
+    const int k = gw + i * W;
+    float s;
     if constexpr (INT4) {
-      constexpr int NQ = (NCH + 1) / 2;
-      float hq[NQ * 16];
-      load_h_halfgroups<NQ>(sh, d, hq);
-      auto use = [&](int i, uint32_t slot) { finish(i, row_dot_int4<NQ>(slot, d, hq)); };
-      ok = warp_stream_run(n1, P.nslot, ring_w, P.slot_bytes, bar_w, phase_bits, kWaitBudget, src1, use) && ok;
+      if (i > 0) row_load_int4<NQ>(P.Crows + static_cast<size_t>(k) * P.crow_bytes, d, q, sc);
+      s = row_dot_int4_hs<NQ>(q, sc, hs, d);
     } else {
-      float hr[NCH * 8];
-      load_h_chunks<NCH>(sh, d, hr);
-      auto use = [&](int i, uint32_t slot) { finish(i, row_dot_bf16<NCH>(slot, d, hr)); };
-      ok = warp_stream_run(n1, P.nslot, ring_w, P.slot_bytes, bar_w, phase_bits, kWaitBudget, src1, use) && ok;
+      if (i > 0) row_load_bf16<NCH>(reinterpret_cast<const uint16_t*>(P.Crows + static_cast<size_t>(k) * P.crow_bytes), d, w);
+      s = row_dot_bf16_hs<NCH>(w, hs, d);
     }
-    if (!ok && lane == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
+    const float u = __shfl_sync(0xFFFFFFFFu, ureg, i & 31);
+    const float key = gumbel ? gumbel_key(s, P.T, u) : s;
+    const uint32_t kk = f2key(key);
+    if (lane == (i & 31)) own_key = kk;
+    if (lane == 0) {
+      P.keys[k] = kk;
+      atomicAdd(hist_hi + (kk >> 24), 1u);
+      atomicAdd(hist_lo + (kk >> kHistShift), 1u);
+      prefetch_l2(P.C2T + static_cast<size_t>(k) * b);
+    }
   }
 
-  // ---------------- phase 2: barrier, boundary bin, own classification ----------------
-  const bool passed = grid_barrier(&P.sync->arrive, static_cast<uint32_t>(G), P.spin_budget, misc);
+  // ---------------- phase 2: barrier, boundary bin, owners publish ----------------
+  grid_arrive(&P.sync->arrive);
+  const bool passed = grid_wait(&P.sync->arrive, static_cast<uint32_t>(G), P.spin_budget, &misc->ok);
   unsigned long long best = 0ull;
+  bool ok = true;
   if (!passed) {
     if (tid == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
   } else {
     const uint32_t p = static_cast<uint32_t>(P.p);
+    uint32_t* hlo = reinterpret_cast<uint32_t*>(scratch);
+    uint32_t hv[8];
+    if (warp == 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) hv[i] = __ldcg(hist_hi + kHiBins - 1 - 8 * lane - i);
+    }
+    for (int i = tid; i < kHistBins; i += kThreads) hlo[i] = __ldcg(hist_lo + i);
+    __syncthreads();
     if (warp == 0) {
       // top-8-bit bins, descending: lane l owns bins 255-8l .. 248-8l
-      uint32_t hv[8], s = 0;
+      uint32_t s = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        hv[i] = __ldcg(hist_hi + kHiBins - 1 - 8 * lane - i);
-        s += hv[i];
-      }
+      for (int i = 0; i < 8; ++i) s += hv[i];
       const uint32_t incl = warp_incl_scan(s), excl = incl - s;
       const int L = __ffs(__ballot_sync(0xFFFFFFFFu, excl < p && p <= incl)) - 1;
       uint32_t thi = 0, above_hi = 0, run = excl;
@@ -277,123 +280,93 @@ __global__ void __launch_bounds__(kThreads, 1) decode_b1_kernel(const B1Params P
       thi = __shfl_sync(0xFFFFFFFFu, thi, L);
       above_hi = __shfl_sync(0xFFFFFFFFu, above_hi, L);
       // its 16 sub-bins of 12 bits, descending
-      const uint32_t x = lane < 16 ? __ldcg(hist_lo + thi * 16 + 15 - lane) : 0u;
+      const uint32_t x = lane < 16 ? hlo[thi * 16 + 15 - lane] : 0u;
       const uint32_t incl2 = warp_incl_scan(x), excl2 = incl2 - x;
       const uint32_t target = p - above_hi;
       const int L2 = __ffs(__ballot_sync(0xFFFFFFFFu, lane < 16 && excl2 < target && target <= incl2)) - 1;
       const uint32_t ex2 = __shfl_sync(0xFFFFFFFFu, excl2, L2);
       const uint32_t m1 = __shfl_sync(0xFFFFFFFFu, x, L2);
       if (lane == 0) {
+        const uint32_t need = target - ex2;
         misc->t1 = thi * 16 + 15 - L2;
-        misc->need = target - ex2;
-        misc->split = (m1 != target - ex2) ? 1u : 0u;
-        misc->fallback = (m1 != target - ex2 && m1 > static_cast<uint32_t>(kBoundaryMax)) ? 1u : 0u;
+        misc->need = need;
+        misc->split = m1 != need ? 1u : 0u;
+        misc->fallback = (m1 != need && m1 > static_cast<uint32_t>(kBoundaryMax)) ? 1u : 0u;
+        misc->n_sure = m1 != need ? p - need : p;
       }
     }
     __syncthreads();
     const uint32_t t1 = misc->t1;
     const bool split = misc->split != 0, fallback = misc->fallback != 0;
+    const int r_sure = static_cast<int>(misc->n_sure) * b, r_all = P.p * b;
 
     if (!fallback) {
-      if (lane < n1) {
-        const int k = gw + lane * W;
-        const uint32_t dg = own_key >> kHistShift;
-        if (dg > t1 || (dg == t1 && !split)) {
-          misc->sure[atomicAdd(&misc->n_sure, 1u)] = k;
-          atomicOr(bitmap + (k >> 5), 1u << (k & 31));
-        } else if (dg == t1) {
-          const uint32_t q = atomicAdd(&misc->n_bnd, 1u);
-          misc->bnd[q] = k;
-          misc->bnd_key[q] = own_key;
-          const uint32_t at = atomicAdd(bnd_count, 1u);
-          if (at < static_cast<uint32_t>(kBoundaryMax))
-            bnd_list[at] = (static_cast<unsigned long long>(own_key) << 32) | static_cast<uint32_t>(k);
-        }
+      const uint32_t dg = own_key >> kHistShift;
+      const bool mine = lane < n1;
+      uint32_t sure = __ballot_sync(0xFFFFFFFFu, mine && (dg > t1 || (dg == t1 && !split)));
+      while (sure) {  // queue the rows of each selected cluster this warp owns
+        const int j = __ffs(sure) - 1;
+        sure &= sure - 1;
+        publish_cluster(P, rq, qcount, bitmap, gw + j * W);
       }
-      __syncthreads();
-      if (split && tid == 0) {  // boundary keys published: arrive at the second barrier
-        __threadfence();
-        atomicAdd(&P.sync->arrive2, 1u);
+      if (mine && split && dg == t1) {
+        const uint32_t at = atomicAdd(bnd_count, 1u);
+        if (at < static_cast<uint32_t>(kBoundaryMax))
+          bnd_list[at] = (static_cast<unsigned long long>(own_key) << 32) | static_cast<uint32_t>(gw + lane * W);
       }
+      __threadfence();
+      if (split) grid_arrive(&P.sync->arrive2);
     } else {
-      // pathological ties (huge boundary bin): every CTA selects over all keys
-      select_top_p_hist(P.scores, nullptr, 1.f, P.c, P.p, hist_lo, ssel, ring);
-      for (int q = tid; q < P.p; q += kThreads) {
-        const int k = ssel[q];
-        if ((k % W) / kWarps == static_cast<int>(blockIdx.x)) {
-          misc->sure[atomicAdd(&misc->n_sure, 1u)] = k;
-          atomicOr(bitmap + (k >> 5), 1u << (k & 31));
-        }
-      }
-      __syncthreads();
+      // pathological ties (a boundary bin larger than the exact-rank list):
+      // every CTA selects over all keys and reads its rows' tokens directly
+      block_select_top_p(P.keys, P.c, P.p, ssel, *reinterpret_cast<SelectSmem*>(scratch));
+      if (blockIdx.x == 0)
+        for (int i = tid; i < P.p; i += kThreads) atomicOr(bitmap + (ssel[i] >> 5), 1u << (ssel[i] & 31));
     }
-    fence_proxy_async_smem();
-    __syncthreads();
 
-    // ---------------- phase 3: stream own selected clusters ----------------
-    float hr[NCH * 8];
-    load_h_chunks<NCH>(sh, d, hr);
-    ok = stream_candidates<NCH>(P, misc->sure, static_cast<int>(misc->n_sure) * P.b, hr, ring_w, bar_w,
-                                phase_bits, best, gumbel);
-    if (!ok && lane == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
+    // ---------------- phase 3: candidate rows of the surely selected clusters ----------------
+    consume_rows<NCH>(P, rq, ssel, fallback, 0, fallback ? r_all : r_sure, gw, W, hs, best, gumbel, ok);
 
     if (split && !fallback) {
-      // ---------------- phase 4: exact rank of own boundary keys ----------------
-      __syncthreads();
-      if (tid == 0) {
-        int bok = 1;
-        if (ld_acquire_u32(&P.sync->arrive2) < static_cast<uint32_t>(G)) {
-          const long long t0 = clock64();
-          while (ld_acquire_u32(&P.sync->arrive2) < static_cast<uint32_t>(G)) {
-            if (clock64() - t0 > P.spin_budget) {
-              bok = 0;
-              break;
-            }
-          }
-        }
-        __threadfence();
-        misc->ok = bok;
-      }
-      __syncthreads();
-      if (!misc->ok) {
-        if (tid == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
+      // ---------------- phase 4: exact rank of boundary keys ----------------
+      const bool got = grid_wait(&P.sync->arrive2, static_cast<uint32_t>(G), P.spin_budget, &misc->ok);
+      if (!got) {
+        ok = false;
       } else {
+        unsigned long long* sl = reinterpret_cast<unsigned long long*>(scratch);
         const uint32_t nb = min(__ldcg(bnd_count), static_cast<uint32_t>(kBoundaryMax));
-        unsigned long long* sl = reinterpret_cast<unsigned long long*>(ring);
         for (uint32_t i = tid; i < nb; i += kThreads) sl[i] = __ldcg(bnd_list + i);
         __syncthreads();
         const uint32_t need = misc->need;
-        for (uint32_t q = warp; q < misc->n_bnd; q += kWarps) {
-          const uint32_t kq = misc->bnd_key[q];
-          const int idq = misc->bnd[q];
+        const uint32_t dg = own_key >> kHistShift;
+        uint32_t mine = __ballot_sync(0xFFFFFFFFu, lane < n1 && dg == t1);
+        while (mine) {
+          const int j = __ffs(mine) - 1;
+          mine &= mine - 1;
+          const uint32_t kq = __shfl_sync(0xFFFFFFFFu, own_key, j);
+          const int idq = gw + j * W;
           uint32_t r = 0;
           for (uint32_t e = lane; e < nb; e += 32) {
             const unsigned long long v = sl[e];
             const uint32_t ke = static_cast<uint32_t>(v >> 32);
-            const int ide = static_cast<int>(v & 0xFFFFFFFFu);
-            r += (ke > kq) || (ke == kq && ide < idq);
+            r += (ke > kq) || (ke == kq && static_cast<int>(v & 0xFFFFFFFFu) < idq);
           }
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xFFFFFFFFu, r, o);
-          if (lane == 0 && r < need) {
-            misc->sure[atomicAdd(&misc->n_bsel, 1u)] = idq;  // sure[] was consumed by phase 3
-            atomicOr(bitmap + (idq >> 5), 1u << (idq & 31));
-          }
+          if (r < need) publish_cluster(P, rq, qcount, bitmap, idq);
         }
-        fence_proxy_async_smem();
-        __syncthreads();
-        const int nbs = static_cast<int>(misc->n_bsel);
-        ok = stream_candidates<NCH>(P, misc->sure, nbs * P.b, hr, ring_w, bar_w, phase_bits, best, gumbel);
-        if (!ok && lane == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
+        __threadfence();
+        consume_rows<NCH>(P, rq, ssel, false, r_sure, r_all, gw, W, hs, best, gumbel, ok);
       }
     }
+    if (!ok && lane == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
   }
   best = warp_max_u64(best);
   if (lane == 0) misc->wbest[warp] = best;
   __syncthreads();
   if (tid == 0) {
     unsigned long long m = 0ull;
-    for (int w = 0; w < kWarps; ++w) m = misc->wbest[w] > m ? misc->wbest[w] : m;
+    for (int i = 0; i < kWarps; ++i) m = misc->wbest[i] > m ? misc->wbest[i] : m;
     if (m) atomicMax(P.best, m);
   }
 
@@ -421,13 +394,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_b1_kernel(const B1Params P
     }
   } else {
     // inverse CDF over softmax(z/T), canonical order (cluster asc, slot asc)
-    const int nc = P.p * P.b, b = P.b;
+    const int nc = P.p * b;
     const float ym = best_logit(bw) / P.T;
-    const int q = (nc + kThreads - 1) / kThreads;
-    const int i0 = min(nc, tid * q), i1 = min(nc, i0 + q);
-    auto zc = [&](int i) { return __ldcg(P.z_slot + static_cast<size_t>(ssel[i / b]) * b + i % b); };
+    const int qn = (nc + kThreads - 1) / kThreads;
+    const int i0 = min(nc, tid * qn), i1 = min(nc, i0 + qn);
+    auto tok_at = [&](int i) { return __ldg(P.C2T + static_cast<size_t>(ssel[i / b]) * b + i % b); };
     float loc = 0.f;
-    for (int i = i0; i < i1; ++i) loc += expf(zc(i) / P.T - ym);
+    for (int i = i0; i < i1; ++i) loc += expf(__ldcg(P.z_tok + tok_at(i)) / P.T - ym);
     if (tid == 0) {
       misc->claim = INT_MAX;
       misc->lastpos = 0;
@@ -439,9 +412,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_b1_kernel(const B1Params P
     float run = before;
     int claim = INT_MAX, lastpos = -1;
     for (int i = i0; i < i1; ++i) {
-      const float w = expf(zc(i) / P.T - ym);
-      if (w > 0.f) lastpos = i;
-      run += w;
+      const float wgt = expf(__ldcg(P.z_tok + tok_at(i)) / P.T - ym);
+      if (wgt > 0.f) lastpos = i;
+      run += wgt;
       if (run > target) {
         claim = i;
         break;
@@ -452,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_b1_kernel(const B1Params P
     __syncthreads();
     if (tid == 0) {
       const int idx = misc->claim != INT_MAX ? misc->claim : misc->lastpos;
-      P.out_tokens[0] = __ldg(P.C2T + static_cast<size_t>(ssel[idx / b]) * b + idx % b);
+      P.out_tokens[0] = tok_at(idx);
       if (P.out_max_logit) P.out_max_logit[0] = best_logit(bw);
     }
   }

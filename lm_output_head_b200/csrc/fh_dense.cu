@@ -1,102 +1,58 @@
 // Dense comparison head z = E h with a fused argmax (FlashHead write-up,
 // section 1.1: the classification head as one v x d matrix product).
 //
-// One persistent launch of one 512-thread CTA per SM: the v token rows are
-// spread round-robin over all warps, each streamed HBM -> shared memory once
-// with cp.async.bulk through a per-warp ring and dotted with every hidden row
-// of the launch. For B = 1 the hidden state lives in registers; otherwise the
-// block of hidden rows lives in shared memory. Per-row maxima are packed
-// (logit, token) words, merged per CTA and then with one 64-bit atomicMax;
-// the last CTA to finish writes the argmax and clears the accumulators.
+// One persistent launch, two 512-thread CTAs per SM: the v token rows are
+// spread round-robin over all warps; a warp streams a row HBM -> registers
+// with non-allocating 16-byte loads and dots it with every hidden row of the
+// launch, staged once per CTA in shared memory as fp32. Per-row maxima are
+// packed (logit, token) words, merged per CTA and then with one 64-bit
+// atomicMax; the last CTA to finish writes the argmax and clears the
+// accumulators.
 #include "fh_device.cuh"
 
 namespace fh {
 namespace {
 
-constexpr int kDenseMaxRows = 32;
+constexpr int kDenseMaxRows = 8;
 
-template <int NCH, bool ONE>
-__global__ void __launch_bounds__(kThreads, 1) dense_kernel(const DenseParams P) {
+template <int NCH>
+__global__ void __launch_bounds__(kThreads, 2) dense_kernel(const DenseParams P) {
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ unsigned long long wbest[kWarps][kDenseMaxRows];
   __shared__ int s_last;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = gridDim.x, W = G * kWarps, gw = blockIdx.x * kWarps + warp;
   const int d = P.d, R = P.rows;
-  uint16_t* sh = reinterpret_cast<uint16_t*>(smem + P.off_h);
-  const uint32_t sh_a = smem_addr(sh);
-  const uint32_t ring_w = smem_addr(smem + P.off_ring) + static_cast<uint32_t>(warp * P.nslot * P.slot_bytes);
-  const uint32_t bar_w = smem_addr(smem + P.off_bar) + static_cast<uint32_t>(warp * P.nslot * 8);
+  float* hs = reinterpret_cast<float*>(smem);  // [R][d]
 
-  const int n = gw < P.v ? (P.v - 1 - gw) / W + 1 : 0;
-  uint32_t phase_bits = 0;
-  auto src = [&](int i, const void*& ptr, uint32_t& bytes) {
-    ptr = P.E + static_cast<size_t>(gw + i * W) * d;
-    bytes = static_cast<uint32_t>(d * 2);
-  };
-  // first copies go out before the hidden rows are staged
-  warp_ring_init(bar_w, P.nslot);
-  warp_stream_prologue(n, P.nslot, ring_w, P.slot_bytes, bar_w, src);
-  const uint4* hsrc = reinterpret_cast<const uint4*>(P.hidden + static_cast<size_t>(P.row0) * d);
-  for (int i = tid; i < R * d / 8; i += kThreads) reinterpret_cast<uint4*>(sh)[i] = hsrc[i];
+  uint4 w[NCH];
+  if (gw < P.v) row_load_bf16<NCH>(P.E + static_cast<size_t>(gw) * d, d, w);  // first row goes out first
+  for (int r = 0; r < R; ++r) stage_h_f32(P.hidden + static_cast<size_t>(P.row0 + r) * d, d, hs + r * d);
   for (int i = tid; i < kWarps * kDenseMaxRows; i += kThreads) (&wbest[0][0])[i] = 0ull;
   __syncthreads();
-  bool ok;
-  if constexpr (ONE) {
-    float hr[NCH * 8];
-    load_h_chunks<NCH>(sh, d, hr);
-    unsigned long long best = 0ull;
-    auto use = [&](int i, uint32_t slot) {
-      const int t = gw + i * W;
-      const float z = row_dot_bf16<NCH>(slot, d, hr);
-      const unsigned long long pk = pack_best(z, t);
-      best = pk > best ? pk : best;
-      if (lane == 0 && P.logits) P.logits[static_cast<size_t>(P.row0) * P.v + t] = z;
-    };
-    ok = warp_stream_run(n, P.nslot, ring_w, P.slot_bytes, bar_w, phase_bits, kWaitBudget, src, use);
-    if (lane == 0) wbest[warp][0] = best;
-  } else {
-    auto use = [&](int i, uint32_t slot) {
-      const int t = gw + i * W;
-      uint4 ew[NCH];
+
+  unsigned long long best[kDenseMaxRows];
 #pragma unroll
-      for (int m = 0; m < NCH; ++m) {
-        const int e = (lane + 32 * m) * 8;
-        ew[m] = e < d ? lds128(slot + 2u * e) : make_uint4(0, 0, 0, 0);
-      }
-      for (int r = 0; r < R; ++r) {
-        const uint32_t hrow = sh_a + static_cast<uint32_t>(r * d * 2);
-        float acc = 0.f;
+  for (int r = 0; r < kDenseMaxRows; ++r) best[r] = 0ull;
+  for (int t = gw; t < P.v; t += W) {
+    if (t != gw) row_load_bf16<NCH>(P.E + static_cast<size_t>(t) * d, d, w);
 #pragma unroll
-        for (int m = 0; m < NCH; ++m) {
-          const int e = (lane + 32 * m) * 8;
-          if (e < d) {
-            const uint4 hv = lds128(hrow + 2u * e);
-            acc = fmaf(bf16lo(ew[m].x), bf16lo(hv.x), acc);
-            acc = fmaf(bf16hi(ew[m].x), bf16hi(hv.x), acc);
-            acc = fmaf(bf16lo(ew[m].y), bf16lo(hv.y), acc);
-            acc = fmaf(bf16hi(ew[m].y), bf16hi(hv.y), acc);
-            acc = fmaf(bf16lo(ew[m].z), bf16lo(hv.z), acc);
-            acc = fmaf(bf16hi(ew[m].z), bf16hi(hv.z), acc);
-            acc = fmaf(bf16lo(ew[m].w), bf16lo(hv.w), acc);
-            acc = fmaf(bf16hi(ew[m].w), bf16hi(hv.w), acc);
-          }
-        }
-        const float z = warp_sum(acc);
-        if (lane == 0) {
-          const unsigned long long pk = pack_best(z, t);
-          if (pk > wbest[warp][r]) wbest[warp][r] = pk;
-          if (P.logits) P.logits[static_cast<size_t>(P.row0 + r) * P.v + t] = z;
-        }
+    for (int r = 0; r < kDenseMaxRows; ++r) {
+      if (r < R) {
+        const float z = row_dot_bf16_hs<NCH>(w, hs + r * d, d);
+        const unsigned long long pk = pack_best(z, t);
+        best[r] = pk > best[r] ? pk : best[r];
+        if (lane == 0 && P.logits) P.logits[static_cast<size_t>(P.row0 + r) * P.v + t] = z;
       }
-    };
-    ok = warp_stream_run(n, P.nslot, ring_w, P.slot_bytes, bar_w, phase_bits, kWaitBudget, src, use);
+    }
   }
-  if (!ok && lane == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
+  if (lane == 0)
+#pragma unroll
+    for (int r = 0; r < kDenseMaxRows; ++r) wbest[warp][r] = best[r];
   __syncthreads();
   for (int r = tid; r < R; r += kThreads) {
     unsigned long long m = 0ull;
-    for (int w = 0; w < kWarps; ++w) m = wbest[w][r] > m ? wbest[w][r] : m;
+    for (int i = 0; i < kWarps; ++i) m = wbest[i][r] > m ? wbest[i][r] : m;
     if (m) atomicMax(P.best + P.row0 + r, m);
   }
   __syncthreads();
@@ -118,10 +74,8 @@ __global__ void __launch_bounds__(kThreads, 1) dense_kernel(const DenseParams P)
 
 cudaError_t launch_dense(const DenseParams& P, int grid, size_t smem, int nch, cudaStream_t st) {
   if (P.rows > kDenseMaxRows) return cudaErrorInvalidValue;
-  const bool one = P.rows == 1;
-#define FH_L(N)                                                       \
-  if (one) dense_kernel<N, true><<<grid, kThreads, smem, st>>>(P);    \
-  else dense_kernel<N, false><<<grid, kThreads, smem, st>>>(P);       \
+#define FH_L(N)                                                    \
+  dense_kernel<N><<<grid, kThreads, smem, st>>>(P);                \
   return cudaGetLastError();
   switch (nch) {
     case 1: FH_L(1)
@@ -139,16 +93,33 @@ cudaError_t launch_dense(const DenseParams& P, int grid, size_t smem, int nch, c
 
 int dense_max_rows() { return kDenseMaxRows; }
 
+cudaError_t occupancy_dense(int nch, size_t smem, int* blocks) {
+  switch (nch) {
+    case 1: return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, dense_kernel<1>, kThreads, smem);
+    case 2: return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, dense_kernel<2>, kThreads, smem);
+    case 3: return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, dense_kernel<3>, kThreads, smem);
+    case 4: return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, dense_kernel<4>, kThreads, smem);
+    case 5: return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, dense_kernel<5>, kThreads, smem);
+    case 6: return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, dense_kernel<6>, kThreads, smem);
+    case 8: return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, dense_kernel<8>, kThreads, smem);
+    case 10: return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, dense_kernel<10>, kThreads, smem);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 cudaError_t set_attrs_dense(int max_smem) {
   cudaError_t e = cudaSuccess;
   auto set = [&](const void* f) {
     if (e == cudaSuccess) e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
   };
-#define FH_S(N)                                                   \
-  set(reinterpret_cast<const void*>(dense_kernel<N, true>));      \
-  set(reinterpret_cast<const void*>(dense_kernel<N, false>));
-  FH_S(1) FH_S(2) FH_S(3) FH_S(4) FH_S(5) FH_S(6) FH_S(8) FH_S(10)
-#undef FH_S
+  set(reinterpret_cast<const void*>(dense_kernel<1>));
+  set(reinterpret_cast<const void*>(dense_kernel<2>));
+  set(reinterpret_cast<const void*>(dense_kernel<3>));
+  set(reinterpret_cast<const void*>(dense_kernel<4>));
+  set(reinterpret_cast<const void*>(dense_kernel<5>));
+  set(reinterpret_cast<const void*>(dense_kernel<6>));
+  set(reinterpret_cast<const void*>(dense_kernel<8>));
+  set(reinterpret_cast<const void*>(dense_kernel<10>));
   return e;
 }
 

@@ -28,7 +28,7 @@ struct SyncWords {
 
 struct B1Params {
   const uint16_t* E;
-  const uint8_t* Crows;   // bf16 rows (d*2 bytes) or packed INT4 rows (rs bytes)
+  const uint8_t* Crows;   // bf16 rows (d*2 bytes) or packed INT4 rows (crow_bytes)
   const int32_t* C2T;
   const uint16_t* hidden;
   const float* u_clusters;
@@ -36,22 +36,22 @@ struct B1Params {
   int32_t* out_tokens;
   int32_t* out_cluster_ids;
   float* out_max_logit;
-  float* scores;          // workspace [c] keys (read only by the tie fallback)
-  float* z_slot;          // workspace [v]: logit of slot k*b + j (sampling)
+  uint32_t* keys;         // workspace [c]: order-preserving keys (read only by the tie fallback)
+  float* z_tok;           // workspace [v]: candidate logits by token id (sampling)
   // per-call state, two buffers used by alternate calls
   uint32_t* hist_hi;      // [2][256]   histogram of key >> 24
   uint32_t* hist_lo;      // [2][4096]  histogram of key >> 20
   uint32_t* bitmap;       // [2][words] selected clusters
   unsigned long long* bnd_list;  // [2][2048] boundary (key << 32 | id)
-  uint32_t* bnd_count;    // [2]
+  uint32_t* counts;       // [2][2]     boundary count, row-queue count
+  int32_t* row_queue;     // [2][nc_max] token id of candidate slot, -1 until written
   unsigned long long* best;
   SyncWords* sync;
-  int v, d, c, b, p, words;
-  int crow_bytes;         // bytes per centroid row in Crows
+  int v, d, c, b, p, words, nc_max;
+  int crow_bytes;
   int mode;
   float T;
-  int nslot, slot_bytes;
-  int off_h, off_bar, off_sel, off_misc, off_ring;
+  int off_h, off_sel, off_misc, off_scratch;
   long long spin_budget;
 };
 
