@@ -17,6 +17,7 @@ int dense_max_rows();
 cudaError_t occupancy_decode_b1(int int4, int nch, size_t smem, int* blocks);
 size_t decode_b1_misc_bytes();
 cudaError_t occupancy_dense(int nch, size_t smem, int* blocks);
+size_t decode_b1_bar_words();
 }  // namespace fh
 
 using namespace fh;
@@ -38,8 +39,8 @@ struct fh_head {
   uint32_t* c2t_counts = nullptr;      // [v]
   uint32_t* b1_keys = nullptr;         // fused B = 1 state
   float* b1_z_tok = nullptr;
-  uint32_t* b1_hist_hi = nullptr;
-  uint32_t* b1_hist_lo = nullptr;
+  uint32_t* b1_hist = nullptr;
+  uint32_t* b1_bars = nullptr;
   uint32_t* b1_bitmap = nullptr;
   unsigned long long* b1_bnd = nullptr;
   uint32_t* b1_counts = nullptr;
@@ -246,8 +247,8 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   const int words = (D.c + 31) / 32;
   const size_t o_keys1 = take(static_cast<size_t>(D.c) * 4);
   const size_t o_ztok = take(static_cast<size_t>(D.v) * 4);
-  const size_t o_hhi = take(2 * 256 * 4);
   const size_t o_hlo = take(2 * kHistBins * 4);
+  const size_t o_bars = take(decode_b1_bar_words() * 4);
   const size_t o_bmp = take(2 * static_cast<size_t>(words) * 4);
   const size_t o_bnd = take(2 * kBoundaryMax * 8);
   const size_t o_bcnt = take(4 * 4);
@@ -275,8 +276,8 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   h->c2t_counts = reinterpret_cast<uint32_t*>(h->ws + o_cnt);
   h->b1_keys = reinterpret_cast<uint32_t*>(h->ws + o_keys1);
   h->b1_z_tok = reinterpret_cast<float*>(h->ws + o_ztok);
-  h->b1_hist_hi = reinterpret_cast<uint32_t*>(h->ws + o_hhi);
-  h->b1_hist_lo = reinterpret_cast<uint32_t*>(h->ws + o_hlo);
+  h->b1_hist = reinterpret_cast<uint32_t*>(h->ws + o_hlo);
+  h->b1_bars = reinterpret_cast<uint32_t*>(h->ws + o_bars);
   h->b1_bitmap = reinterpret_cast<uint32_t*>(h->ws + o_bmp);
   h->b1_bnd = reinterpret_cast<unsigned long long*>(h->ws + o_bnd);
   h->b1_counts = reinterpret_cast<uint32_t*>(h->ws + o_bcnt);
@@ -334,8 +335,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
     h->b1_off_misc = static_cast<int>(o);
     o += up(decode_b1_misc_bytes(), 128);
     h->b1_off_scratch = static_cast<int>(o);
-    o += up(std::max(std::max(static_cast<size_t>(kHistBins) * 4, static_cast<size_t>(kBoundaryMax) * 8),
-                     sizeof(SelectSmem)), 128);
+    o += up(sizeof(SelectSmem), 128);
     h->b1_smem = o;
     int blocks = 0;
     e = occupancy_decode_b1(D.fmt == FH_CENTROID_INT4_G32, h->nch, h->b1_smem, &blocks);
@@ -482,8 +482,8 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
     P.out_max_logit = out_max_logit;
     P.keys = h->b1_keys;
     P.z_tok = h->b1_z_tok;
-    P.hist_hi = h->b1_hist_hi;
-    P.hist_lo = h->b1_hist_lo;
+    P.hist = h->b1_hist;
+    P.bars = h->b1_bars;
     P.bitmap = h->b1_bitmap;
     P.bnd_list = h->b1_bnd;
     P.counts = h->b1_counts;

@@ -10,21 +10,23 @@
 //     cluster k belongs to global warp k mod W, which streams its centroid
 //     row and computes the key -- the score, or when sampling the Gumbel key
 //     s/T - ln(-ln u) (section 1.2.3). The key stays in a lane register of the
-//     owning warp and is counted into two device-wide histograms of its top 8
-//     and top 12 bits (fire-and-forget atomics).
-//  2. device-wide barrier; each CTA reads the histograms once and finds the
-//     12-bit bin t1 holding the p-th largest key. Keys above t1 are selected;
-//     keys inside t1 form the boundary. Owners publish the b token ids of
-//     each selected cluster (the C2T row, section 1.2.1: slot k*b + j holds
-//     token C2T[k][j]) into a device-wide row queue.
-//  3. the candidate rows are spread round-robin over every warp of the grid:
-//     a warp polls its queue slot for the token id, streams the token row and
+//     owning warp and is counted into a device-wide histogram of its top 12
+//     bits (fire-and-forget atomics).
+//  2. device-wide barrier; each CTA scans the histogram once and finds the
+//     bin t1 holding the p-th largest key. Keys above t1 are selected; keys
+//     inside t1 form the boundary. Owners publish the b token ids of each
+//     selected cluster (its C2T row, section 1.2.1: slot k*b + j holds token
+//     C2T[k][j]) into a device-wide row queue, and the boundary keys into a
+//     small list.
+//  3. candidate rows are spread round-robin over every warp of the grid: a
+//     warp polls its queue slot for the token id, streams the token row and
 //     keeps a packed (logit, token) maximum (section 1.2.4, stage 2).
-//  4. only when the boundary bin is split (some but not all of its keys are
-//     needed): owners published their boundary keys to a small list; after a
-//     second barrier each owner ranks its boundary keys exactly (key desc, id
-//     asc) against the list and queues the chosen clusters' rows, which the
-//     consumers pick up as in step 3.
+//  4. when the boundary bin is split (some but not all of its keys needed),
+//     a warp that owns boundary keys ranks them exactly (key desc, id asc)
+//     against the list as soon as a second barrier says the list is
+//     complete -- checked inside its polling loop, so no wait can deadlock --
+//     and queues the chosen clusters, whose rows the consumers pick up as in
+//     step 3.
 //  5. CTA maxima meet in one 64-bit atomicMax; the last CTA to finish (exit
 //     ticket) writes the token: the argmax, or, when sampling, the inverse-CDF
 //     draw over softmax(z/T) in canonical order (cluster asc, slot asc),
@@ -32,6 +34,8 @@
 //
 // No CTA ever reads all c keys, and HBM traffic is the algorithmic minimum:
 // each centroid row once, each selected token row once, plus C2T rows and h.
+// Device-wide counters are spread over 8 cache lines so that arrivals do not
+// serialise on one address.
 #include <climits>
 
 #include "fh_device.cuh"
@@ -39,7 +43,8 @@
 namespace fh {
 namespace {
 
-constexpr int kHiBins = 256;
+constexpr int kBarLanes = 8;       // counters per device-wide barrier
+constexpr int kBarStride = 32;     // words between counters (one 128-byte line each)
 
 struct B1Misc {
   unsigned long long wbest[kWarps];
@@ -47,16 +52,32 @@ struct B1Misc {
   uint32_t uscan[kWarps + 1];
   int claim, lastpos, ok, last;
   uint32_t t1, need, split, fallback, n_sure;
+  uint32_t cta_sure, qbase;
 };
 
-// Device-wide barrier over the cooperative grid; false if `budget` cycles pass first.
-__device__ bool grid_wait(uint32_t* counter, uint32_t target, long long budget, int* flag) {
+__device__ __forceinline__ void bar_arrive(uint32_t* bar) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(bar + (blockIdx.x % kBarLanes) * kBarStride, 1u);
+  }
+}
+
+__device__ __forceinline__ uint32_t bar_count(const uint32_t* bar) {
+  uint32_t s = 0;
+#pragma unroll
+  for (int i = 0; i < kBarLanes; ++i) s += ld_acquire_u32(bar + i * kBarStride);
+  return s;
+}
+
+// All CTAs wait until `target` arrivals; false if `budget` cycles pass first.
+__device__ bool bar_wait(const uint32_t* bar, uint32_t target, long long budget, int* flag) {
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
-    if (ld_acquire_u32(counter) < target) {
+    if (bar_count(bar) < target) {
       const long long t0 = clock64();
-      while (ld_acquire_u32(counter) < target) {
+      while (bar_count(bar) < target) {
         if (clock64() - t0 > budget) {
           ok = 0;
           break;
@@ -70,75 +91,51 @@ __device__ bool grid_wait(uint32_t* counter, uint32_t target, long long budget, 
   return *flag != 0;
 }
 
-__device__ __forceinline__ void grid_arrive(uint32_t* counter) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(counter, 1u);
-  }
-}
-
-__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x) {
+// Queue the b token ids of cluster k at row-queue position pos (one warp).
+__device__ __forceinline__ void queue_cluster(const B1Params& P, int32_t* rq, uint32_t* bitmap, uint32_t pos,
+                                              int k) {
   const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
-    if (lane >= o) x += y;
-  }
-  return x;
-}
-
-// Poll a row-queue slot until an owner has written the token id (bounded).
-__device__ __forceinline__ int poll_token(const int32_t* slot, long long budget) {
-  int t = static_cast<int>(ld_acquire_u32(reinterpret_cast<const unsigned*>(slot)));
-  if (t >= 0) return t;
-  const long long t0 = clock64();
-  while ((t = static_cast<int>(ld_acquire_u32(reinterpret_cast<const unsigned*>(slot)))) < 0) {
-    if (clock64() - t0 > budget) return -1;
-  }
-  return t;
-}
-
-// Queue the b token rows of cluster k (one warp): slots pos*b .. pos*b + b - 1.
-__device__ __forceinline__ void publish_cluster(const B1Params& P, int32_t* rq, uint32_t* qcount, uint32_t* bitmap,
-                                                int k) {
-  const int lane = threadIdx.x & 31;
-  uint32_t pos = 0;
-  if (lane == 0) {
-    pos = atomicAdd(qcount, 1u);
-    atomicOr(bitmap + (k >> 5), 1u << (k & 31));
-  }
-  pos = __shfl_sync(0xFFFFFFFFu, pos, 0);
+  if (lane == 0) atomicOr(bitmap + (k >> 5), 1u << (k & 31));
   if (pos >= static_cast<uint32_t>(P.p)) return;  // only an inconsistent histogram could overfill the queue
   for (int j = lane; j < P.b; j += 32)
     rq[static_cast<size_t>(pos) * P.b + j] = __ldg(P.C2T + static_cast<size_t>(k) * P.b + j);
 }
 
-// Consume candidate rows r = r0 + gw + i*W (< r1) of the row queue.
-template <int NCH>
-__device__ __forceinline__ void consume_rows(const B1Params& P, const int32_t* rq, const int32_t* ssel, bool direct,
-                                             int r0, int r1, int gw, int W, const float* hs,
-                                             unsigned long long& best, bool gumbel, bool& ok) {
+// Exact rank of each of this warp's boundary keys (lanes set in `mine`)
+// against the published boundary list; the chosen clusters are queued.
+__device__ void rank_boundary(const B1Params& P, int32_t* rq, uint32_t* bitmap, uint32_t* qcount,
+                              const unsigned long long* bnd_list, const uint32_t* bnd_count, uint32_t mine,
+                              uint32_t own_key, int gw, int W, uint32_t need) {
   const int lane = threadIdx.x & 31;
-  for (int r = r0 + gw; r < r1; r += W) {
-    int t;
-    if (direct) {
-      t = __ldg(P.C2T + static_cast<size_t>(ssel[r / P.b]) * P.b + r % P.b);
-    } else {
-      t = 0;
-      if (lane == 0) t = poll_token(rq + r, P.spin_budget);
-      t = __shfl_sync(0xFFFFFFFFu, t, 0);
-      if (t < 0) {
-        ok = false;
-        continue;
+  const uint32_t nb = min(__ldcg(bnd_count), static_cast<uint32_t>(kBoundaryMax));
+  while (mine) {
+    const int j = __ffs(mine) - 1;
+    mine &= mine - 1;
+    const uint32_t kq = __shfl_sync(0xFFFFFFFFu, own_key, j);
+    const int idq = gw + j * W;
+    uint32_t r = 0;
+    for (uint32_t e0 = 0; e0 < nb; e0 += 128) {
+      unsigned long long v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t e = e0 + lane + 32 * u;
+        v[u] = e < nb ? __ldcg(bnd_list + e) : 0ull;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t e = e0 + lane + 32 * u;
+        const uint32_t ke = static_cast<uint32_t>(v[u] >> 32);
+        r += e < nb && ((ke > kq) || (ke == kq && static_cast<int>(v[u] & 0xFFFFFFFFu) < idq));
       }
     }
-    uint4 w[NCH];
-    row_load_bf16<NCH>(P.E + static_cast<size_t>(t) * P.d, P.d, w);
-    const float z = row_dot_bf16_hs<NCH>(w, hs, P.d);
-    const unsigned long long pk = pack_best(z, t);
-    best = pk > best ? pk : best;
-    if (gumbel && lane == 0) P.z_tok[t] = z;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xFFFFFFFFu, r, o);
+    if (r < need) {
+      uint32_t pos = 0;
+      if (lane == 0) pos = atomicAdd(qcount, 1u);
+      pos = __shfl_sync(0xFFFFFFFFu, pos, 0);
+      queue_cluster(P, rq, bitmap, pos, idq);
+    }
   }
 }
 
@@ -177,40 +174,57 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   float* hs = reinterpret_cast<float*>(smem + P.off_h);
   int32_t* ssel = reinterpret_cast<int32_t*>(smem + P.off_sel);
   B1Misc* misc = reinterpret_cast<B1Misc*>(smem + P.off_misc);
-  uint8_t* scratch = smem + P.off_scratch;  // histogram copy, boundary list, or fallback select state
+  uint8_t* scratch = smem + P.off_scratch;  // fallback select state
 
   // per-call state: two buffers used by alternate calls; this call clears the other one
   const uint32_t epoch = P.sync->epoch;
   const uint32_t par = epoch & 1u, nxt = par ^ 1u;
-  uint32_t* hist_hi = P.hist_hi + par * kHiBins;
-  uint32_t* hist_lo = P.hist_lo + par * kHistBins;
+  uint32_t* hist = P.hist + par * kHistBins;
   uint32_t* bitmap = P.bitmap + par * P.words;
   unsigned long long* bnd_list = P.bnd_list + par * kBoundaryMax;
   uint32_t* bnd_count = P.counts + 2 * par;
   uint32_t* qcount = P.counts + 2 * par + 1;
   int32_t* rq = P.row_queue + static_cast<size_t>(par) * P.nc_max;
+  uint32_t* bar1 = P.bars;
+  uint32_t* bar2 = P.bars + kBarLanes * kBarStride;
 
   // ---------------- phase 1: centroid scores ----------------
+  // h goes out first (every CTA needs it before its first dot), then the
+  // warp's first centroid row, then h is converted into shared memory.
+  uint4 hraw = make_uint4(0, 0, 0, 0);
+  if (tid < d / 8) hraw = *reinterpret_cast<const uint4*>(P.hidden + 8 * tid);
   const int n1 = gw < P.c ? (P.c - 1 - gw) / W + 1 : 0;  // <= 32 (host-checked)
   constexpr int NQ = (NCH + 1) / 2;
   uint4 w[NCH];
   uint2 q[NQ];
   uint32_t sc[NQ];
-  if (n1 > 0) {  // the first centroid row goes out before anything else
+  if (n1 > 0) {
     if constexpr (INT4) row_load_int4<NQ>(P.Crows + static_cast<size_t>(gw) * P.crow_bytes, d, q, sc);
     else row_load_bf16<NCH>(reinterpret_cast<const uint16_t*>(P.Crows + static_cast<size_t>(gw) * P.crow_bytes), d, w);
   }
   float ureg = 0.f;  // lane j holds u of item j
   if (gumbel && lane < n1) ureg = __ldg(P.u_clusters + gw + lane * W);
-  stage_h_f32(P.hidden, d, hs);
+  if (tid < d / 8) {
+    float4 a, c4;
+    a.x = bf16lo(hraw.x); a.y = bf16hi(hraw.x); a.z = bf16lo(hraw.y); a.w = bf16hi(hraw.y);
+    c4.x = bf16lo(hraw.z); c4.y = bf16hi(hraw.z); c4.z = bf16lo(hraw.w); c4.w = bf16hi(hraw.w);
+    reinterpret_cast<float4*>(hs)[2 * tid] = a;
+    reinterpret_cast<float4*>(hs)[2 * tid + 1] = c4;
+  }
+  for (int i = tid + kThreads; i < d / 8; i += kThreads) {  // d > 4096 only
+    const uint4 x = *reinterpret_cast<const uint4*>(P.hidden + 8 * i);
+    float4 a, c4;
+    a.x = bf16lo(x.x); a.y = bf16hi(x.x); a.z = bf16lo(x.y); a.w = bf16hi(x.y);
+    c4.x = bf16lo(x.z); c4.y = bf16hi(x.z); c4.z = bf16lo(x.w); c4.w = bf16hi(x.w);
+    reinterpret_cast<float4*>(hs)[2 * i] = a;
+    reinterpret_cast<float4*>(hs)[2 * i + 1] = c4;
+  }
   {
-    const int nz = kHiBins + kHistBins + P.words + 2 + P.nc_max;
+    const int nz = kHistBins + P.words + 2 + P.nc_max;
     const int per = (nz + G - 1) / G;
     for (int i = tid; i < per; i += kThreads) {
       int z = blockIdx.x * per + i;
-      if (z < kHiBins) { P.hist_hi[nxt * kHiBins + z] = 0u; continue; }
-      z -= kHiBins;
-      if (z < kHistBins) { P.hist_lo[nxt * kHistBins + z] = 0u; continue; }
+      if (z < kHistBins) { P.hist[nxt * kHistBins + z] = 0u; continue; }
       z -= kHistBins;
       if (z < P.words) { P.bitmap[nxt * P.words + z] = 0u; continue; }
       z -= P.words;
@@ -219,6 +233,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
       if (z < P.nc_max) P.row_queue[static_cast<size_t>(nxt) * P.nc_max + z] = -1;
     }
   }
+  if (tid == 0) misc->cta_sure = 0u;
   __syncthreads();
 
   uint32_t own_key = 0u;  // lane j: key of the warp's item j
@@ -238,84 +253,75 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     if (lane == (i & 31)) own_key = kk;
     if (lane == 0) {
       P.keys[k] = kk;
-      atomicAdd(hist_hi + (kk >> 24), 1u);
-      atomicAdd(hist_lo + (kk >> kHistShift), 1u);
+      atomicAdd(hist + (kk >> kHistShift), 1u);
       prefetch_l2(P.C2T + static_cast<size_t>(k) * b);
     }
   }
 
   // ---------------- phase 2: barrier, boundary bin, owners publish ----------------
-  grid_arrive(&P.sync->arrive);
-  const bool passed = grid_wait(&P.sync->arrive, static_cast<uint32_t>(G), P.spin_budget, &misc->ok);
+  bar_arrive(bar1);
+  const bool passed = bar_wait(bar1, static_cast<uint32_t>(G), P.spin_budget, &misc->ok);
   unsigned long long best = 0ull;
   bool ok = true;
   if (!passed) {
     if (tid == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
   } else {
     const uint32_t p = static_cast<uint32_t>(P.p);
-    uint32_t* hlo = reinterpret_cast<uint32_t*>(scratch);
-    uint32_t hv[8];
-    if (warp == 0) {
+    {
+      // bin t1 of the p-th largest key: thread t owns bins 4095-8t .. 4088-8t
+      constexpr int kBpt = kHistBins / kThreads;
+      uint32_t hv[kBpt], loc = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) hv[i] = __ldcg(hist_hi + kHiBins - 1 - 8 * lane - i);
-    }
-    for (int i = tid; i < kHistBins; i += kThreads) hlo[i] = __ldcg(hist_lo + i);
-    __syncthreads();
-    if (warp == 0) {
-      // top-8-bit bins, descending: lane l owns bins 255-8l .. 248-8l
-      uint32_t s = 0;
+      for (int i = 0; i < kBpt; ++i) {
+        hv[i] = __ldcg(hist + kHistBins - 1 - kBpt * tid - i);
+        loc += hv[i];
+      }
+      const uint32_t above = block_exclusive_scan<kThreads, uint32_t>(loc, misc->uscan, nullptr);
+      uint32_t run = above;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) s += hv[i];
-      const uint32_t incl = warp_incl_scan(s), excl = incl - s;
-      const int L = __ffs(__ballot_sync(0xFFFFFFFFu, excl < p && p <= incl)) - 1;
-      uint32_t thi = 0, above_hi = 0, run = excl;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < kBpt; ++i) {
         if (run < p && run + hv[i] >= p) {
-          thi = kHiBins - 1 - 8 * lane - i;
-          above_hi = run;
+          const uint32_t need = p - run;
+          misc->t1 = static_cast<uint32_t>(kHistBins - 1 - kBpt * tid - i);
+          misc->need = need;
+          misc->split = hv[i] != need ? 1u : 0u;
+          misc->fallback = (hv[i] != need && hv[i] > static_cast<uint32_t>(kBoundaryMax)) ? 1u : 0u;
+          misc->n_sure = hv[i] != need ? run : p;
         }
         run += hv[i];
       }
-      thi = __shfl_sync(0xFFFFFFFFu, thi, L);
-      above_hi = __shfl_sync(0xFFFFFFFFu, above_hi, L);
-      // its 16 sub-bins of 12 bits, descending
-      const uint32_t x = lane < 16 ? hlo[thi * 16 + 15 - lane] : 0u;
-      const uint32_t incl2 = warp_incl_scan(x), excl2 = incl2 - x;
-      const uint32_t target = p - above_hi;
-      const int L2 = __ffs(__ballot_sync(0xFFFFFFFFu, lane < 16 && excl2 < target && target <= incl2)) - 1;
-      const uint32_t ex2 = __shfl_sync(0xFFFFFFFFu, excl2, L2);
-      const uint32_t m1 = __shfl_sync(0xFFFFFFFFu, x, L2);
-      if (lane == 0) {
-        const uint32_t need = target - ex2;
-        misc->t1 = thi * 16 + 15 - L2;
-        misc->need = need;
-        misc->split = m1 != need ? 1u : 0u;
-        misc->fallback = (m1 != need && m1 > static_cast<uint32_t>(kBoundaryMax)) ? 1u : 0u;
-        misc->n_sure = m1 != need ? p - need : p;
-      }
     }
     __syncthreads();
-    const uint32_t t1 = misc->t1;
+    const uint32_t t1 = misc->t1, need = misc->need;
     const bool split = misc->split != 0, fallback = misc->fallback != 0;
     const int r_sure = static_cast<int>(misc->n_sure) * b, r_all = P.p * b;
+    const uint32_t dg = own_key >> kHistShift;
+    const bool mine = lane < n1;
+    uint32_t bnd_mine = 0u;
 
     if (!fallback) {
-      const uint32_t dg = own_key >> kHistShift;
-      const bool mine = lane < n1;
-      uint32_t sure = __ballot_sync(0xFFFFFFFFu, mine && (dg > t1 || (dg == t1 && !split)));
-      while (sure) {  // queue the rows of each selected cluster this warp owns
-        const int j = __ffs(sure) - 1;
-        sure &= sure - 1;
-        publish_cluster(P, rq, qcount, bitmap, gw + j * W);
+      // one queue reservation per CTA for its surely selected clusters
+      const uint32_t sure = __ballot_sync(0xFFFFFFFFu, mine && (dg > t1 || (dg == t1 && !split)));
+      uint32_t off = 0;
+      if (lane == 0 && sure) off = atomicAdd(&misc->cta_sure, static_cast<uint32_t>(__popc(sure)));
+      off = __shfl_sync(0xFFFFFFFFu, off, 0);
+      __syncthreads();
+      if (tid == 0) misc->qbase = misc->cta_sure ? atomicAdd(qcount, misc->cta_sure) : 0u;
+      __syncthreads();
+      uint32_t pos = misc->qbase + off, sm = sure;
+      while (sm) {
+        const int j = __ffs(sm) - 1;
+        sm &= sm - 1;
+        queue_cluster(P, rq, bitmap, pos++, gw + j * W);
       }
-      if (mine && split && dg == t1) {
+      bnd_mine = __ballot_sync(0xFFFFFFFFu, mine && split && dg == t1);
+      if (bnd_mine & (1u << lane)) {
         const uint32_t at = atomicAdd(bnd_count, 1u);
         if (at < static_cast<uint32_t>(kBoundaryMax))
           bnd_list[at] = (static_cast<unsigned long long>(own_key) << 32) | static_cast<uint32_t>(gw + lane * W);
       }
       __threadfence();
-      if (split) grid_arrive(&P.sync->arrive2);
+      if (split) bar_arrive(bar2);
     } else {
       // pathological ties (a boundary bin larger than the exact-rank list):
       // every CTA selects over all keys and reads its rows' tokens directly
@@ -324,40 +330,55 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
         for (int i = tid; i < P.p; i += kThreads) atomicOr(bitmap + (ssel[i] >> 5), 1u << (ssel[i] & 31));
     }
 
-    // ---------------- phase 3: candidate rows of the surely selected clusters ----------------
-    consume_rows<NCH>(P, rq, ssel, fallback, 0, fallback ? r_all : r_sure, gw, W, hs, best, gumbel, ok);
-
-    if (split && !fallback) {
-      // ---------------- phase 4: exact rank of boundary keys ----------------
-      const bool got = grid_wait(&P.sync->arrive2, static_cast<uint32_t>(G), P.spin_budget, &misc->ok);
-      if (!got) {
-        ok = false;
+    // ---------------- phases 3-4: consume candidate rows ----------------
+    bool ranked = bnd_mine == 0u;
+    const long long budget = P.spin_budget;
+    for (int r = gw; r < r_all; r += W) {
+      int t;
+      if (fallback) {
+        t = __ldg(P.C2T + static_cast<size_t>(ssel[r / b]) * b + r % b);
       } else {
-        unsigned long long* sl = reinterpret_cast<unsigned long long*>(scratch);
-        const uint32_t nb = min(__ldcg(bnd_count), static_cast<uint32_t>(kBoundaryMax));
-        for (uint32_t i = tid; i < nb; i += kThreads) sl[i] = __ldcg(bnd_list + i);
-        __syncthreads();
-        const uint32_t need = misc->need;
-        const uint32_t dg = own_key >> kHistShift;
-        uint32_t mine = __ballot_sync(0xFFFFFFFFu, lane < n1 && dg == t1);
-        while (mine) {
-          const int j = __ffs(mine) - 1;
-          mine &= mine - 1;
-          const uint32_t kq = __shfl_sync(0xFFFFFFFFu, own_key, j);
-          const int idq = gw + j * W;
-          uint32_t r = 0;
-          for (uint32_t e = lane; e < nb; e += 32) {
-            const unsigned long long v = sl[e];
-            const uint32_t ke = static_cast<uint32_t>(v >> 32);
-            r += (ke > kq) || (ke == kq && static_cast<int>(v & 0xFFFFFFFFu) < idq);
+        long long t0 = 0;
+        for (;;) {
+          if (!ranked) {  // publish this warp's boundary choices once the list is complete
+            uint32_t ready = 0;
+            if (lane == 0) ready = bar_count(bar2) >= static_cast<uint32_t>(G);
+            if (__shfl_sync(0xFFFFFFFFu, ready, 0)) {
+              rank_boundary(P, rq, bitmap, qcount, bnd_list, bnd_count, bnd_mine, own_key, gw, W, need);
+              ranked = true;
+            }
           }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xFFFFFFFFu, r, o);
-          if (r < need) publish_cluster(P, rq, qcount, bitmap, idq);
+          int v = 0;
+          if (lane == 0) v = static_cast<int>(ld_acquire_u32(reinterpret_cast<const unsigned*>(rq + r)));
+          t = __shfl_sync(0xFFFFFFFFu, v, 0);
+          if (t >= 0) break;
+          if (t0 == 0) t0 = clock64();
+          else if (clock64() - t0 > budget) break;
         }
-        __threadfence();
-        consume_rows<NCH>(P, rq, ssel, false, r_sure, r_all, gw, W, hs, best, gumbel, ok);
+        if (t < 0) {
+          ok = false;
+          continue;
+        }
       }
+      uint4 e[NCH];
+      row_load_bf16<NCH>(P.E + static_cast<size_t>(t) * d, d, e);
+      const float z = row_dot_bf16_hs<NCH>(e, hs, d);
+      const unsigned long long pk = pack_best(z, t);
+      best = pk > best ? pk : best;
+      if (gumbel && lane == 0) P.z_tok[t] = z;
+    }
+    if (!ranked) {  // no rows left to poll on: wait for the list, then publish
+      long long t0 = clock64();
+      uint32_t ready = 0;
+      for (;;) {
+        if (lane == 0) ready = bar_count(bar2) >= static_cast<uint32_t>(G);
+        if (__shfl_sync(0xFFFFFFFFu, ready, 0)) break;
+        if (clock64() - t0 > budget) break;
+      }
+      if (__shfl_sync(0xFFFFFFFFu, ready, 0))
+        rank_boundary(P, rq, bitmap, qcount, bnd_list, bnd_count, bnd_mine, own_key, gw, W, need);
+      else
+        ok = false;
     }
     if (!ok && lane == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
   }
@@ -429,14 +450,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
       if (P.out_max_logit) P.out_max_logit[0] = best_logit(bw);
     }
   }
+  if (tid < 2 * kBarLanes) P.bars[tid * kBarStride] = 0u;
   if (tid == 0) {
     *P.best = 0ull;
-    P.sync->arrive = 0u;
-    P.sync->arrive2 = 0u;
     P.sync->ticket = 0u;
     P.sync->epoch = epoch + 1u;
-    __threadfence();
   }
+  __threadfence();
 }
 
 template <int NCH>
@@ -458,6 +478,7 @@ cudaError_t launch_nch(const B1Params& P, int grid, size_t smem, int int4, cudaS
 }  // namespace
 
 size_t decode_b1_misc_bytes() { return sizeof(B1Misc); }
+size_t decode_b1_bar_words() { return 2 * kBarLanes * kBarStride; }
 
 cudaError_t launch_decode_b1(const B1Params& P, int grid, size_t smem, int int4, int nch, cudaStream_t st) {
   switch (nch) {

@@ -39,8 +39,8 @@ struct B1Params {
   uint32_t* keys;         // workspace [c]: order-preserving keys (read only by the tie fallback)
   float* z_tok;           // workspace [v]: candidate logits by token id (sampling)
   // per-call state, two buffers used by alternate calls
-  uint32_t* hist_hi;      // [2][256]   histogram of key >> 24
-  uint32_t* hist_lo;      // [2][4096]  histogram of key >> 20
+  uint32_t* hist;         // [2][4096]  histogram of key >> 20
+  uint32_t* bars;         // two device-wide barriers, 8 counters each, one per 128-byte line
   uint32_t* bitmap;       // [2][words] selected clusters
   unsigned long long* bnd_list;  // [2][2048] boundary (key << 32 | id)
   uint32_t* counts;       // [2][2]     boundary count, row-queue count
