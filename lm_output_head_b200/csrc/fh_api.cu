@@ -202,7 +202,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   } else {
     return FH_ERR_INVALID_ARG;
   }
-  if (D.d > kMaxD) return FH_ERR_UNSUPPORTED;
+  if (D.d > kMaxD) return FH_ERR_UNSUPPORTED;  // kMaxD <= 4 * kThreads: h widens in one round
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   int dev = 0;

@@ -7,8 +7,9 @@
 // -> top_p_clusters -> token_scores) runs as phases of one kernel:
 //
 //  1. centroid scores (section 1.2.2; INT4 centroids per section 1.2.4):
-//     cluster k belongs to global warp k mod W, which streams its centroid
-//     row and computes the key -- the score, or when sampling the Gumbel key
+//     cluster k belongs to CTA k mod G (warp (k / G) mod 16), so every CTA
+//     owns c/G clusters; the owning warp streams the centroid row and
+//     computes the key -- the score, or when sampling the Gumbel key
 //     s/T - ln(-ln u) (section 1.2.3). The key stays in a lane register of the
 //     owning warp and is counted into a device-wide histogram of its top 12
 //     bits (fire-and-forget atomics).
@@ -18,8 +19,8 @@
 //     selected cluster (its C2T row, section 1.2.1: slot k*b + j holds token
 //     C2T[k][j]) into a device-wide row queue, and the boundary keys into a
 //     small list.
-//  3. candidate rows are spread round-robin over every warp of the grid: a
-//     warp polls its queue slot for the token id, streams the token row and
+//  3. candidate rows are spread over every warp of the grid the same way
+//     (row r to CTA r mod G): a warp polls its queue slot for the token id, streams the token row and
 //     keeps a packed (logit, token) maximum (section 1.2.4, stage 2).
 //  4. when the boundary bin is split (some but not all of its keys needed),
 //     a warp that owns boundary keys ranks them exactly (key desc, id asc)
@@ -47,6 +48,7 @@ constexpr int kBarLanes = 8;       // counters per device-wide barrier
 constexpr int kBarStride = 32;     // words between counters (one 128-byte line each)
 
 struct B1Misc {
+  unsigned long long hbar;
   unsigned long long wbest[kWarps];
   float scan[kWarps + 1];
   uint32_t uscan[kWarps + 1];
@@ -105,14 +107,14 @@ __device__ __forceinline__ void queue_cluster(const B1Params& P, int32_t* rq, ui
 // against the published boundary list; the chosen clusters are queued.
 __device__ void rank_boundary(const B1Params& P, int32_t* rq, uint32_t* bitmap, uint32_t* qcount,
                               const unsigned long long* bnd_list, const uint32_t* bnd_count, uint32_t mine,
-                              uint32_t own_key, int gw, int W, uint32_t need) {
+                              uint32_t own_key, int cw, int cstride, uint32_t need) {
   const int lane = threadIdx.x & 31;
   const uint32_t nb = min(__ldcg(bnd_count), static_cast<uint32_t>(kBoundaryMax));
   while (mine) {
     const int j = __ffs(mine) - 1;
     mine &= mine - 1;
     const uint32_t kq = __shfl_sync(0xFFFFFFFFu, own_key, j);
-    const int idq = gw + j * W;
+    const int idq = cw + j * cstride;
     uint32_t r = 0;
     for (uint32_t e0 = 0; e0 < nb; e0 += 128) {
       unsigned long long v[4];
@@ -166,8 +168,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = gridDim.x;
-  const int W = G * kWarps;
-  const int gw = blockIdx.x * kWarps + warp;
   const int d = P.d, b = P.b;
   const bool gumbel = P.mode == 1;
 
@@ -189,36 +189,31 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   uint32_t* bar2 = P.bars + kBarLanes * kBarStride;
 
   // ---------------- phase 1: centroid scores ----------------
-  // h goes out first (every CTA needs it before its first dot), then the
-  // warp's first centroid row, then h is converted into shared memory.
-  uint4 hraw = make_uint4(0, 0, 0, 0);
-  if (tid < d / 8) hraw = *reinterpret_cast<const uint4*>(P.hidden + 8 * tid);
-  const int n1 = gw < P.c ? (P.c - 1 - gw) / W + 1 : 0;  // <= 32 (host-checked)
+  // Cluster k is owned by CTA k mod G, warp (k / G) mod 16, item k / (16 G):
+  // every CTA owns c/G clusters, so phase 1 ends at the same time everywhere.
+  // h goes out first, as one bulk copy per CTA (bf16, into the upper half of
+  // the fp32 buffer); then the warp's first centroid row.
+  const uint32_t hbar = smem_addr(&misc->hbar);
+  uint16_t* hraw = reinterpret_cast<uint16_t*>(hs + d / 2);
+  if (tid == 0) {
+    mbar_init(hbar, 1);
+    fence_mbar_init();
+    mbar_expect_tx(hbar, static_cast<uint32_t>(d * 2));
+    bulk_g2s(smem_addr(hraw), P.hidden, static_cast<uint32_t>(d * 2), hbar);
+  }
+  const int cw = static_cast<int>(blockIdx.x) + G * warp;  // first cluster of this warp
+  const int n1 = cw < P.c ? (P.c - 1 - cw) / (G * kWarps) + 1 : 0;  // <= 32 (host-checked)
+  auto cluster_of = [&](int i) { return cw + i * G * kWarps; };
   constexpr int NQ = (NCH + 1) / 2;
   uint4 w[NCH];
   uint2 q[NQ];
   uint32_t sc[NQ];
   if (n1 > 0) {
-    if constexpr (INT4) row_load_int4<NQ>(P.Crows + static_cast<size_t>(gw) * P.crow_bytes, d, q, sc);
-    else row_load_bf16<NCH>(reinterpret_cast<const uint16_t*>(P.Crows + static_cast<size_t>(gw) * P.crow_bytes), d, w);
+    if constexpr (INT4) row_load_int4<NQ>(P.Crows + static_cast<size_t>(cw) * P.crow_bytes, d, q, sc);
+    else row_load_bf16<NCH>(reinterpret_cast<const uint16_t*>(P.Crows + static_cast<size_t>(cw) * P.crow_bytes), d, w);
   }
   float ureg = 0.f;  // lane j holds u of item j
-  if (gumbel && lane < n1) ureg = __ldg(P.u_clusters + gw + lane * W);
-  if (tid < d / 8) {
-    float4 a, c4;
-    a.x = bf16lo(hraw.x); a.y = bf16hi(hraw.x); a.z = bf16lo(hraw.y); a.w = bf16hi(hraw.y);
-    c4.x = bf16lo(hraw.z); c4.y = bf16hi(hraw.z); c4.z = bf16lo(hraw.w); c4.w = bf16hi(hraw.w);
-    reinterpret_cast<float4*>(hs)[2 * tid] = a;
-    reinterpret_cast<float4*>(hs)[2 * tid + 1] = c4;
-  }
-  for (int i = tid + kThreads; i < d / 8; i += kThreads) {  // d > 4096 only
-    const uint4 x = *reinterpret_cast<const uint4*>(P.hidden + 8 * i);
-    float4 a, c4;
-    a.x = bf16lo(x.x); a.y = bf16hi(x.x); a.z = bf16lo(x.y); a.w = bf16hi(x.y);
-    c4.x = bf16lo(x.z); c4.y = bf16hi(x.z); c4.z = bf16lo(x.w); c4.w = bf16hi(x.w);
-    reinterpret_cast<float4*>(hs)[2 * i] = a;
-    reinterpret_cast<float4*>(hs)[2 * i + 1] = c4;
-  }
+  if (gumbel && lane < n1) ureg = __ldg(P.u_clusters + cluster_of(lane));
   {
     const int nz = kHistBins + P.words + 2 + P.nc_max;
     const int per = (nz + G - 1) / G;
@@ -234,11 +229,31 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     }
   }
   if (tid == 0) misc->cta_sure = 0u;
-  __syncthreads();
+  __syncthreads();  // hbar initialised before anyone waits on it
+  if (!mbar_wait_bounded(hbar, 0u, kWaitBudget)) {
+    if (lane == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
+  }
+  // widen h in place (d <= 4 * kThreads, so one round: every chunk is read
+  // before any is written): element e moves from hraw[e] to hs[e]
+  {
+    float hv[8];
+    const int i = tid;
+    if (i < d / 8) {
+      const uint4 x = *reinterpret_cast<const uint4*>(hraw + 8 * i);
+      hv[0] = bf16lo(x.x); hv[1] = bf16hi(x.x); hv[2] = bf16lo(x.y); hv[3] = bf16hi(x.y);
+      hv[4] = bf16lo(x.z); hv[5] = bf16hi(x.z); hv[6] = bf16lo(x.w); hv[7] = bf16hi(x.w);
+    }
+    __syncthreads();
+    if (i < d / 8) {
+      reinterpret_cast<float4*>(hs)[2 * i] = make_float4(hv[0], hv[1], hv[2], hv[3]);
+      reinterpret_cast<float4*>(hs)[2 * i + 1] = make_float4(hv[4], hv[5], hv[6], hv[7]);
+    }
+    __syncthreads();
+  }
 
   uint32_t own_key = 0u;  // lane j: key of the warp's item j
   for (int i = 0; i < n1; ++i) {
-    const int k = gw + i * W;
+    const int k = cluster_of(i);
     float s;
     if constexpr (INT4) {
       if (i > 0) row_load_int4<NQ>(P.Crows + static_cast<size_t>(k) * P.crow_bytes, d, q, sc);
@@ -294,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     __syncthreads();
     const uint32_t t1 = misc->t1, need = misc->need;
     const bool split = misc->split != 0, fallback = misc->fallback != 0;
-    const int r_sure = static_cast<int>(misc->n_sure) * b, r_all = P.p * b;
+    const int r_all = P.p * b;
     const uint32_t dg = own_key >> kHistShift;
     const bool mine = lane < n1;
     uint32_t bnd_mine = 0u;
@@ -312,13 +327,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
       while (sm) {
         const int j = __ffs(sm) - 1;
         sm &= sm - 1;
-        queue_cluster(P, rq, bitmap, pos++, gw + j * W);
+        queue_cluster(P, rq, bitmap, pos++, cluster_of(j));
       }
       bnd_mine = __ballot_sync(0xFFFFFFFFu, mine && split && dg == t1);
       if (bnd_mine & (1u << lane)) {
         const uint32_t at = atomicAdd(bnd_count, 1u);
         if (at < static_cast<uint32_t>(kBoundaryMax))
-          bnd_list[at] = (static_cast<unsigned long long>(own_key) << 32) | static_cast<uint32_t>(gw + lane * W);
+          bnd_list[at] = (static_cast<unsigned long long>(own_key) << 32) | static_cast<uint32_t>(cluster_of(lane));
       }
       __threadfence();
       if (split) bar_arrive(bar2);
@@ -333,7 +348,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     // ---------------- phases 3-4: consume candidate rows ----------------
     bool ranked = bnd_mine == 0u;
     const long long budget = P.spin_budget;
-    for (int r = gw; r < r_all; r += W) {
+    // candidate row r goes to CTA r mod G, warp (r / G) mod 16: balanced like phase 1
+    for (int r = static_cast<int>(blockIdx.x) + G * warp; r < r_all; r += G * kWarps) {
       int t;
       if (fallback) {
         t = __ldg(P.C2T + static_cast<size_t>(ssel[r / b]) * b + r % b);
@@ -344,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
             uint32_t ready = 0;
             if (lane == 0) ready = bar_count(bar2) >= static_cast<uint32_t>(G);
             if (__shfl_sync(0xFFFFFFFFu, ready, 0)) {
-              rank_boundary(P, rq, bitmap, qcount, bnd_list, bnd_count, bnd_mine, own_key, gw, W, need);
+              rank_boundary(P, rq, bitmap, qcount, bnd_list, bnd_count, bnd_mine, own_key, cw, G * kWarps, need);
               ranked = true;
             }
           }
@@ -376,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
         if (clock64() - t0 > budget) break;
       }
       if (__shfl_sync(0xFFFFFFFFu, ready, 0))
-        rank_boundary(P, rq, bitmap, qcount, bnd_list, bnd_count, bnd_mine, own_key, gw, W, need);
+        rank_boundary(P, rq, bitmap, qcount, bnd_list, bnd_count, bnd_mine, own_key, cw, G * kWarps, need);
       else
         ok = false;
     }
