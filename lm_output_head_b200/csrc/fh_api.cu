@@ -55,7 +55,7 @@ struct fh_head {
   long long spin_budget = kDefaultSpinBudget;
   // fused B = 1 plan
   bool fused_ok = false;
-  int b1_off_h = 0, b1_off_sel = 0, b1_off_misc = 0, b1_off_scratch = 0;
+  int b1_off_h = 0, b1_off_sel = 0, b1_off_misc = 0, b1_off_scratch = 0, b1_off_slots = 0, b1_slot_bytes = 0;
   size_t b1_smem = 0;
 };
 
@@ -336,6 +336,9 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
     o += up(decode_b1_misc_bytes(), 128);
     h->b1_off_scratch = static_cast<int>(o);
     o += up(sizeof(SelectSmem), 128);
+    h->b1_off_slots = static_cast<int>(o);
+    h->b1_slot_bytes = static_cast<int>(up(static_cast<size_t>(h->crow_bytes), 128));
+    o += static_cast<size_t>(kWarps) * h->b1_slot_bytes;
     h->b1_smem = o;
     int blocks = 0;
     e = occupancy_decode_b1(D.fmt == FH_CENTROID_INT4_G32, h->nch, h->b1_smem, &blocks);
@@ -504,6 +507,8 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
     P.off_sel = h->b1_off_sel;
     P.off_misc = h->b1_off_misc;
     P.off_scratch = h->b1_off_scratch;
+    P.off_slots = h->b1_off_slots;
+    P.slot_bytes = h->b1_slot_bytes;
     P.spin_budget = h->spin_budget;
     cudaError_t e = launch_decode_b1(P, h->b1_grid, h->b1_smem, D.fmt == FH_CENTROID_INT4_G32, h->nch, st);
     return e == cudaSuccess ? FH_OK : cuda_fail(e);

@@ -49,6 +49,7 @@ constexpr int kBarStride = 32;     // words between counters (one 128-byte line 
 
 struct B1Misc {
   unsigned long long hbar;
+  unsigned long long wbar[kWarps];
   unsigned long long wbest[kWarps];
   float scan[kWarps + 1];
   uint32_t uscan[kWarps + 1];
@@ -65,10 +66,14 @@ __device__ __forceinline__ void bar_arrive(uint32_t* bar) {
   }
 }
 
+// Sum of the counters: relaxed loads, all in flight together (the waiter
+// fences once after seeing the target).
 __device__ __forceinline__ uint32_t bar_count(const uint32_t* bar) {
-  uint32_t s = 0;
+  uint32_t v[kBarLanes], s = 0;
 #pragma unroll
-  for (int i = 0; i < kBarLanes; ++i) s += ld_acquire_u32(bar + i * kBarStride);
+  for (int i = 0; i < kBarLanes; ++i) v[i] = ld_relaxed_u32(bar + i * kBarStride);
+#pragma unroll
+  for (int i = 0; i < kBarLanes; ++i) s += v[i];
   return s;
 }
 
@@ -208,6 +213,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   uint4 w[NCH];
   uint2 q[NQ];
   uint32_t sc[NQ];
+  // the warp's second row (if any) is requested at once into its shared-memory slot
+  const uint32_t wbar = smem_addr(&misc->wbar[warp]);
+  const uint32_t slot = smem_addr(smem + P.off_slots) + static_cast<uint32_t>(warp * P.slot_bytes);
+  if (lane == 0) {
+    mbar_init(wbar, 1);
+    fence_mbar_init();
+    if (n1 >= 2) {
+      mbar_expect_tx(wbar, static_cast<uint32_t>(P.crow_bytes));
+      bulk_g2s(slot, P.Crows + static_cast<size_t>(cluster_of(1)) * P.crow_bytes, static_cast<uint32_t>(P.crow_bytes),
+               wbar);
+    }
+  }
   if (n1 > 0) {
     if constexpr (INT4) row_load_int4<NQ>(P.Crows + static_cast<size_t>(cw) * P.crow_bytes, d, q, sc);
     else row_load_bf16<NCH>(reinterpret_cast<const uint16_t*>(P.Crows + static_cast<size_t>(cw) * P.crow_bytes), d, w);
@@ -255,7 +272,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   for (int i = 0; i < n1; ++i) {
     const int k = cluster_of(i);
     float s;
-    if constexpr (INT4) {
+    if (i == 1) {  // the row that landed in the slot
+      if (!mbar_wait_bounded(wbar, 0u, kWaitBudget) && lane == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
+      if constexpr (INT4) s = srow_dot_int4_hs<NQ>(slot, hs, d);
+      else s = srow_dot_bf16_hs<NCH>(slot, hs, d);
+    } else if constexpr (INT4) {
       if (i > 0) row_load_int4<NQ>(P.Crows + static_cast<size_t>(k) * P.crow_bytes, d, q, sc);
       s = row_dot_int4_hs<NQ>(q, sc, hs, d);
     } else {
@@ -360,6 +381,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
             uint32_t ready = 0;
             if (lane == 0) ready = bar_count(bar2) >= static_cast<uint32_t>(G);
             if (__shfl_sync(0xFFFFFFFFu, ready, 0)) {
+              __threadfence();
               rank_boundary(P, rq, bitmap, qcount, bnd_list, bnd_count, bnd_mine, own_key, cw, G * kWarps, need);
               ranked = true;
             }
@@ -391,10 +413,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
         if (__shfl_sync(0xFFFFFFFFu, ready, 0)) break;
         if (clock64() - t0 > budget) break;
       }
-      if (__shfl_sync(0xFFFFFFFFu, ready, 0))
+      if (__shfl_sync(0xFFFFFFFFu, ready, 0)) {
+        __threadfence();
         rank_boundary(P, rq, bitmap, qcount, bnd_list, bnd_count, bnd_mine, own_key, cw, G * kWarps, need);
-      else
+      }
+      else {
         ok = false;
+      }
     }
     if (!ok && lane == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
   }

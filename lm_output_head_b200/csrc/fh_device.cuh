@@ -91,6 +91,12 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned* p) {
   return v;
 }
 
+__device__ __forceinline__ uint32_t ld_relaxed_u32(const unsigned* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -609,6 +615,50 @@ __device__ __forceinline__ float row_dot_int4_hs(const uint2 (&q)[NQ], const uin
     }
   }
   return warp_sum(acc);
+}
+
+// The same dots for a row held in shared memory (landed by a bulk copy).
+template <int NCH>
+__device__ __forceinline__ float srow_dot_bf16_hs(uint32_t row, const float* hs, int d) {
+  const int lane = threadIdx.x & 31;
+  float acc = 0.f;
+#pragma unroll
+  for (int m = 0; m < NCH; ++m) {
+    const int e = (lane + 32 * m) * 8;
+    if (e < d) {
+      const uint4 w = lds128(row + 2u * e);
+      const float4 a = *reinterpret_cast<const float4*>(hs + e);
+      const float4 b = *reinterpret_cast<const float4*>(hs + e + 4);
+      acc = fmaf(bf16lo(w.x), a.x, acc);
+      acc = fmaf(bf16hi(w.x), a.y, acc);
+      acc = fmaf(bf16lo(w.y), a.z, acc);
+      acc = fmaf(bf16hi(w.y), a.w, acc);
+      acc = fmaf(bf16lo(w.z), b.x, acc);
+      acc = fmaf(bf16hi(w.z), b.y, acc);
+      acc = fmaf(bf16lo(w.w), b.z, acc);
+      acc = fmaf(bf16hi(w.w), b.w, acc);
+    }
+  }
+  return warp_sum(acc);
+}
+
+template <int NQ>
+__device__ __forceinline__ float srow_dot_int4_hs(uint32_t row, const float* hs, int d) {
+  uint2 q[NQ];
+  uint32_t sc[NQ];
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int m = 0; m < NQ; ++m) {
+    const int g = lane + 32 * m;
+    if (g * 16 < d) {
+      q[m] = lds64(row + 8u * g);
+      sc[m] = lds16(row + d / 2 + 2u * (g >> 1));
+    } else {
+      q[m] = make_uint2(0u, 0u);
+      sc[m] = 0u;
+    }
+  }
+  return row_dot_int4_hs<NQ>(q, sc, hs, d);
 }
 
 // Stage a bf16 vector of d elements (d % 8 == 0) into shared memory as fp32.

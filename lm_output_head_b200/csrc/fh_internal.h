@@ -51,7 +51,7 @@ struct B1Params {
   int crow_bytes;
   int mode;
   float T;
-  int off_h, off_sel, off_misc, off_scratch;
+  int off_h, off_sel, off_misc, off_scratch, off_slots, slot_bytes;
   long long spin_budget;
 };
 
