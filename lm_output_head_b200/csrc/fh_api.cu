@@ -17,7 +17,7 @@ int dense_max_rows();
 cudaError_t occupancy_decode_b1(int int4, int nch, size_t smem, int* blocks);
 size_t decode_b1_misc_bytes();
 cudaError_t occupancy_dense(int nch, size_t smem, int* blocks);
-size_t decode_b1_bar_words();
+
 }  // namespace fh
 
 using namespace fh;
@@ -38,12 +38,7 @@ struct fh_head {
   int32_t* row_ok = nullptr;           // [max_batch]
   uint32_t* c2t_counts = nullptr;      // [v]
   uint32_t* b1_keys = nullptr;         // fused B = 1 state
-  float* b1_z_tok = nullptr;
-  uint32_t* b1_hist = nullptr;
-  uint32_t* b1_bars = nullptr;
-  uint32_t* b1_bitmap = nullptr;
-  unsigned long long* b1_bnd = nullptr;
-  uint32_t* b1_counts = nullptr;
+  float* b1_z_row = nullptr;
   int32_t* b1_queue = nullptr;
   int words = 0;
   int b1_grid = 0;
@@ -55,7 +50,7 @@ struct fh_head {
   long long spin_budget = kDefaultSpinBudget;
   // fused B = 1 plan
   bool fused_ok = false;
-  int b1_off_h = 0, b1_off_sel = 0, b1_off_misc = 0, b1_off_scratch = 0, b1_off_slots = 0, b1_slot_bytes = 0;
+  int b1_off_h = 0, b1_off_sel = 0, b1_off_misc = 0, b1_off_slots = 0, b1_slot_bytes = 0;
   size_t b1_smem = 0;
 };
 
@@ -246,12 +241,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   const size_t o_hist = take(mb * kHistBins * 4);
   const int words = (D.c + 31) / 32;
   const size_t o_keys1 = take(static_cast<size_t>(D.c) * 4);
-  const size_t o_ztok = take(static_cast<size_t>(D.v) * 4);
-  const size_t o_hlo = take(2 * kHistBins * 4);
-  const size_t o_bars = take(decode_b1_bar_words() * 4);
-  const size_t o_bmp = take(2 * static_cast<size_t>(words) * 4);
-  const size_t o_bnd = take(2 * kBoundaryMax * 8);
-  const size_t o_bcnt = take(4 * 4);
+  const size_t o_zrow = take(nc * 4);
   const size_t o_queue = take(2 * nc * 4);
   const size_t o_crow = D.fmt == FH_CENTROID_INT4_G32 ? take(static_cast<size_t>(D.c) * h->crow_bytes) : 0;
   h->ws_bytes = off;
@@ -275,12 +265,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   h->row_ok = reinterpret_cast<int32_t*>(h->ws + o_rok);
   h->c2t_counts = reinterpret_cast<uint32_t*>(h->ws + o_cnt);
   h->b1_keys = reinterpret_cast<uint32_t*>(h->ws + o_keys1);
-  h->b1_z_tok = reinterpret_cast<float*>(h->ws + o_ztok);
-  h->b1_hist = reinterpret_cast<uint32_t*>(h->ws + o_hlo);
-  h->b1_bars = reinterpret_cast<uint32_t*>(h->ws + o_bars);
-  h->b1_bitmap = reinterpret_cast<uint32_t*>(h->ws + o_bmp);
-  h->b1_bnd = reinterpret_cast<unsigned long long*>(h->ws + o_bnd);
-  h->b1_counts = reinterpret_cast<uint32_t*>(h->ws + o_bcnt);
+  h->b1_z_row = reinterpret_cast<float*>(h->ws + o_zrow);
   h->b1_queue = reinterpret_cast<int32_t*>(h->ws + o_queue);
   h->words = words;
   h->hist = reinterpret_cast<uint32_t*>(h->ws + o_hist);
@@ -325,7 +310,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
     return status;
   }
 
-  // ---- fused B = 1 plan: h (fp32), selection list, misc, scratch ----
+  // ---- fused B = 1 plan: h (fp32), selection list, misc, per-warp row slots ----
   {
     size_t o = 0;
     h->b1_off_h = static_cast<int>(o);
@@ -334,11 +319,10 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
     o += up(static_cast<size_t>(D.max_probes) * 4, 128);
     h->b1_off_misc = static_cast<int>(o);
     o += up(decode_b1_misc_bytes(), 128);
-    h->b1_off_scratch = static_cast<int>(o);
-    o += up(sizeof(SelectSmem), 128);
     h->b1_off_slots = static_cast<int>(o);
-    h->b1_slot_bytes = static_cast<int>(up(static_cast<size_t>(h->crow_bytes), 128));
-    o += static_cast<size_t>(kWarps) * h->b1_slot_bytes;
+    h->b1_slot_bytes = static_cast<int>(up(std::max(static_cast<size_t>(h->crow_bytes), static_cast<size_t>(D.d) * 2), 128));
+    // the slots double as the selector's scratch once phase 1 is done
+    o += std::max(static_cast<size_t>(kWarps) * h->b1_slot_bytes, hist_select_smem_bytes(D.c, false));
     h->b1_smem = o;
     int blocks = 0;
     e = occupancy_decode_b1(D.fmt == FH_CENTROID_INT4_G32, h->nch, h->b1_smem, &blocks);
@@ -484,12 +468,7 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
     P.out_cluster_ids = out_cluster_ids;
     P.out_max_logit = out_max_logit;
     P.keys = h->b1_keys;
-    P.z_tok = h->b1_z_tok;
-    P.hist = h->b1_hist;
-    P.bars = h->b1_bars;
-    P.bitmap = h->b1_bitmap;
-    P.bnd_list = h->b1_bnd;
-    P.counts = h->b1_counts;
+    P.z_row = h->b1_z_row;
     P.row_queue = h->b1_queue;
     P.best = h->best;
     P.sync = h->sync;
@@ -498,7 +477,6 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
     P.c = D.c;
     P.b = D.b;
     P.p = p;
-    P.words = h->words;
     P.nc_max = D.max_probes * D.b;
     P.crow_bytes = h->crow_bytes;
     P.mode = mode;
@@ -506,7 +484,6 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
     P.off_h = h->b1_off_h;
     P.off_sel = h->b1_off_sel;
     P.off_misc = h->b1_off_misc;
-    P.off_scratch = h->b1_off_scratch;
     P.off_slots = h->b1_off_slots;
     P.slot_bytes = h->b1_slot_bytes;
     P.spin_budget = h->spin_budget;

@@ -373,31 +373,36 @@ struct HistSelectSmem {
 };
 
 // Bytes of shared scratch the select needs for c keys: the struct, a c-byte
-// flag array, and c keys for the radix fallback.
-__host__ __device__ inline size_t hist_select_smem_bytes(int c) {
+// flag array, the radix fallback state, and (when the keys are not in global
+// memory as keys already) c keys for that fallback.
+__host__ __device__ inline size_t hist_select_smem_bytes(int c, bool keys_in_smem = true) {
   return ((sizeof(HistSelectSmem) + 127) & ~size_t(127)) + ((static_cast<size_t>(c) + 127) & ~size_t(127)) +
-         ((static_cast<size_t>(c) * 4 + 127) & ~size_t(127)) + sizeof(SelectSmem);
+         ((sizeof(SelectSmem) + 127) & ~size_t(127)) +
+         (keys_in_smem ? ((static_cast<size_t>(c) * 4 + 127) & ~size_t(127)) : 0);
 }
 
-// Top-p of the c keys derived from `scores` (global, read through L2):
-// key = scores[k], or the Gumbel key scores[k]/T - ln(-ln u[k]) when u != null.
-// `hist_g` (global, 4096 bins of key >> 20) may be null. Writes the chosen
-// ids in ascending order to `sel`. All kThreads threads must call it.
-__device__ inline void select_top_p_hist(const float* scores, const float* u, float T, int c, int p,
-                                         const uint32_t* hist_g, int32_t* sel, uint8_t* scratch) {
+// Core of the histogram-driven select. `load_key(id)` returns the order-
+// preserving key of cluster id (< c). `hist_g` (global, 4096 bins of
+// key >> 20) may be null: then the histogram is built in shared memory.
+// `gkeys`: the same keys in global memory for the radix fallback, or null to
+// stage them in shared memory. Writes the chosen ids ascending to `sel`.
+template <class LoadKey>
+__device__ inline void select_top_p_core(LoadKey load_key, int c, int p, const uint32_t* hist_g,
+                                         const uint32_t* gkeys, int32_t* sel, uint8_t* scratch) {
   HistSelectSmem& sm = *reinterpret_cast<HistSelectSmem*>(scratch);
   uint8_t* flag = scratch + ((sizeof(HistSelectSmem) + 127) & ~size_t(127));
-  uint32_t* skey = reinterpret_cast<uint32_t*>(flag + ((static_cast<size_t>(c) + 127) & ~size_t(127)));
-  SelectSmem* fsm = reinterpret_cast<SelectSmem*>(reinterpret_cast<uint8_t*>(skey) +
-                                                   ((static_cast<size_t>(c) * 4 + 127) & ~size_t(127)));
+  SelectSmem* fsm = reinterpret_cast<SelectSmem*>(flag + ((static_cast<size_t>(c) + 127) & ~size_t(127)));
+  uint32_t* skey =
+      reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(fsm) + ((sizeof(SelectSmem) + 127) & ~size_t(127)));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t lt_mask = (1u << lane) - 1u;
 
-  if (c > kWarps * 32 * kKeysPerThreadMax) {  // too many keys for registers: radix select in smem
-    for (int k = tid; k < c; k += kThreads)
-      skey[k] = f2key(u ? gumbel_key(__ldcg(scores + k), T, __ldcg(u + k)) : __ldcg(scores + k));
-    __syncthreads();
-    block_select_top_p(skey, c, p, sel, *fsm);
+  if (c > kWarps * 32 * kKeysPerThreadMax) {  // too many keys for registers: radix select
+    if (!gkeys) {
+      for (int k = tid; k < c; k += kThreads) skey[k] = load_key(k);
+      __syncthreads();
+    }
+    block_select_top_p(gkeys ? gkeys : skey, c, p, sel, *fsm);
     return;
   }
 
@@ -408,12 +413,7 @@ __device__ inline void select_top_p_hist(const float* scores, const float* u, fl
 #pragma unroll
   for (int i = 0; i < kKeysPerThreadMax; ++i) {
     const int id = wbase + i * 32 + lane;
-    float v = 0.f;
-    if (i < kpt && id < c) {
-      v = __ldcg(scores + id);
-      if (u) v = gumbel_key(v, T, __ldcg(u + id));
-    }
-    key[i] = f2key(v);
+    key[i] = (i < kpt && id < c) ? load_key(id) : 0u;
   }
   for (int i = tid; i < (c + 15) / 16; i += kThreads) reinterpret_cast<uint4*>(flag)[i] = make_uint4(0, 0, 0, 0);
   if (hist_g == nullptr) {
@@ -454,13 +454,15 @@ __device__ inline void select_top_p_hist(const float* scores, const float* u, fl
   const bool all_in_bin = (m1 == need);
 
   if (!all_in_bin && m1 > static_cast<uint32_t>(kBoundaryMax)) {  // pathological ties: radix fallback
+    if (!gkeys) {
 #pragma unroll
-    for (int i = 0; i < kKeysPerThreadMax; ++i) {
-      const int id = wbase + i * 32 + lane;
-      if (i < kpt && id < c) skey[id] = key[i];
+      for (int i = 0; i < kKeysPerThreadMax; ++i) {
+        const int id = wbase + i * 32 + lane;
+        if (i < kpt && id < c) skey[id] = key[i];
+      }
+      __syncthreads();
     }
-    __syncthreads();
-    block_select_top_p(skey, c, p, sel, *fsm);
+    block_select_top_p(gkeys ? gkeys : skey, c, p, sel, *fsm);
     return;
   }
   if (!all_in_bin) {
@@ -520,6 +522,27 @@ __device__ inline void select_top_p_hist(const float* scores, const float* u, fl
     pos += __popc(m);
   }
   __syncthreads();
+}
+
+
+// Top-p of the c keys derived from `scores` (global, read through L2):
+// key = scores[k], or the Gumbel key scores[k]/T - ln(-ln u[k]) when u != null.
+// `hist_g` (global, 4096 bins of key >> 20) may be null. Writes the chosen
+// ids in ascending order to `sel`. All kThreads threads must call it.
+__device__ inline void select_top_p_hist(const float* scores, const float* u, float T, int c, int p,
+                                         const uint32_t* hist_g, int32_t* sel, uint8_t* scratch) {
+  auto load_key = [&](int id) -> uint32_t {
+    float v = __ldcg(scores + id);
+    if (u) v = gumbel_key(v, T, __ldcg(u + id));
+    return f2key(v);
+  };
+  select_top_p_core(load_key, c, p, hist_g, nullptr, sel, scratch);
+}
+
+// Top-p of order-preserving keys already in global memory (one reader CTA).
+__device__ inline void select_top_p_gkeys(const uint32_t* gkeys, int c, int p, int32_t* sel, uint8_t* scratch) {
+  auto load_key = [&](int id) -> uint32_t { return __ldcg(gkeys + id); };
+  select_top_p_core(load_key, c, p, nullptr, gkeys, sel, scratch);
 }
 
 // ---------------------------------------------------------------------------

@@ -36,22 +36,16 @@ struct B1Params {
   int32_t* out_tokens;
   int32_t* out_cluster_ids;
   float* out_max_logit;
-  uint32_t* keys;         // workspace [c]: order-preserving keys (read only by the tie fallback)
-  float* z_tok;           // workspace [v]: candidate logits by token id (sampling)
-  // per-call state, two buffers used by alternate calls
-  uint32_t* hist;         // [2][4096]  histogram of key >> 20
-  uint32_t* bars;         // two device-wide barriers, 8 counters each, one per 128-byte line
-  uint32_t* bitmap;       // [2][words] selected clusters
-  unsigned long long* bnd_list;  // [2][2048] boundary (key << 32 | id)
-  uint32_t* counts;       // [2][2]     boundary count, row-queue count
-  int32_t* row_queue;     // [2][nc_max] token id of candidate slot, -1 until written
+  uint32_t* keys;         // workspace [c]: order-preserving keys of the clusters
+  float* z_row;           // workspace [nc_max]: candidate logits in queue order (sampling)
+  int32_t* row_queue;     // workspace [2][nc_max]: candidate token ids, -1 until written; alternate calls
   unsigned long long* best;
   SyncWords* sync;
-  int v, d, c, b, p, words, nc_max;
+  int v, d, c, b, p, nc_max;
   int crow_bytes;
   int mode;
   float T;
-  int off_h, off_sel, off_misc, off_scratch, off_slots, slot_bytes;
+  int off_h, off_sel, off_misc, off_slots, slot_bytes;
   long long spin_budget;
 };
 
