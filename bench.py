@@ -202,15 +202,23 @@ def run_ours(args):
 
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    flush64 = flush.view(torch.int64)
     stream = torch.cuda.current_stream(dev)
+
+    def flush_l2():
+        # write a buffer twice the L2, then read it back: no line of the head
+        # survives, and the lines left behind are clean (their write-back is
+        # not charged to the next timed call)
+        flush.fill_(1)
+        flush64.sum()
 
     def step(i):
         dh.decode(Hdev[i % n_states:i % n_states + 1], cfg.p, out_tokens=out, stream=stream)
 
-    def timed_loop(fn, K, W, flush_l2=True):
+    def timed_loop(fn, K, W, flush_first=True):
         for i in range(W):
-            if flush_l2:
-                flush.zero_()
+            if flush_first:
+                flush_l2()
             fn(i)
         torch.cuda.synchronize(dev)
         if world > 1:
@@ -220,8 +228,8 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
         wall0 = time.time()
         for i in range(K):
-            if flush_l2:
-                flush.zero_()
+            if flush_first:
+                flush_l2()
             starts[i].record(stream)
             fn(W + i)
             ends[i].record(stream)
@@ -260,7 +268,7 @@ def run_ours(args):
     ke = max(3, min(args.steps, 500))
     e2e_ms = []
     for i in range(ke + 3):
-        flush.zero_()
+        flush_l2()
         s0 = torch.cuda.Event(enable_timing=True)
         s1 = torch.cuda.Event(enable_timing=True)
         s0.record(stream)
@@ -298,7 +306,7 @@ def run_ours(args):
         "data": "synthetic (seeded planted-cluster head; 75% planted / 25% flat hidden states)",
         "config": {"workload": WORKLOAD, "global_batch": world, "per_gpu_batch": 1,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "flushed before every step (2 x L2 memset outside the timed events)",
+                   "l2": "flushed before every step: 2 x L2 buffer written then read, outside the timed events",
                    "states": n_states},
         "us_per_token": round(mean_ms * 1e3, 3),
         "latency_us": {"p50": round(statistics.median(ms) * 1e3, 3),

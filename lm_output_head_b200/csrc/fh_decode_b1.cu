@@ -173,7 +173,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     selector_top_p(P.keys, P.c, P.p, ssel, slots);
     if (P.out_cluster_ids)
       for (int i = tid; i < P.p; i += kThreads) P.out_cluster_ids[i] = ssel[i];
-    for (int r = tid; r < r_all; r += kThreads) rq[r] = __ldg(P.C2T + static_cast<size_t>(ssel[r / b]) * b + r % b);
+    // thread q writes the C2T row of the q-th chosen cluster: slots q*b .. q*b + b - 1
+    const bool vec = (b % 4 == 0) && ((reinterpret_cast<uintptr_t>(P.C2T) & 15) == 0);
+    for (int qi = tid; qi < P.p; qi += kThreads) {
+      const int32_t* src = P.C2T + static_cast<size_t>(ssel[qi]) * b;
+      int32_t* dst = rq + static_cast<size_t>(qi) * b;
+      if (vec) {
+        for (int j = 0; j < b; j += 4)
+          *reinterpret_cast<int4*>(dst + j) = __ldg(reinterpret_cast<const int4*>(src + j));
+      } else {
+        for (int j = 0; j < b; ++j) dst[j] = __ldg(src + j);
+      }
+    }
     fence_proxy_async_smem();  // the slots were generic scratch; bulk copies follow
     __syncthreads();
   }

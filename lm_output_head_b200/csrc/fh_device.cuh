@@ -360,7 +360,7 @@ __device__ inline void block_select_top_p(const uint32_t* skey, int n, int p, in
 // built here in shared memory.
 constexpr int kHistBins = 4096;
 constexpr int kHistShift = 20;
-constexpr int kKeysPerThreadMax = 32;          // keys held in registers: c <= 16384
+constexpr int kKeysPerThreadMax = 32;          // keys held in registers: c <= 32 * 512
 constexpr int kBoundaryMax = 2048;              // exact all-pairs ranking up to this many ties-in-bin
 
 struct HistSelectSmem {
@@ -381,12 +381,15 @@ __host__ __device__ inline size_t hist_select_smem_bytes(int c, bool keys_in_sme
          (keys_in_smem ? ((static_cast<size_t>(c) * 4 + 127) & ~size_t(127)) : 0);
 }
 
-// Core of the histogram-driven select. `load_key(id)` returns the order-
-// preserving key of cluster id (< c). `hist_g` (global, 4096 bins of
-// key >> 20) may be null: then the histogram is built in shared memory.
-// `gkeys`: the same keys in global memory for the radix fallback, or null to
-// stage them in shared memory. Writes the chosen ids ascending to `sel`.
-template <class LoadKey>
+// Core of the histogram-driven select, laid out for short dependency chains:
+// thread t owns the contiguous ids [t*kpt, t*kpt + kpt) (kpt = ceil(c/512)),
+// so one block scan orders the output. `load_key(id)` returns the order-
+// preserving key of cluster id (< c); all of a thread's loads are independent.
+// `hist_g` (global, 4096 bins of key >> 20) may be null: then the histogram
+// is built in shared memory with fire-and-forget atomics. `gkeys`: the same
+// keys in global memory for the radix fallback, or null to stage them in
+// shared memory. Writes the chosen ids ascending to `sel`.
+template <int KMAX, class LoadKey>
 __device__ inline void select_top_p_core(LoadKey load_key, int c, int p, const uint32_t* hist_g,
                                          const uint32_t* gkeys, int32_t* sel, uint8_t* scratch) {
   HistSelectSmem& sm = *reinterpret_cast<HistSelectSmem*>(scratch);
@@ -394,10 +397,9 @@ __device__ inline void select_top_p_core(LoadKey load_key, int c, int p, const u
   SelectSmem* fsm = reinterpret_cast<SelectSmem*>(flag + ((static_cast<size_t>(c) + 127) & ~size_t(127)));
   uint32_t* skey =
       reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(fsm) + ((sizeof(SelectSmem) + 127) & ~size_t(127)));
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t lt_mask = (1u << lane) - 1u;
+  const int tid = threadIdx.x;
 
-  if (c > kWarps * 32 * kKeysPerThreadMax) {  // too many keys for registers: radix select
+  if (c > kThreads * KMAX) {  // too many keys for registers: radix select
     if (!gkeys) {
       for (int k = tid; k < c; k += kThreads) skey[k] = load_key(k);
       __syncthreads();
@@ -406,13 +408,12 @@ __device__ inline void select_top_p_core(LoadKey load_key, int c, int p, const u
     return;
   }
 
-  // keys in registers, warp-block layout: warp w holds ids [w*kpt*32, (w+1)*kpt*32)
-  const int kpt = (c + kWarps * 32 - 1) / (kWarps * 32);
-  const int wbase = warp * kpt * 32;
-  uint32_t key[kKeysPerThreadMax];
+  const int kpt = (c + kThreads - 1) / kThreads;
+  const int id0 = tid * kpt;
+  uint32_t key[KMAX];
 #pragma unroll
-  for (int i = 0; i < kKeysPerThreadMax; ++i) {
-    const int id = wbase + i * 32 + lane;
+  for (int i = 0; i < KMAX; ++i) {
+    const int id = id0 + i;
     key[i] = (i < kpt && id < c) ? load_key(id) : 0u;
   }
   for (int i = tid; i < (c + 15) / 16; i += kThreads) reinterpret_cast<uint4*>(flag)[i] = make_uint4(0, 0, 0, 0);
@@ -420,10 +421,8 @@ __device__ inline void select_top_p_core(LoadKey load_key, int c, int p, const u
     for (int i = tid; i < kHistBins; i += kThreads) sm.hist[i] = 0u;
     __syncthreads();
 #pragma unroll
-    for (int i = 0; i < kKeysPerThreadMax; ++i) {
-      const int id = wbase + i * 32 + lane;
-      if (i < kpt && id < c) atomicAdd(&sm.hist[key[i] >> kHistShift], 1u);
-    }
+    for (int i = 0; i < KMAX; ++i)
+      if (i < kpt && id0 + i < c) atomicAdd(&sm.hist[key[i] >> kHistShift], 1u);
   } else {
     for (int i = tid; i < kHistBins; i += kThreads) sm.hist[i] = __ldcg(hist_g + i);
   }
@@ -432,21 +431,22 @@ __device__ inline void select_top_p_core(LoadKey load_key, int c, int p, const u
 
   // bin t1 holding the p-th largest key: thread t owns bins 4095-8t .. 4088-8t
   constexpr int kBpt = kHistBins / kThreads;
-  uint32_t loc = 0;
+  uint32_t hv[kBpt], loc = 0;
 #pragma unroll
-  for (int i = 0; i < kBpt; ++i) loc += sm.hist[kHistBins - 1 - kBpt * tid - i];
+  for (int i = 0; i < kBpt; ++i) {
+    hv[i] = sm.hist[kHistBins - 1 - kBpt * tid - i];
+    loc += hv[i];
+  }
   const uint32_t above = block_exclusive_scan<kThreads, uint32_t>(loc, sm.scan, nullptr);
   uint32_t run = above;
 #pragma unroll
   for (int i = 0; i < kBpt; ++i) {
-    const int b = kHistBins - 1 - kBpt * tid - i;
-    const uint32_t h = sm.hist[b];
-    if (run < static_cast<uint32_t>(p) && run + h >= static_cast<uint32_t>(p)) {
-      sm.t1 = static_cast<uint32_t>(b);
+    if (run < static_cast<uint32_t>(p) && run + hv[i] >= static_cast<uint32_t>(p)) {
+      sm.t1 = static_cast<uint32_t>(kHistBins - 1 - kBpt * tid - i);
       sm.above = run;
-      sm.m1 = h;
+      sm.m1 = hv[i];
     }
-    run += h;
+    run += hv[i];
   }
   __syncthreads();
   const uint32_t t1 = sm.t1, m1 = sm.m1;
@@ -456,30 +456,22 @@ __device__ inline void select_top_p_core(LoadKey load_key, int c, int p, const u
   if (!all_in_bin && m1 > static_cast<uint32_t>(kBoundaryMax)) {  // pathological ties: radix fallback
     if (!gkeys) {
 #pragma unroll
-      for (int i = 0; i < kKeysPerThreadMax; ++i) {
-        const int id = wbase + i * 32 + lane;
-        if (i < kpt && id < c) skey[id] = key[i];
-      }
+      for (int i = 0; i < KMAX; ++i)
+        if (i < kpt && id0 + i < c) skey[id0 + i] = key[i];
       __syncthreads();
     }
     block_select_top_p(gkeys ? gkeys : skey, c, p, sel, *fsm);
     return;
   }
   if (!all_in_bin) {
-    // gather the boundary bin, rank it exactly, flag the chosen ids
+    // gather the boundary bin, rank it exactly (key desc, id asc), flag the chosen ids
 #pragma unroll
-    for (int i = 0; i < kKeysPerThreadMax; ++i) {
-      const int id = wbase + i * 32 + lane;
-      const bool in = i < kpt && id < c && (key[i] >> kHistShift) == t1;
-      const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
-      if (m) {
-        uint32_t base = 0;
-        if (lane == 0) base = atomicAdd(&sm.ncand, static_cast<uint32_t>(__popc(m)));
-        base = __shfl_sync(0xFFFFFFFFu, base, 0);
-        const uint32_t at = base + __popc(m & lt_mask);
-        if (in && at < static_cast<uint32_t>(kBoundaryMax)) {
+    for (int i = 0; i < KMAX; ++i) {
+      if (i < kpt && id0 + i < c && (key[i] >> kHistShift) == t1) {
+        const uint32_t at = atomicAdd(&sm.ncand, 1u);
+        if (at < static_cast<uint32_t>(kBoundaryMax)) {
           sm.ckey[at] = key[i];
-          sm.cid[at] = id;
+          sm.cid[at] = id0 + i;
         }
       }
     }
@@ -489,41 +481,52 @@ __device__ inline void select_top_p_core(LoadKey load_key, int c, int p, const u
       const uint32_t ka = sm.ckey[a];
       const int ia = sm.cid[a];
       uint32_t r = 0;
-      for (uint32_t b = 0; b < nb; ++b) {
-        const uint32_t kb = sm.ckey[b];
-        r += (kb > ka) || (kb == ka && sm.cid[b] < ia);
+      uint32_t bb = 0;
+      for (; bb + 8 <= nb; bb += 8) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t kb = sm.ckey[bb + u];
+          r += (kb > ka) || (kb == ka && sm.cid[bb + u] < ia);
+        }
+      }
+      for (; bb < nb; ++bb) {
+        const uint32_t kb = sm.ckey[bb];
+        r += (kb > ka) || (kb == ka && sm.cid[bb] < ia);
       }
       if (r < need) flag[ia] = 1;
     }
     __syncthreads();
   }
 
-  // ascending-id compaction with ballots
+  // ascending-id compaction: one block scan of per-thread counts
   uint32_t cnt = 0;
 #pragma unroll
-  for (int i = 0; i < kKeysPerThreadMax; ++i) {
-    const int id = wbase + i * 32 + lane;
+  for (int i = 0; i < KMAX; ++i) {
+    const int id = id0 + i;
     const uint32_t dg = key[i] >> kHistShift;
-    const bool take = i < kpt && id < c && (dg > t1 || (dg == t1 && (all_in_bin || flag[id])));
-    cnt += __popc(__ballot_sync(0xFFFFFFFFu, take));
+    cnt += (i < kpt && id < c && (dg > t1 || (dg == t1 && (all_in_bin || flag[id])))) ? 1u : 0u;
   }
-  if (lane == 0) sm.wcount[warp] = cnt;
-  __syncthreads();
-  uint32_t pos = 0;
-  for (int w = 0; w < warp; ++w) pos += sm.wcount[w];
+  uint32_t pos = block_exclusive_scan<kThreads, uint32_t>(cnt, sm.scan, nullptr);
 #pragma unroll
-  for (int i = 0; i < kKeysPerThreadMax; ++i) {
-    const int id = wbase + i * 32 + lane;
+  for (int i = 0; i < KMAX; ++i) {
+    const int id = id0 + i;
     const uint32_t dg = key[i] >> kHistShift;
-    const bool take = i < kpt && id < c && (dg > t1 || (dg == t1 && (all_in_bin || flag[id])));
-    const uint32_t m = __ballot_sync(0xFFFFFFFFu, take);
-    const uint32_t at = pos + __popc(m & lt_mask);
-    if (take && at < static_cast<uint32_t>(p)) sel[at] = id;
-    pos += __popc(m);
+    if (i < kpt && id < c && (dg > t1 || (dg == t1 && (all_in_bin || flag[id])))) {
+      if (pos < static_cast<uint32_t>(p)) sel[pos] = id;
+      ++pos;
+    }
   }
   __syncthreads();
 }
 
+// Dispatch on the number of keys each thread holds in registers.
+template <class LoadKey>
+__device__ inline void select_top_p_any(LoadKey load_key, int c, int p, const uint32_t* hist_g, const uint32_t* gkeys,
+                                        int32_t* sel, uint8_t* scratch) {
+  if (c <= kThreads * 8) select_top_p_core<8>(load_key, c, p, hist_g, gkeys, sel, scratch);
+  else if (c <= kThreads * 16) select_top_p_core<16>(load_key, c, p, hist_g, gkeys, sel, scratch);
+  else select_top_p_core<kKeysPerThreadMax>(load_key, c, p, hist_g, gkeys, sel, scratch);
+}
 
 // Top-p of the c keys derived from `scores` (global, read through L2):
 // key = scores[k], or the Gumbel key scores[k]/T - ln(-ln u[k]) when u != null.
@@ -536,13 +539,13 @@ __device__ inline void select_top_p_hist(const float* scores, const float* u, fl
     if (u) v = gumbel_key(v, T, __ldcg(u + id));
     return f2key(v);
   };
-  select_top_p_core(load_key, c, p, hist_g, nullptr, sel, scratch);
+  select_top_p_any(load_key, c, p, hist_g, nullptr, sel, scratch);
 }
 
 // Top-p of order-preserving keys already in global memory (one reader CTA).
 __device__ inline void select_top_p_gkeys(const uint32_t* gkeys, int c, int p, int32_t* sel, uint8_t* scratch) {
   auto load_key = [&](int id) -> uint32_t { return __ldcg(gkeys + id); };
-  select_top_p_core(load_key, c, p, nullptr, gkeys, sel, scratch);
+  select_top_p_any(load_key, c, p, nullptr, gkeys, sel, scratch);
 }
 
 // ---------------------------------------------------------------------------
