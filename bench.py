@@ -5,8 +5,9 @@ d = 2048, c = 8016 balanced clusters of b = 16, p = 512 probes, bf16 E and C
 -- decoding one hidden state per step (B = 1, greedy), cycling through 1024
 seeded planted/flat hidden states. A step is one ``fh_decode`` call: centroid
 scores, top-p selection, C2T gather, candidate logits and argmax, all in the
-library's fused kernel. L2 is flushed (a 2 x L2 memset, outside the timed
-events) before every step, so C and E come from HBM each time.
+library's fused kernel. Before every step (outside the timed events) a buffer
+twice the L2 is written and read back, so C and E come from HBM each time and
+the L2 holds only clean lines.
 
 Reported: head tokens/s (whole job, all ranks), us/token, the HBM roofline of
 the fused kernel (algorithmic bytes = centroid bytes + p*b*d*2 + C2T rows + h +

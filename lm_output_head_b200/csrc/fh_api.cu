@@ -43,7 +43,6 @@ struct fh_head {
   int words = 0;
   int b1_grid = 0;
   int dense_grid = 0;
-  uint32_t* hist = nullptr;            // [max_batch, 4096] batched key histograms
   const uint8_t* crows = nullptr;      // centroid rows (bf16 borrowed, or packed INT4 in ws)
   int crow_bytes = 0;
   int nch = 0;
@@ -93,7 +92,7 @@ int ring_slots(size_t budget, size_t fixed, size_t slot) {
 }
 
 fh_status launch_scores_rows(fh_head* h, const void* hidden, int32_t B, int mode, float T,
-                             const float* u, float* out, uint32_t* hist, cudaStream_t st) {
+                             const float* u, float* out, cudaStream_t st) {
   const fh_head_desc& D = h->desc;
   const size_t slot = up(static_cast<size_t>(h->crow_bytes), 128);
   const int nslot = 2;
@@ -109,7 +108,6 @@ fh_status launch_scores_rows(fh_head* h, const void* hidden, int32_t B, int mode
     P.hidden = static_cast<const uint16_t*>(hidden);
     P.u_clusters = u;
     P.out = out;
-    P.hist = hist;
     P.status = &h->sync->status;
     P.d = D.d;
     P.c = D.c;
@@ -238,7 +236,6 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   const size_t o_log = take(mb * nc * 4);
   const size_t o_rok = take(mb * 4);
   const size_t o_cnt = take(static_cast<size_t>(D.v) * 4);
-  const size_t o_hist = take(mb * kHistBins * 4);
   const int words = (D.c + 31) / 32;
   const size_t o_keys1 = take(static_cast<size_t>(D.c) * 4);
   const size_t o_zrow = take(nc * 4);
@@ -268,7 +265,6 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   h->b1_z_row = reinterpret_cast<float*>(h->ws + o_zrow);
   h->b1_queue = reinterpret_cast<int32_t*>(h->ws + o_queue);
   h->words = words;
-  h->hist = reinterpret_cast<uint32_t*>(h->ws + o_hist);
   h->crows = D.fmt == FH_CENTROID_INT4_G32 ? h->ws + o_crow : static_cast<const uint8_t*>(D.C);
 
   fh_status status = FH_OK;
@@ -322,7 +318,8 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
     h->b1_off_slots = static_cast<int>(o);
     h->b1_slot_bytes = static_cast<int>(up(std::max(static_cast<size_t>(h->crow_bytes), static_cast<size_t>(D.d) * 2), 128));
     // the slots double as the selector's scratch once phase 1 is done
-    o += std::max(static_cast<size_t>(kWarps) * h->b1_slot_bytes, hist_select_smem_bytes(D.c, false));
+    o += std::max(std::max(static_cast<size_t>(kWarps) * h->b1_slot_bytes, hist_select_smem_bytes(D.c)),
+                  up(sizeof(FastSelSmem), 128) + up(static_cast<size_t>(D.c), 128));
     h->b1_smem = o;
     int blocks = 0;
     e = occupancy_decode_b1(D.fmt == FH_CENTROID_INT4_G32, h->nch, h->b1_smem, &blocks);
@@ -391,7 +388,7 @@ fh_status fh_centroid_scores(fh_head* h, const void* hidden, int32_t B, float* s
   fh_status s = check_call(h, hidden, B);
   if (s != FH_OK) return s;
   if (!scores || !aligned(scores, 4)) return FH_ERR_INVALID_ARG;
-  return launch_scores_rows(h, hidden, B, 0, 1.f, nullptr, scores, nullptr, reinterpret_cast<cudaStream_t>(stream));
+  return launch_scores_rows(h, hidden, B, 0, 1.f, nullptr, scores, reinterpret_cast<cudaStream_t>(stream));
 }
 
 fh_status fh_select_clusters(fh_head* h, const float* scores, int32_t B, int32_t p, int32_t mode, float T,
@@ -492,11 +489,10 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
   }
 
   // batched path: keys -> per-row select -> candidates -> epilogue
-  s = launch_scores_rows(h, hidden, B, gumbel ? 1 : 0, gumbel ? T : 1.f, u_clusters, h->keys, h->hist, st);
+  s = launch_scores_rows(h, hidden, B, gumbel ? 1 : 0, gumbel ? T : 1.f, u_clusters, h->keys, st);
   if (s != FH_OK) return s;
   SelectParams SP{};
   SP.in = h->keys;
-  SP.hist = h->hist;
   SP.C2T = D.C2T;
   SP.sel = h->sel;
   SP.cand_tok = h->cand_tok;

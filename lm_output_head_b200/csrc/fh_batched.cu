@@ -51,7 +51,6 @@ __global__ void __launch_bounds__(kThreads, 1) scores_kernel(const ScoresParams 
     const size_t o = static_cast<size_t>(P.row0 + r) * P.c + k;
     const float key = P.mode == 1 ? gumbel_key(s, P.T, __ldg(P.u_clusters + o)) : s;
     P.out[o] = key;
-    if (P.hist) atomicAdd(P.hist + static_cast<size_t>(P.row0 + r) * kHistBins + (f2key(key) >> kHistShift), 1u);
   };
   bool ok;
   if constexpr (INT4) {
@@ -152,10 +151,8 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelectParams 
   uint8_t* scratch = smem + ((static_cast<size_t>(P.p) * 4 + 127) & ~size_t(127));
   const float* in = P.in + static_cast<size_t>(row) * P.c;
   const float* u = P.perturb ? P.u_clusters + static_cast<size_t>(row) * P.c : nullptr;
-  uint32_t* hist = P.hist ? P.hist + static_cast<size_t>(row) * kHistBins : nullptr;
-  select_top_p_hist(in, u, P.T, P.c, P.p, hist, ssel, scratch);
-  if (hist)  // consumed: clear it for the next call
-    for (int i = threadIdx.x; i < kHistBins; i += kThreads) hist[i] = 0u;
+  select_stage_scores(in, u, P.T, P.c, scratch);
+  select_top_p_staged(P.c, P.p, ssel, scratch);
   int32_t* gsel = P.sel + static_cast<size_t>(row) * P.p;
   for (int i = threadIdx.x; i < P.p; i += kThreads) gsel[i] = ssel[i];
   write_candidates(P, ssel, row);

@@ -47,12 +47,6 @@ struct B1Misc {
   int claim, lastpos, last, selector;
 };
 
-// The selector's exact top-p (runs on one CTA per call): kept out of line so
-// that its register-resident keys do not constrain the streaming phases.
-__device__ __noinline__ void selector_top_p(const uint32_t* keys, int c, int p, int32_t* sel, uint8_t* scratch) {
-  select_top_p_gkeys(keys, c, p, sel, scratch);
-}
-
 // Wait (bounded) until `slot` holds a token id written by the selector.
 __device__ __forceinline__ int poll_slot(const int32_t* slot, long long budget) {
   int t = static_cast<int>(ld_relaxed_u32(reinterpret_cast<const unsigned*>(slot)));
@@ -118,6 +112,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   }
   float ureg = 0.f;  // lane j holds u of item j
   if (gumbel && lane < n1) ureg = __ldg(P.u_clusters + cw + lane * cstride);
+  if (lane < n1) prefetch_l2(P.C2T + static_cast<size_t>(cw + lane * cstride) * b);  // for speculation / the selector
+  const float spec_ratio = P.sync->spec_ratio;
   for (int z = static_cast<int>(blockIdx.x) * kThreads + tid; z < P.nc_max; z += G * kThreads)
     P.row_queue[static_cast<size_t>(nxt) * P.nc_max + z] = -1;
   __syncthreads();  // hbar initialised before anyone waits on it
@@ -137,6 +133,19 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     }
     __syncthreads();
   }
+  // Speculation: clusters whose key clears spec_ratio * |h|/sqrt(d) (the last
+  // call's p-th key on that scale, less a margin) get their token rows
+  // prefetched into L2 now, while the selection is still to come.
+  float hscale = 0.f;
+  {
+    float q2 = 0.f;
+    for (int e = lane; e < d; e += 32) q2 = fmaf(hs[e], hs[e], q2);
+    hscale = sqrtf(warp_sum(q2) / static_cast<float>(d));
+    if (gumbel) hscale /= P.T;
+  }
+  const bool spec = spec_ratio != 0.f;
+  const float t_est = spec_ratio * hscale;
+  const float t_spec = t_est - 0.02f * fabsf(t_est);
   for (int i = 0; i < n1; ++i) {
     const int k = cw + i * cstride;
     float s;
@@ -154,9 +163,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     }
     const float u = __shfl_sync(0xFFFFFFFFu, ureg, i & 31);
     const float key = gumbel ? gumbel_key(s, P.T, u) : s;
-    if (lane == 0) {
-      P.keys[k] = f2key(key);
-      prefetch_l2(P.C2T + static_cast<size_t>(k) * b);
+    if (lane == 0) P.keys[k] = f2key(key);
+    if (spec && key >= t_spec) {
+      for (int j = lane; j < b; j += 32) {
+        const int tok = __ldg(P.C2T + static_cast<size_t>(k) * b + j);
+        bulk_prefetch_l2(P.E + static_cast<size_t>(tok) * d, static_cast<uint32_t>(d * 2));
+      }
     }
   }
 
@@ -170,7 +182,19 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   const int r_all = P.p * b;
   if (misc->selector) {
     __threadfence();
-    selector_top_p(P.keys, P.c, P.p, ssel, slots);
+    if (P.c <= kThreads * 16) {
+      select_fast<16>(P.keys, P.c, P.p, ssel, slots);
+    } else if (P.c <= kThreads * 32) {
+      select_fast<32>(P.keys, P.c, P.p, ssel, slots);
+    } else {
+      select_stage_gkeys(P.keys, P.c, slots);
+      select_top_p_staged(P.c, P.p, ssel, slots);
+    }
+    if (tid == 0 && P.c <= kThreads * 32 && hscale > 0.f) {  // prior for the next call's speculation
+      const FastSelSmem& fs = *reinterpret_cast<const FastSelSmem*>(slots);
+      const float tstar = fs.scale > 0.f ? fs.lo + static_cast<float>(fs.t1) / fs.scale : fs.lo;
+      P.sync->spec_ratio = tstar / hscale;
+    }
     if (P.out_cluster_ids)
       for (int i = tid; i < P.p; i += kThreads) P.out_cluster_ids[i] = ssel[i];
     // thread q writes the C2T row of the q-th chosen cluster: slots q*b .. q*b + b - 1

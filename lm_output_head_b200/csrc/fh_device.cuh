@@ -85,6 +85,11 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
+// Bring `bytes` (multiple of 16, 16-byte aligned) into L2 without waiting.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned* p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -348,105 +353,100 @@ __device__ inline void block_select_top_p(const uint32_t* skey, int n, int p, in
 }
 
 // ---------------------------------------------------------------------------
-// histogram-driven top-p select
+// histogram-driven top-p select (compact code: it runs once per call)
 // ---------------------------------------------------------------------------
-// A 4096-bin histogram of the top 12 key bits (sign, exponent, 3 mantissa
-// bits) locates the bin holding the p-th largest key; every key above that
-// bin is taken, and the keys inside it are ranked exactly (key desc, id asc)
-// against each other -- a few hundred at most for real score distributions,
-// so the exact step is a small all-pairs count rather than more radix passes.
-// The histogram either arrives precomputed in global memory (built with
-// fire-and-forget atomics by the kernel that produced the scores) or is
-// built here in shared memory.
+// The keys' value range [lo, hi] is split into 4096 equal-width bins (linear
+// in the key's float value, so even a concentrated score distribution puts
+// only a few dozen keys in any bin and the shared-memory atomics that build
+// the histogram rarely collide). A scan locates the bin holding the p-th
+// largest key; every key above that bin is taken, and the keys inside it are
+// ranked exactly (key desc, id asc) against each other. Keys live in shared
+// memory and every loop stays a loop: the code runs once per call.
 constexpr int kHistBins = 4096;
-constexpr int kHistShift = 20;
-constexpr int kKeysPerThreadMax = 32;          // keys held in registers: c <= 32 * 512
-constexpr int kBoundaryMax = 2048;              // exact all-pairs ranking up to this many ties-in-bin
+constexpr int kBoundaryMax = 2048;  // exact all-pairs ranking up to this many keys in the boundary bin
 
 struct HistSelectSmem {
   uint32_t hist[kHistBins];
   uint32_t ckey[kBoundaryMax];
   int32_t cid[kBoundaryMax];
   uint32_t scan[kWarps + 1];
-  uint32_t wcount[kWarps];
+  uint32_t wmin[kWarps], wmax[kWarps];
   uint32_t t1, above, m1, ncand;
+  float lo, scale;
+  SelectSmem radix;
 };
 
-// Bytes of shared scratch the select needs for c keys: the struct, a c-byte
-// flag array, the radix fallback state, and (when the keys are not in global
-// memory as keys already) c keys for that fallback.
-__host__ __device__ inline size_t hist_select_smem_bytes(int c, bool keys_in_smem = true) {
-  return ((sizeof(HistSelectSmem) + 127) & ~size_t(127)) + ((static_cast<size_t>(c) + 127) & ~size_t(127)) +
-         ((sizeof(SelectSmem) + 127) & ~size_t(127)) +
-         (keys_in_smem ? ((static_cast<size_t>(c) * 4 + 127) & ~size_t(127)) : 0);
+// Shared scratch for c keys: the struct, the keys, a c-byte flag array.
+__host__ __device__ inline size_t hist_select_smem_bytes(int c) {
+  return ((sizeof(HistSelectSmem) + 127) & ~size_t(127)) + ((static_cast<size_t>(c) * 4 + 127) & ~size_t(127)) +
+         ((static_cast<size_t>(c) + 127) & ~size_t(127));
 }
 
-// Core of the histogram-driven select, laid out for short dependency chains:
-// thread t owns the contiguous ids [t*kpt, t*kpt + kpt) (kpt = ceil(c/512)),
-// so one block scan orders the output. `load_key(id)` returns the order-
-// preserving key of cluster id (< c); all of a thread's loads are independent.
-// `hist_g` (global, 4096 bins of key >> 20) may be null: then the histogram
-// is built in shared memory with fire-and-forget atomics. `gkeys`: the same
-// keys in global memory for the radix fallback, or null to stage them in
-// shared memory. Writes the chosen ids ascending to `sel`.
-template <int KMAX, class LoadKey>
-__device__ inline void select_top_p_core(LoadKey load_key, int c, int p, const uint32_t* hist_g,
-                                         const uint32_t* gkeys, int32_t* sel, uint8_t* scratch) {
+__device__ __forceinline__ uint32_t* select_keys_area(uint8_t* scratch) {
+  return reinterpret_cast<uint32_t*>(scratch + ((sizeof(HistSelectSmem) + 127) & ~size_t(127)));
+}
+
+// Monotone bin of an order-preserving key: linear in its float value over [lo, lo + 4096/scale].
+__device__ __forceinline__ uint32_t value_bin(uint32_t key, float lo, float scale) {
+  const float x = (key2f(key) - lo) * scale;
+  return static_cast<uint32_t>(fminf(fmaxf(x, 0.f), static_cast<float>(kHistBins - 1)));
+}
+
+// Top-p of the c keys already staged in select_keys_area(scratch); writes the
+// chosen ids ascending to `sel`. All kThreads threads must call it.
+static __device__ __noinline__ void select_top_p_staged(int c, int p, int32_t* sel, uint8_t* scratch) {
   HistSelectSmem& sm = *reinterpret_cast<HistSelectSmem*>(scratch);
-  uint8_t* flag = scratch + ((sizeof(HistSelectSmem) + 127) & ~size_t(127));
-  SelectSmem* fsm = reinterpret_cast<SelectSmem*>(flag + ((static_cast<size_t>(c) + 127) & ~size_t(127)));
-  uint32_t* skey =
-      reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(fsm) + ((sizeof(SelectSmem) + 127) & ~size_t(127)));
-  const int tid = threadIdx.x;
+  const uint32_t* key = select_keys_area(scratch);
+  uint8_t* flag = reinterpret_cast<uint8_t*>(select_keys_area(scratch)) + ((static_cast<size_t>(c) * 4 + 127) & ~size_t(127));
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  if (c > kThreads * KMAX) {  // too many keys for registers: radix select
-    if (!gkeys) {
-      for (int k = tid; k < c; k += kThreads) skey[k] = load_key(k);
-      __syncthreads();
-    }
-    block_select_top_p(gkeys ? gkeys : skey, c, p, sel, *fsm);
-    return;
+  // value range of the keys
+  uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+  for (int k = tid; k < c; k += kThreads) {
+    mn = min(mn, key[k]);
+    mx = max(mx, key[k]);
   }
-
-  const int kpt = (c + kThreads - 1) / kThreads;
-  const int id0 = tid * kpt;
-  uint32_t key[KMAX];
-#pragma unroll
-  for (int i = 0; i < KMAX; ++i) {
-    const int id = id0 + i;
-    key[i] = (i < kpt && id < c) ? load_key(id) : 0u;
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = min(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
+    mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
   }
+  if (lane == 0) {
+    sm.wmin[warp] = mn;
+    sm.wmax[warp] = mx;
+  }
+  for (int i = tid; i < kHistBins; i += kThreads) sm.hist[i] = 0u;
   for (int i = tid; i < (c + 15) / 16; i += kThreads) reinterpret_cast<uint4*>(flag)[i] = make_uint4(0, 0, 0, 0);
-  if (hist_g == nullptr) {
-    for (int i = tid; i < kHistBins; i += kThreads) sm.hist[i] = 0u;
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < KMAX; ++i)
-      if (i < kpt && id0 + i < c) atomicAdd(&sm.hist[key[i] >> kHistShift], 1u);
-  } else {
-    for (int i = tid; i < kHistBins; i += kThreads) sm.hist[i] = __ldcg(hist_g + i);
+  __syncthreads();
+  if (tid == 0) {
+    for (int w = 0; w < kWarps; ++w) {
+      mn = min(mn, sm.wmin[w]);
+      mx = max(mx, sm.wmax[w]);
+    }
+    const float flo = key2f(mn), fhi = key2f(mx);
+    const float span = fhi - flo;
+    sm.lo = flo;
+    sm.scale = span > 0.f ? static_cast<float>(kHistBins) / span : 0.f;
+    sm.ncand = 0u;
   }
-  if (tid == 0) sm.ncand = 0u;
+  __syncthreads();
+  const float lo = sm.lo, scale = sm.scale;
+#pragma unroll 4
+  for (int k = tid; k < c; k += kThreads) atomicAdd(&sm.hist[value_bin(key[k], lo, scale)], 1u);
   __syncthreads();
 
   // bin t1 holding the p-th largest key: thread t owns bins 4095-8t .. 4088-8t
   constexpr int kBpt = kHistBins / kThreads;
-  uint32_t hv[kBpt], loc = 0;
-#pragma unroll
+  uint32_t loc = 0;
+  for (int i = 0; i < kBpt; ++i) loc += sm.hist[kHistBins - 1 - kBpt * tid - i];
+  uint32_t run = block_exclusive_scan<kThreads, uint32_t>(loc, sm.scan, nullptr);
   for (int i = 0; i < kBpt; ++i) {
-    hv[i] = sm.hist[kHistBins - 1 - kBpt * tid - i];
-    loc += hv[i];
-  }
-  const uint32_t above = block_exclusive_scan<kThreads, uint32_t>(loc, sm.scan, nullptr);
-  uint32_t run = above;
-#pragma unroll
-  for (int i = 0; i < kBpt; ++i) {
-    if (run < static_cast<uint32_t>(p) && run + hv[i] >= static_cast<uint32_t>(p)) {
+    const uint32_t h = sm.hist[kHistBins - 1 - kBpt * tid - i];
+    if (run < static_cast<uint32_t>(p) && run + h >= static_cast<uint32_t>(p)) {
       sm.t1 = static_cast<uint32_t>(kHistBins - 1 - kBpt * tid - i);
       sm.above = run;
-      sm.m1 = hv[i];
+      sm.m1 = h;
     }
-    run += hv[i];
+    run += h;
   }
   __syncthreads();
   const uint32_t t1 = sm.t1, m1 = sm.m1;
@@ -454,24 +454,18 @@ __device__ inline void select_top_p_core(LoadKey load_key, int c, int p, const u
   const bool all_in_bin = (m1 == need);
 
   if (!all_in_bin && m1 > static_cast<uint32_t>(kBoundaryMax)) {  // pathological ties: radix fallback
-    if (!gkeys) {
-#pragma unroll
-      for (int i = 0; i < KMAX; ++i)
-        if (i < kpt && id0 + i < c) skey[id0 + i] = key[i];
-      __syncthreads();
-    }
-    block_select_top_p(gkeys ? gkeys : skey, c, p, sel, *fsm);
+    block_select_top_p(key, c, p, sel, sm.radix);
     return;
   }
   if (!all_in_bin) {
     // gather the boundary bin, rank it exactly (key desc, id asc), flag the chosen ids
-#pragma unroll
-    for (int i = 0; i < KMAX; ++i) {
-      if (i < kpt && id0 + i < c && (key[i] >> kHistShift) == t1) {
+    for (int k = tid; k < c; k += kThreads) {
+      const uint32_t kk = key[k];
+      if (value_bin(kk, lo, scale) == t1) {
         const uint32_t at = atomicAdd(&sm.ncand, 1u);
         if (at < static_cast<uint32_t>(kBoundaryMax)) {
-          sm.ckey[at] = key[i];
-          sm.cid[at] = id0 + i;
+          sm.ckey[at] = kk;
+          sm.cid[at] = k;
         }
       }
     }
@@ -481,15 +475,8 @@ __device__ inline void select_top_p_core(LoadKey load_key, int c, int p, const u
       const uint32_t ka = sm.ckey[a];
       const int ia = sm.cid[a];
       uint32_t r = 0;
-      uint32_t bb = 0;
-      for (; bb + 8 <= nb; bb += 8) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint32_t kb = sm.ckey[bb + u];
-          r += (kb > ka) || (kb == ka && sm.cid[bb + u] < ia);
-        }
-      }
-      for (; bb < nb; ++bb) {
+#pragma unroll 8
+      for (uint32_t bb = 0; bb < nb; ++bb) {
         const uint32_t kb = sm.ckey[bb];
         r += (kb > ka) || (kb == ka && sm.cid[bb] < ia);
       }
@@ -498,54 +485,187 @@ __device__ inline void select_top_p_core(LoadKey load_key, int c, int p, const u
     __syncthreads();
   }
 
-  // ascending-id compaction: one block scan of per-thread counts
+  // ascending-id compaction: thread t owns ids [t*kpt, t*kpt + kpt); one block scan
+  const int kpt = (c + kThreads - 1) / kThreads;
+  const int id0 = min(c, tid * kpt), id1 = min(c, id0 + kpt);
   uint32_t cnt = 0;
-#pragma unroll
-  for (int i = 0; i < KMAX; ++i) {
-    const int id = id0 + i;
-    const uint32_t dg = key[i] >> kHistShift;
-    cnt += (i < kpt && id < c && (dg > t1 || (dg == t1 && (all_in_bin || flag[id])))) ? 1u : 0u;
+  for (int k = id0; k < id1; ++k) {
+    const uint32_t bn = value_bin(key[k], lo, scale);
+    cnt += (bn > t1 || (bn == t1 && (all_in_bin || flag[k]))) ? 1u : 0u;
   }
   uint32_t pos = block_exclusive_scan<kThreads, uint32_t>(cnt, sm.scan, nullptr);
-#pragma unroll
-  for (int i = 0; i < KMAX; ++i) {
-    const int id = id0 + i;
-    const uint32_t dg = key[i] >> kHistShift;
-    if (i < kpt && id < c && (dg > t1 || (dg == t1 && (all_in_bin || flag[id])))) {
-      if (pos < static_cast<uint32_t>(p)) sel[pos] = id;
+  for (int k = id0; k < id1; ++k) {
+    const uint32_t bn = value_bin(key[k], lo, scale);
+    if (bn > t1 || (bn == t1 && (all_in_bin || flag[k]))) {
+      if (pos < static_cast<uint32_t>(p)) sel[pos] = k;
       ++pos;
     }
   }
   __syncthreads();
 }
 
-// Dispatch on the number of keys each thread holds in registers.
-template <class LoadKey>
-__device__ inline void select_top_p_any(LoadKey load_key, int c, int p, const uint32_t* hist_g, const uint32_t* gkeys,
-                                        int32_t* sel, uint8_t* scratch) {
-  if (c <= kThreads * 8) select_top_p_core<8>(load_key, c, p, hist_g, gkeys, sel, scratch);
-  else if (c <= kThreads * 16) select_top_p_core<16>(load_key, c, p, hist_g, gkeys, sel, scratch);
-  else select_top_p_core<kKeysPerThreadMax>(load_key, c, p, hist_g, gkeys, sel, scratch);
+// Top-p for one CTA whose c keys (order-preserving u32, global memory) fit in
+// registers (c <= 16 * 32 * KMAX): warp w holds ids w*Q + 32 i + lane
+// (bank-conflict free), the value-linear histogram is built once in shared
+// memory, a two-level search (warp totals, then one warp) finds the boundary
+// bin, and ballots do the gather and the ascending-id compaction.
+struct FastSelSmem {
+  uint32_t hist[kHistBins];
+  uint32_t ckey[kBoundaryMax];
+  int32_t cid[kBoundaryMax];
+  uint32_t wmin[kWarps], wmax[kWarps], wtot[kWarps], wcnt[kWarps];
+  uint32_t t1, above, m1, ncand;
+  float lo, scale;
+};
+
+template <int KMAX>
+static __device__ __noinline__ void select_fast(const uint32_t* gkeys, int c, int p, int32_t* sel, uint8_t* scratch) {
+  FastSelSmem& sm = *reinterpret_cast<FastSelSmem*>(scratch);
+  uint8_t* flag = scratch + ((sizeof(FastSelSmem) + 127) & ~size_t(127));
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
+  const int Q = ((c + kWarps * 32 - 1) / (kWarps * 32)) * 32;  // ids per warp, multiple of 32
+  const int base = warp * Q;
+  const int nit = Q / 32;
+  uint32_t key[KMAX];
+#pragma unroll
+  for (int i = 0; i < KMAX; ++i) {
+    const int id = base + 32 * i + lane;
+    key[i] = (i < nit && id < c) ? __ldcg(gkeys + id) : 0u;
+  }
+  // value range
+  uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+#pragma unroll
+  for (int i = 0; i < KMAX; ++i) {
+    const int id = base + 32 * i + lane;
+    if (i < nit && id < c) { mn = min(mn, key[i]); mx = max(mx, key[i]); }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = min(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
+    mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+  }
+  if (lane == 0) { sm.wmin[warp] = mn; sm.wmax[warp] = mx; }
+  for (int i = tid; i < kHistBins; i += kThreads) sm.hist[i] = 0u;
+  for (int i = tid; i < (c + 15) / 16; i += kThreads) reinterpret_cast<uint4*>(flag)[i] = make_uint4(0, 0, 0, 0);
+  if (tid == 0) sm.ncand = 0u;
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) { mn = min(mn, sm.wmin[w]); mx = max(mx, sm.wmax[w]); }
+  const float lo = key2f(mn), span = key2f(mx) - lo;
+  const float scale = span > 0.f ? static_cast<float>(kHistBins) / span : 0.f;
+  if (tid == 0) {
+    sm.lo = lo;
+    sm.scale = scale;
+  }
+  uint32_t bin[KMAX];
+#pragma unroll
+  for (int i = 0; i < KMAX; ++i) {
+    const int id = base + 32 * i + lane;
+    bin[i] = value_bin(key[i], lo, scale);
+    if (i < nit && id < c) atomicAdd(&sm.hist[bin[i]], 1u);
+  }
+  __syncthreads();
+  // two-level search from the top: warp w owns bins [4095 - 256 w - 255, 4095 - 256 w]
+  {
+    uint32_t s = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s += sm.hist[kHistBins - 1 - 256 * warp - (lane + 32 * i)];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+    if (lane == 0) sm.wtot[warp] = s;
+  }
+  __syncthreads();
+  {
+    uint32_t above_w = 0;
+    for (int w = 0; w < warp; ++w) above_w += sm.wtot[w];
+    const uint32_t pp = static_cast<uint32_t>(p);
+    if (above_w < pp && above_w + sm.wtot[warp] >= pp) {
+      // this warp's 256 bins, descending: lane l owns 8 consecutive bins 4095-256w-8l .. -7
+      uint32_t hv[8], s = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { hv[i] = sm.hist[kHistBins - 1 - 256 * warp - 8 * lane - i]; s += hv[i]; }
+      uint32_t incl = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) { const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o); if (lane >= o) incl += y; }
+      uint32_t run = above_w + incl - s;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (run < pp && run + hv[i] >= pp) { sm.t1 = kHistBins - 1 - 256 * warp - 8 * lane - i; sm.above = run; sm.m1 = hv[i]; }
+        run += hv[i];
+      }
+    }
+  }
+  __syncthreads();
+  const uint32_t t1 = sm.t1, m1 = sm.m1, need = static_cast<uint32_t>(p) - sm.above;
+  const bool all_in_bin = m1 == need;
+  if (!all_in_bin) {
+#pragma unroll
+    for (int i = 0; i < KMAX; ++i) {
+      const int id = base + 32 * i + lane;
+      const bool in = i < nit && id < c && bin[i] == t1;
+      const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
+      if (m) {
+        uint32_t at0 = 0;
+        if (lane == 0) at0 = atomicAdd(&sm.ncand, static_cast<uint32_t>(__popc(m)));
+        at0 = __shfl_sync(0xFFFFFFFFu, at0, 0);
+        const uint32_t at = at0 + __popc(m & lt);
+        if (in && at < static_cast<uint32_t>(kBoundaryMax)) { sm.ckey[at] = key[i]; sm.cid[at] = id; }
+      }
+    }
+    __syncthreads();
+    const uint32_t nb = min(sm.ncand, static_cast<uint32_t>(kBoundaryMax));
+    for (uint32_t a = tid; a < nb; a += kThreads) {
+      const uint32_t ka = sm.ckey[a];
+      const int ia = sm.cid[a];
+      uint32_t r = 0;
+#pragma unroll 8
+      for (uint32_t bb = 0; bb < nb; ++bb) { const uint32_t kb = sm.ckey[bb]; r += (kb > ka) || (kb == ka && sm.cid[bb] < ia); }
+      if (r < need) flag[ia] = 1;
+    }
+    __syncthreads();
+  }
+  // ballot compaction in id order
+  uint32_t cnt = 0, tm[KMAX];
+#pragma unroll
+  for (int i = 0; i < KMAX; ++i) {
+    const int id = base + 32 * i + lane;
+    const bool take = i < nit && id < c && (bin[i] > t1 || (bin[i] == t1 && (all_in_bin || flag[id])));
+    tm[i] = __ballot_sync(0xFFFFFFFFu, take);
+    cnt += __popc(tm[i]);
+  }
+  if (lane == 0) sm.wcnt[warp] = cnt;
+  __syncthreads();
+  uint32_t pos = 0;
+  for (int w = 0; w < warp; ++w) pos += sm.wcnt[w];
+#pragma unroll
+  for (int i = 0; i < KMAX; ++i) {
+    const int id = base + 32 * i + lane;
+    if ((tm[i] >> lane) & 1u) { const uint32_t at = pos + __popc(tm[i] & lt); if (at < static_cast<uint32_t>(p)) sel[at] = id; }
+    pos += __popc(tm[i]);
+  }
+  __syncthreads();
 }
 
-// Top-p of the c keys derived from `scores` (global, read through L2):
-// key = scores[k], or the Gumbel key scores[k]/T - ln(-ln u[k]) when u != null.
-// `hist_g` (global, 4096 bins of key >> 20) may be null. Writes the chosen
-// ids in ascending order to `sel`. All kThreads threads must call it.
-__device__ inline void select_top_p_hist(const float* scores, const float* u, float T, int c, int p,
-                                         const uint32_t* hist_g, int32_t* sel, uint8_t* scratch) {
-  auto load_key = [&](int id) -> uint32_t {
-    float v = __ldcg(scores + id);
-    if (u) v = gumbel_key(v, T, __ldcg(u + id));
-    return f2key(v);
-  };
-  select_top_p_any(load_key, c, p, hist_g, nullptr, sel, scratch);
+// Stage keys: order-preserving u32 keys from global memory (4 in flight per thread).
+__device__ __forceinline__ void select_stage_gkeys(const uint32_t* gkeys, int c, uint8_t* scratch) {
+  uint32_t* key = select_keys_area(scratch);
+#pragma unroll 4
+  for (int k = threadIdx.x; k < c; k += kThreads) key[k] = __ldcg(gkeys + k);
+  __syncthreads();
 }
 
-// Top-p of order-preserving keys already in global memory (one reader CTA).
-__device__ inline void select_top_p_gkeys(const uint32_t* gkeys, int c, int p, int32_t* sel, uint8_t* scratch) {
-  auto load_key = [&](int id) -> uint32_t { return __ldcg(gkeys + id); };
-  select_top_p_any(load_key, c, p, nullptr, gkeys, sel, scratch);
+// Stage keys from fp32 scores, optionally Gumbel-perturbed: scores/T - ln(-ln u).
+__device__ __forceinline__ void select_stage_scores(const float* scores, const float* u, float T, int c,
+                                                    uint8_t* scratch) {
+  uint32_t* key = select_keys_area(scratch);
+#pragma unroll 4
+  for (int k = threadIdx.x; k < c; k += kThreads) {
+    float v = __ldcg(scores + k);
+    if (u) v = gumbel_key(v, T, __ldcg(u + k));
+    key[k] = f2key(v);
+  }
+  __syncthreads();
 }
 
 // ---------------------------------------------------------------------------

@@ -22,8 +22,9 @@ struct SyncWords {
   uint32_t ticket;        // kernel exit tickets (last CTA finalises)
   uint32_t union_count;   // distinct clusters of the last batched decode
   uint32_t epoch;         // fused B = 1 calls so far (selects the per-call buffers)
-  uint32_t arrive2;       // second barrier (boundary list complete)
-  uint32_t pad[2];
+  uint32_t arrive2;       // second barrier (unused by the current kernels)
+  float spec_ratio;       // p-th key / (|h| / sqrt(d)) of the last fused call: speculation prior
+  uint32_t pad;
 };
 
 struct B1Params {
@@ -54,7 +55,6 @@ struct ScoresParams {
   const uint16_t* hidden;  // [B, d]
   const float* u_clusters; // [B, c] (gumbel)
   float* out;              // [B, c]
-  uint32_t* hist;          // [B, 4096] key histograms (accumulated), or null
   int*  status;
   int d, c, crow_bytes;
   int row0, rows;          // hidden rows [row0, row0+rows) in this launch
@@ -66,7 +66,6 @@ struct ScoresParams {
 
 struct SelectParams {
   const float* in;         // [B, c] scores or keys
-  uint32_t* hist;          // [B, 4096] key histograms of `in` (cleared after use), or null
   const float* u_clusters; // [B, c] when perturb
   const int32_t* ids_in;   // [B, p] explicit ids (sort mode) or null
   const int32_t* C2T;
