@@ -39,7 +39,7 @@ struct fh_head {
   uint32_t* c2t_counts = nullptr;      // [v]
   uint32_t* b1_keys = nullptr;         // fused B = 1 state
   float* b1_z_row = nullptr;
-  int32_t* b1_queue = nullptr;
+  int32_t* b1_sel = nullptr;
   int words = 0;
   int b1_grid = 0;
   int dense_grid = 0;
@@ -239,7 +239,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   const int words = (D.c + 31) / 32;
   const size_t o_keys1 = take(static_cast<size_t>(D.c) * 4);
   const size_t o_zrow = take(nc * 4);
-  const size_t o_queue = take(2 * nc * 4);
+  const size_t o_sel1 = take(static_cast<size_t>(mp) * 4);
   const size_t o_crow = D.fmt == FH_CENTROID_INT4_G32 ? take(static_cast<size_t>(D.c) * h->crow_bytes) : 0;
   h->ws_bytes = off;
 
@@ -263,7 +263,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   h->c2t_counts = reinterpret_cast<uint32_t*>(h->ws + o_cnt);
   h->b1_keys = reinterpret_cast<uint32_t*>(h->ws + o_keys1);
   h->b1_z_row = reinterpret_cast<float*>(h->ws + o_zrow);
-  h->b1_queue = reinterpret_cast<int32_t*>(h->ws + o_queue);
+  h->b1_sel = reinterpret_cast<int32_t*>(h->ws + o_sel1);
   h->words = words;
   h->crows = D.fmt == FH_CENTROID_INT4_G32 ? h->ws + o_crow : static_cast<const uint8_t*>(D.C);
 
@@ -284,7 +284,6 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
       }
     }
     e = cudaMemsetAsync(h->ws, 0, h->ws_bytes, st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(h->b1_queue, 0xFF, 2 * nc * 4, st);  // empty row-queue slots are -1
     if (e != cudaSuccess) { status = cuda_fail(e); break; }
     C2TCheckParams cp{D.C2T, h->c2t_counts, &h->sync->status, static_cast<long long>(D.v), D.v};
     e = launch_c2t_check(cp, st);
@@ -319,7 +318,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
     h->b1_slot_bytes = static_cast<int>(up(std::max(static_cast<size_t>(h->crow_bytes), static_cast<size_t>(D.d) * 2), 128));
     // the slots double as the selector's scratch once phase 1 is done
     o += std::max(std::max(static_cast<size_t>(kWarps) * h->b1_slot_bytes, hist_select_smem_bytes(D.c)),
-                  up(sizeof(FastSelSmem), 128) + up(static_cast<size_t>(D.c), 128));
+                  up(sizeof(RegSelSmem), 128));
     h->b1_smem = o;
     int blocks = 0;
     e = occupancy_decode_b1(D.fmt == FH_CENTROID_INT4_G32, h->nch, h->b1_smem, &blocks);
@@ -466,7 +465,7 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
     P.out_max_logit = out_max_logit;
     P.keys = h->b1_keys;
     P.z_row = h->b1_z_row;
-    P.row_queue = h->b1_queue;
+    P.sel_list = h->b1_sel;
     P.best = h->best;
     P.sync = h->sync;
     P.v = D.v;
@@ -474,7 +473,6 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
     P.c = D.c;
     P.b = D.b;
     P.p = p;
-    P.nc_max = D.max_probes * D.b;
     P.crow_bytes = h->crow_bytes;
     P.mode = mode;
     P.T = gumbel ? T : 1.f;

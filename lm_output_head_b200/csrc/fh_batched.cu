@@ -148,11 +148,12 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelectParams 
   extern __shared__ __align__(1024) uint8_t smem[];
   const int row = blockIdx.x;
   int32_t* ssel = reinterpret_cast<int32_t*>(smem);
-  uint8_t* scratch = smem + ((static_cast<size_t>(P.p) * 4 + 127) & ~size_t(127));
+  const uint32_t scratch_off = static_cast<uint32_t>((static_cast<size_t>(P.p) * 4 + 127) & ~size_t(127));
+  uint8_t* scratch = smem + scratch_off;
   const float* in = P.in + static_cast<size_t>(row) * P.c;
   const float* u = P.perturb ? P.u_clusters + static_cast<size_t>(row) * P.c : nullptr;
   select_stage_scores(in, u, P.T, P.c, scratch);
-  select_top_p_staged(P.c, P.p, ssel, scratch);
+  select_top_p_staged(P.c, P.p, 0u, scratch_off);
   int32_t* gsel = P.sel + static_cast<size_t>(row) * P.p;
   for (int i = threadIdx.x; i < P.p; i += kThreads) gsel[i] = ssel[i];
   write_candidates(P, ssel, row);

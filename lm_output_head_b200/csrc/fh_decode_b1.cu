@@ -15,20 +15,21 @@
 //  2. the last CTA to finish phase 1 (one atomic ticket) becomes the
 //     selector: it reads the c keys once, selects the p largest exactly
 //     (key desc, id asc; histogram + exact rank of the boundary bin in shared
-//     memory) and writes the p*b candidate token ids -- slot q*b + j holds
-//     C2T[k_q][j] for the q-th chosen cluster k_q in ascending order
-//     (section 1.2.1) -- into a row queue: the canonical candidate order.
-//  3. candidate row r belongs to CTA r mod G, warp (r / G) mod 16; each warp
-//     polls only its own queue slots, then streams its rows (first in
-//     registers, second into its slot) and keeps a packed (logit, token)
-//     maximum (section 1.2.4, stage 2).
+//     memory), publishes the chosen ids in ascending order and raises a
+//     ready flag. Candidate row r is then slot r % b of the (r / b)-th chosen
+//     cluster: the canonical candidate order (section 1.2.1).
+//  3. one thread per CTA polls the flag with backoff; candidate row r belongs
+//     to CTA r mod G, warp (r / G) mod 16, which maps it through C2T (rows
+//     prefetched to L2 in phase 1), streams it (first row in registers,
+//     second into its slot) and keeps a packed (logit, token) maximum
+//     (section 1.2.4, stage 2).
 //  4. CTA maxima meet in one 64-bit atomicMax; the last CTA to finish (exit
 //     ticket) writes the token: the argmax, or, when sampling, the inverse-CDF
-//     draw over softmax(z/T) walking the queue in order.
+//     draw over softmax(z/T) walking the candidates in canonical order.
 //
-// Device-wide coordination is two atomic tickets and polls of distinct queue
-// lines; no device-wide barrier, no histogram atomics on hot lines, and no
-// CTA but the selector reads all c keys. HBM traffic is the algorithmic
+// Device-wide coordination is two atomic tickets and one flag; no
+// device-wide barrier, no histogram atomics on hot lines, and no CTA but the
+// selector reads all c keys. HBM traffic is the algorithmic
 // minimum: each centroid row once, each selected token row once, plus C2T
 // rows and h.
 #include <climits>
@@ -47,19 +48,6 @@ struct B1Misc {
   int claim, lastpos, last, selector;
 };
 
-// Wait (bounded) until `slot` holds a token id written by the selector.
-__device__ __forceinline__ int poll_slot(const int32_t* slot, long long budget) {
-  int t = static_cast<int>(ld_relaxed_u32(reinterpret_cast<const unsigned*>(slot)));
-  if (t >= 0) return t;
-  const long long t0 = clock64();
-  for (;;) {
-    __nanosleep(64);
-    t = static_cast<int>(ld_relaxed_u32(reinterpret_cast<const unsigned*>(slot)));
-    if (t >= 0) return t;
-    if (clock64() - t0 > budget) return -1;
-  }
-}
-
 template <int NCH, bool INT4>
 __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -73,10 +61,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   B1Misc* misc = reinterpret_cast<B1Misc*>(smem + P.off_misc);
   uint8_t* slots = smem + P.off_slots;  // per-warp row slots; the selector's scratch after phase 1
 
-  // the row queue has two buffers used by alternate calls; this call clears the other one
-  const uint32_t epoch = P.sync->epoch;
-  const uint32_t par = epoch & 1u, nxt = par ^ 1u;
-  int32_t* rq = P.row_queue + static_cast<size_t>(par) * P.nc_max;
+  const uint32_t epoch = P.sync->epoch;  // calls on one head are stream-ordered
 
   // ---------------- phase 1: centroid scores ----------------
   const uint32_t hbar = smem_addr(&misc->hbar);
@@ -112,10 +97,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   }
   float ureg = 0.f;  // lane j holds u of item j
   if (gumbel && lane < n1) ureg = __ldg(P.u_clusters + cw + lane * cstride);
-  if (lane < n1) prefetch_l2(P.C2T + static_cast<size_t>(cw + lane * cstride) * b);  // for speculation / the selector
-  const float spec_ratio = P.sync->spec_ratio;
-  for (int z = static_cast<int>(blockIdx.x) * kThreads + tid; z < P.nc_max; z += G * kThreads)
-    P.row_queue[static_cast<size_t>(nxt) * P.nc_max + z] = -1;
+  if (lane < n1) prefetch_l2(P.C2T + static_cast<size_t>(cw + lane * cstride) * b);  // read in phase 3 if chosen
   __syncthreads();  // hbar initialised before anyone waits on it
   if (!mbar_wait_bounded(hbar, 0u, kWaitBudget) && lane == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
   {
@@ -133,19 +115,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     }
     __syncthreads();
   }
-  // Speculation: clusters whose key clears spec_ratio * |h|/sqrt(d) (the last
-  // call's p-th key on that scale, less a margin) get their token rows
-  // prefetched into L2 now, while the selection is still to come.
-  float hscale = 0.f;
-  {
-    float q2 = 0.f;
-    for (int e = lane; e < d; e += 32) q2 = fmaf(hs[e], hs[e], q2);
-    hscale = sqrtf(warp_sum(q2) / static_cast<float>(d));
-    if (gumbel) hscale /= P.T;
-  }
-  const bool spec = spec_ratio != 0.f;
-  const float t_est = spec_ratio * hscale;
-  const float t_spec = t_est - 0.02f * fabsf(t_est);
   for (int i = 0; i < n1; ++i) {
     const int k = cw + i * cstride;
     float s;
@@ -164,12 +133,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     const float u = __shfl_sync(0xFFFFFFFFu, ureg, i & 31);
     const float key = gumbel ? gumbel_key(s, P.T, u) : s;
     if (lane == 0) P.keys[k] = f2key(key);
-    if (spec && key >= t_spec) {
-      for (int j = lane; j < b; j += 32) {
-        const int tok = __ldg(P.C2T + static_cast<size_t>(k) * b + j);
-        bulk_prefetch_l2(P.E + static_cast<size_t>(tok) * d, static_cast<uint32_t>(d * 2));
-      }
-    }
   }
 
   // ---------------- phase 2: the last CTA to finish selects ----------------
@@ -183,51 +146,60 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   if (misc->selector) {
     __threadfence();
     if (P.c <= kThreads * 16) {
-      select_fast<16>(P.keys, P.c, P.p, ssel, slots);
+      select_reg<16>(P.keys, P.c, P.p, P.off_sel, P.off_slots);
     } else if (P.c <= kThreads * 32) {
-      select_fast<32>(P.keys, P.c, P.p, ssel, slots);
+      select_reg<32>(P.keys, P.c, P.p, P.off_sel, P.off_slots);
     } else {
       select_stage_gkeys(P.keys, P.c, slots);
-      select_top_p_staged(P.c, P.p, ssel, slots);
+      select_top_p_staged(P.c, P.p, P.off_sel, P.off_slots);
     }
-    if (tid == 0 && P.c <= kThreads * 32 && hscale > 0.f) {  // prior for the next call's speculation
-      const FastSelSmem& fs = *reinterpret_cast<const FastSelSmem*>(slots);
-      const float tstar = fs.scale > 0.f ? fs.lo + static_cast<float>(fs.t1) / fs.scale : fs.lo;
-      P.sync->spec_ratio = tstar / hscale;
+    for (int i = tid; i < P.p; i += kThreads) {
+      P.sel_list[i] = ssel[i];
+      if (P.out_cluster_ids) P.out_cluster_ids[i] = ssel[i];
     }
-    if (P.out_cluster_ids)
-      for (int i = tid; i < P.p; i += kThreads) P.out_cluster_ids[i] = ssel[i];
-    // thread q writes the C2T row of the q-th chosen cluster: slots q*b .. q*b + b - 1
-    const bool vec = (b % 4 == 0) && ((reinterpret_cast<uintptr_t>(P.C2T) & 15) == 0);
-    for (int qi = tid; qi < P.p; qi += kThreads) {
-      const int32_t* src = P.C2T + static_cast<size_t>(ssel[qi]) * b;
-      int32_t* dst = rq + static_cast<size_t>(qi) * b;
-      if (vec) {
-        for (int j = 0; j < b; j += 4)
-          *reinterpret_cast<int4*>(dst + j) = __ldg(reinterpret_cast<const int4*>(src + j));
-      } else {
-        for (int j = 0; j < b; ++j) dst[j] = __ldg(src + j);
-      }
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      st_release_u32(&P.sync->ready, epoch + 1u);  // the selection of this call is published
     }
     fence_proxy_async_smem();  // the slots were generic scratch; bulk copies follow
-    __syncthreads();
+  } else {
+    // one thread per CTA waits (bounded, with backoff) for the selector's flag
+    if (tid == 0) {
+      int okw = 1;
+      const long long t0 = clock64();
+      while (ld_acquire_u32(&P.sync->ready) != epoch + 1u) {
+        __nanosleep(200);
+        if (clock64() - t0 > P.spin_budget) {
+          okw = 0;
+          break;
+        }
+      }
+      misc->claim = okw;
+    }
   }
+  __syncthreads();
+  const bool sel_ok = misc->selector || misc->claim;
 
   // ---------------- phase 3: candidate rows ----------------
   // rows r0 = blockIdx + G * warp, r0 + 16 G, ...: two at a time are polled
   // together and streamed together (registers, slot).
   unsigned long long best = 0ull;
   bool ok = true;
-  const long long budget = P.spin_budget;
-  for (int r0 = cw; r0 < r_all; r0 += 2 * cstride) {
+  if (!sel_ok) ok = false;
+  for (int r0 = cw; sel_ok && r0 < r_all; r0 += 2 * cstride) {
     const int r1 = r0 + cstride;
     const bool two = r1 < r_all;
+    // candidate row r is slot r % b of the (r / b)-th chosen cluster (canonical order)
     int t = 0;
-    if (lane == 0) t = poll_slot(rq + r0, budget);
-    else if (lane == 1 && two) t = poll_slot(rq + r1, budget);
+    if (lane == 0 || (lane == 1 && two)) {
+      const int r = lane == 0 ? r0 : r1;
+      const int k = __ldcg(P.sel_list + r / b);
+      t = (k >= 0 && k < P.c) ? __ldg(P.C2T + static_cast<size_t>(k) * b + r % b) : -1;
+    }
     const int t0 = __shfl_sync(0xFFFFFFFFu, t, 0);
     const int t1 = two ? __shfl_sync(0xFFFFFFFFu, t, 1) : 0;
-    if (t0 < 0 || t1 < 0) {
+    if (t0 < 0 || t1 < 0) {  // only an inconsistent selection; never read outside E
       ok = false;
       break;
     }
@@ -280,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
       if (P.out_max_logit) P.out_max_logit[0] = best_logit(bw);
     }
   } else {
-    // inverse CDF over softmax(z/T) in queue order = canonical order (cluster asc, slot asc)
+    // inverse CDF over softmax(z/T) in canonical order (cluster asc, slot asc)
     const float ym = best_logit(bw) / P.T;
     const int qn = (r_all + kThreads - 1) / kThreads;
     const int i0 = min(r_all, tid * qn), i1 = min(r_all, i0 + qn);
@@ -310,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     __syncthreads();
     if (tid == 0) {
       const int idx = misc->claim != INT_MAX ? misc->claim : misc->lastpos;
-      P.out_tokens[0] = __ldcg(rq + idx);
+      P.out_tokens[0] = __ldg(P.C2T + static_cast<size_t>(__ldcg(P.sel_list + idx / b)) * b + idx % b);
       if (P.out_max_logit) P.out_max_logit[0] = best_logit(bw);
     }
   }

@@ -96,6 +96,10 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned* p) {
   return v;
 }
 
+__device__ __forceinline__ void st_release_u32(unsigned* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ uint32_t ld_relaxed_u32(const unsigned* p) {
   uint32_t v;
   asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -392,9 +396,18 @@ __device__ __forceinline__ uint32_t value_bin(uint32_t key, float lo, float scal
   return static_cast<uint32_t>(fminf(fmaxf(x, 0.f), static_cast<float>(kHistBins - 1)));
 }
 
+// The launching kernel's dynamic shared memory. The out-of-line selectors
+// below take byte offsets into it rather than pointers: a pointer argument of
+// a non-inlined function is generic, and generic loads, stores and atomics
+// into shared memory measured 2-3x slower than shared-space ones here.
+extern __shared__ __align__(1024) uint8_t fh_dyn_smem[];
+
 // Top-p of the c keys already staged in select_keys_area(scratch); writes the
-// chosen ids ascending to `sel`. All kThreads threads must call it.
-static __device__ __noinline__ void select_top_p_staged(int c, int p, int32_t* sel, uint8_t* scratch) {
+// chosen ids ascending to `sel` (both byte offsets into the dynamic shared
+// memory). All kThreads threads must call it.
+static __device__ __noinline__ void select_top_p_staged(int c, int p, uint32_t sel_off, uint32_t scratch_off) {
+  int32_t* sel = reinterpret_cast<int32_t*>(fh_dyn_smem + sel_off);
+  uint8_t* scratch = fh_dyn_smem + scratch_off;
   HistSelectSmem& sm = *reinterpret_cast<HistSelectSmem*>(scratch);
   const uint32_t* key = select_keys_area(scratch);
   uint8_t* flag = reinterpret_cast<uint8_t*>(select_keys_area(scratch)) + ((static_cast<size_t>(c) * 4 + 127) & ~size_t(127));
@@ -504,94 +517,151 @@ static __device__ __noinline__ void select_top_p_staged(int c, int p, int32_t* s
   __syncthreads();
 }
 
-// Top-p for one CTA whose c keys (order-preserving u32, global memory) fit in
-// registers (c <= 16 * 32 * KMAX): warp w holds ids w*Q + 32 i + lane
-// (bank-conflict free), the value-linear histogram is built once in shared
-// memory, a two-level search (warp totals, then one warp) finds the boundary
-// bin, and ballots do the gather and the ascending-id compaction.
-struct FastSelSmem {
+// Stage keys: order-preserving u32 keys from global memory (4 in flight per thread).
+__device__ __forceinline__ void select_stage_gkeys(const uint32_t* gkeys, int c, uint8_t* scratch) {
+  uint32_t* key = select_keys_area(scratch);
+#pragma unroll 4
+  for (int k = threadIdx.x; k < c; k += kThreads) key[k] = __ldcg(gkeys + k);
+  __syncthreads();
+}
+
+// Exclusive block scan of one u32 per thread: warp scans by shuffles, one
+// barrier, then every thread adds the totals of the warps before it.
+// `wsum` (kWarps words) must not be reused before the next barrier.
+__device__ __forceinline__ uint32_t block_scan_excl_u32(uint32_t v, uint32_t* wsum, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wsum[warp] = x;
+  __syncthreads();
+  uint32_t before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const uint32_t t = wsum[w];
+    before += w < warp ? t : 0u;
+    all += t;
+  }
+  if (total) *total = all;
+  return before + x - v;
+}
+
+// Top-p for one CTA whose c keys (order-preserving u32 in global memory) fit
+// in registers, KPT per thread (c <= kThreads * KPT). Thread t owns ids
+// t*KPT .. t*KPT + KPT - 1, so each thread's keys are in id order and block
+// scans do the gather and the output. One CTA runs it alone, so it is written
+// for few instructions per key: each key's bin is computed once (in the
+// key's register), then two KPT-bit masks (above / in the boundary bin) carry
+// everything after the histogram. Steps: value range (warp reductions), a
+// value-linear 4096-bin histogram in shared memory, a two-level search for
+// the bin holding the p-th largest key, an id-ordered gather (keys reloaded
+// from global memory) and exact all-pairs rank of that bin (key desc, id
+// asc), and one scan that writes the chosen ids ascending to `sel`. More than
+// kBoundaryMax keys in that bin (heavy ties) falls back to the staged
+// selector. `sel_off` / `scratch_off` are byte offsets into the dynamic
+// shared memory; the scratch must hold hist_select_smem_bytes(c) bytes.
+struct RegSelSmem {
   uint32_t hist[kHistBins];
   uint32_t ckey[kBoundaryMax];
-  int32_t cid[kBoundaryMax];
-  uint32_t wmin[kWarps], wmax[kWarps], wtot[kWarps], wcnt[kWarps];
-  uint32_t t1, above, m1, ncand;
-  float lo, scale;
+  uint8_t ctake[kBoundaryMax];
+  uint32_t wmin[kWarps], wmax[kWarps], wtot[kWarps], wa[kWarps], wb[kWarps];
+  uint32_t t1, above, m1;
 };
 
-template <int KMAX>
-static __device__ __noinline__ void select_fast(const uint32_t* gkeys, int c, int p, int32_t* sel, uint8_t* scratch) {
-  FastSelSmem& sm = *reinterpret_cast<FastSelSmem*>(scratch);
-  uint8_t* flag = scratch + ((sizeof(FastSelSmem) + 127) & ~size_t(127));
+template <int KPT>
+static __device__ __noinline__ void select_reg(const uint32_t* gkeys, int c, int p, uint32_t sel_off,
+                                               uint32_t scratch_off) {
+  static_assert(KPT % 4 == 0 && KPT <= 32, "vector loads of 4 keys; one 32-bit mask per thread");
+  int32_t* sel = reinterpret_cast<int32_t*>(fh_dyn_smem + sel_off);
+  RegSelSmem& sm = *reinterpret_cast<RegSelSmem*>(fh_dyn_smem + scratch_off);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t lt = (1u << lane) - 1u;
-  const int Q = ((c + kWarps * 32 - 1) / (kWarps * 32)) * 32;  // ids per warp, multiple of 32
-  const int base = warp * Q;
-  const int nit = Q / 32;
-  uint32_t key[KMAX];
+  const int id0 = tid * KPT;
+  const int nv = max(0, min(KPT, c - id0));  // valid keys of this thread
+  uint32_t kb[KPT];                          // the keys, then their bins
+  if (nv == KPT && (reinterpret_cast<uintptr_t>(gkeys) & 15) == 0) {
 #pragma unroll
-  for (int i = 0; i < KMAX; ++i) {
-    const int id = base + 32 * i + lane;
-    key[i] = (i < nit && id < c) ? __ldcg(gkeys + id) : 0u;
+    for (int j = 0; j < KPT; j += 4) {
+      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(gkeys + id0 + j));
+      kb[j] = v.x;
+      kb[j + 1] = v.y;
+      kb[j + 2] = v.z;
+      kb[j + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) kb[j] = j < nv ? __ldcg(gkeys + id0 + j) : 0u;
   }
+
   // value range
   uint32_t mn = 0xFFFFFFFFu, mx = 0u;
 #pragma unroll
-  for (int i = 0; i < KMAX; ++i) {
-    const int id = base + 32 * i + lane;
-    if (i < nit && id < c) { mn = min(mn, key[i]); mx = max(mx, key[i]); }
+  for (int j = 0; j < KPT; ++j) {
+    mn = min(mn, j < nv ? kb[j] : 0xFFFFFFFFu);
+    mx = max(mx, kb[j]);  // invalid keys are 0
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    mn = min(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
-    mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+  mn = __reduce_min_sync(0xFFFFFFFFu, mn);
+  mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+  if (lane == 0) {
+    sm.wmin[warp] = mn;
+    sm.wmax[warp] = mx;
   }
-  if (lane == 0) { sm.wmin[warp] = mn; sm.wmax[warp] = mx; }
-  for (int i = tid; i < kHistBins; i += kThreads) sm.hist[i] = 0u;
-  for (int i = tid; i < (c + 15) / 16; i += kThreads) reinterpret_cast<uint4*>(flag)[i] = make_uint4(0, 0, 0, 0);
-  if (tid == 0) sm.ncand = 0u;
+  for (int i = tid; i < kHistBins / 4; i += kThreads) reinterpret_cast<uint4*>(sm.hist)[i] = make_uint4(0, 0, 0, 0);
   __syncthreads();
 #pragma unroll
-  for (int w = 0; w < kWarps; ++w) { mn = min(mn, sm.wmin[w]); mx = max(mx, sm.wmax[w]); }
+  for (int w = 0; w < kWarps; ++w) {
+    mn = min(mn, sm.wmin[w]);
+    mx = max(mx, sm.wmax[w]);
+  }
   const float lo = key2f(mn), span = key2f(mx) - lo;
   const float scale = span > 0.f ? static_cast<float>(kHistBins) / span : 0.f;
-  if (tid == 0) {
-    sm.lo = lo;
-    sm.scale = scale;
-  }
-  uint32_t bin[KMAX];
+
+  // bins (computed once, in place) and the histogram
 #pragma unroll
-  for (int i = 0; i < KMAX; ++i) {
-    const int id = base + 32 * i + lane;
-    bin[i] = value_bin(key[i], lo, scale);
-    if (i < nit && id < c) atomicAdd(&sm.hist[bin[i]], 1u);
+  for (int j = 0; j < KPT; ++j) {
+    kb[j] = value_bin(kb[j], lo, scale);
+    if (j < nv) atomicAdd(&sm.hist[kb[j]], 1u);
   }
   __syncthreads();
-  // two-level search from the top: warp w owns bins [4095 - 256 w - 255, 4095 - 256 w]
+
+  // two-level search from the top: warp w owns bins 4095 - 256 w .. 3840 - 256 w
   {
     uint32_t s = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) s += sm.hist[kHistBins - 1 - 256 * warp - (lane + 32 * i)];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+    s = __reduce_add_sync(0xFFFFFFFFu, s);
     if (lane == 0) sm.wtot[warp] = s;
   }
   __syncthreads();
   {
     uint32_t above_w = 0;
-    for (int w = 0; w < warp; ++w) above_w += sm.wtot[w];
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) above_w += w < warp ? sm.wtot[w] : 0u;
     const uint32_t pp = static_cast<uint32_t>(p);
     if (above_w < pp && above_w + sm.wtot[warp] >= pp) {
-      // this warp's 256 bins, descending: lane l owns 8 consecutive bins 4095-256w-8l .. -7
+      // this warp's 256 bins, descending: lane l owns 8 consecutive bins
       uint32_t hv[8], s = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) { hv[i] = sm.hist[kHistBins - 1 - 256 * warp - 8 * lane - i]; s += hv[i]; }
+      for (int i = 0; i < 8; ++i) {
+        hv[i] = sm.hist[kHistBins - 1 - 256 * warp - 8 * lane - i];
+        s += hv[i];
+      }
       uint32_t incl = s;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) { const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o); if (lane >= o) incl += y; }
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+      }
       uint32_t run = above_w + incl - s;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        if (run < pp && run + hv[i] >= pp) { sm.t1 = kHistBins - 1 - 256 * warp - 8 * lane - i; sm.above = run; sm.m1 = hv[i]; }
+        if (run < pp && run + hv[i] >= pp) {
+          sm.t1 = kHistBins - 1 - 256 * warp - 8 * lane - i;
+          sm.above = run;
+          sm.m1 = hv[i];
+        }
         run += hv[i];
       }
     }
@@ -599,59 +669,49 @@ static __device__ __noinline__ void select_fast(const uint32_t* gkeys, int c, in
   __syncthreads();
   const uint32_t t1 = sm.t1, m1 = sm.m1, need = static_cast<uint32_t>(p) - sm.above;
   const bool all_in_bin = m1 == need;
-  if (!all_in_bin) {
-#pragma unroll
-    for (int i = 0; i < KMAX; ++i) {
-      const int id = base + 32 * i + lane;
-      const bool in = i < nit && id < c && bin[i] == t1;
-      const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
-      if (m) {
-        uint32_t at0 = 0;
-        if (lane == 0) at0 = atomicAdd(&sm.ncand, static_cast<uint32_t>(__popc(m)));
-        at0 = __shfl_sync(0xFFFFFFFFu, at0, 0);
-        const uint32_t at = at0 + __popc(m & lt);
-        if (in && at < static_cast<uint32_t>(kBoundaryMax)) { sm.ckey[at] = key[i]; sm.cid[at] = id; }
-      }
-    }
+  if (!all_in_bin && m1 > static_cast<uint32_t>(kBoundaryMax)) {  // heavy ties: exact staged selector
     __syncthreads();
-    const uint32_t nb = min(sm.ncand, static_cast<uint32_t>(kBoundaryMax));
-    for (uint32_t a = tid; a < nb; a += kThreads) {
+    select_stage_gkeys(gkeys, c, fh_dyn_smem + scratch_off);
+    select_top_p_staged(c, p, sel_off, scratch_off);
+    return;
+  }
+
+  uint32_t gt = 0u, eq = 0u;  // bit j: key j above / in the boundary bin
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    gt |= (j < nv && kb[j] > t1) ? (1u << j) : 0u;
+    eq |= (j < nv && kb[j] == t1) ? (1u << j) : 0u;
+  }
+  if (all_in_bin) {
+    gt |= eq;
+  } else {
+    // id-ordered gather of the boundary bin, exact rank, take flags back
+    const uint32_t boff = block_scan_excl_u32(static_cast<uint32_t>(__popc(eq)), sm.wa, nullptr);
+    uint32_t at = boff;
+    for (uint32_t m = eq; m; m &= m - 1u) sm.ckey[at++] = __ldcg(gkeys + id0 + (__ffs(m) - 1));
+    __syncthreads();
+    for (uint32_t a = tid; a < m1; a += kThreads) {
       const uint32_t ka = sm.ckey[a];
-      const int ia = sm.cid[a];
       uint32_t r = 0;
 #pragma unroll 8
-      for (uint32_t bb = 0; bb < nb; ++bb) { const uint32_t kb = sm.ckey[bb]; r += (kb > ka) || (kb == ka && sm.cid[bb] < ia); }
-      if (r < need) flag[ia] = 1;
+      for (uint32_t bb = 0; bb < m1; ++bb) {
+        const uint32_t kbb = sm.ckey[bb];
+        r += (kbb > ka || (kbb == ka && bb < a)) ? 1u : 0u;  // index order is id order
+      }
+      sm.ctake[a] = r < need ? 1 : 0;
     }
     __syncthreads();
+    at = boff;
+    for (uint32_t m = eq; m; m &= m - 1u)
+      if (sm.ctake[at++]) gt |= 1u << (__ffs(m) - 1);
   }
-  // ballot compaction in id order
-  uint32_t cnt = 0, tm[KMAX];
-#pragma unroll
-  for (int i = 0; i < KMAX; ++i) {
-    const int id = base + 32 * i + lane;
-    const bool take = i < nit && id < c && (bin[i] > t1 || (bin[i] == t1 && (all_in_bin || flag[id])));
-    tm[i] = __ballot_sync(0xFFFFFFFFu, take);
-    cnt += __popc(tm[i]);
-  }
-  if (lane == 0) sm.wcnt[warp] = cnt;
-  __syncthreads();
-  uint32_t pos = 0;
-  for (int w = 0; w < warp; ++w) pos += sm.wcnt[w];
-#pragma unroll
-  for (int i = 0; i < KMAX; ++i) {
-    const int id = base + 32 * i + lane;
-    if ((tm[i] >> lane) & 1u) { const uint32_t at = pos + __popc(tm[i] & lt); if (at < static_cast<uint32_t>(p)) sel[at] = id; }
-    pos += __popc(tm[i]);
-  }
-  __syncthreads();
-}
 
-// Stage keys: order-preserving u32 keys from global memory (4 in flight per thread).
-__device__ __forceinline__ void select_stage_gkeys(const uint32_t* gkeys, int c, uint8_t* scratch) {
-  uint32_t* key = select_keys_area(scratch);
-#pragma unroll 4
-  for (int k = threadIdx.x; k < c; k += kThreads) key[k] = __ldcg(gkeys + k);
+  // ascending-id output
+  uint32_t pos = block_scan_excl_u32(static_cast<uint32_t>(__popc(gt)), sm.wb, nullptr);
+  for (uint32_t m = gt; m; m &= m - 1u) {
+    if (pos < static_cast<uint32_t>(p)) sel[pos] = id0 + (__ffs(m) - 1);
+    ++pos;
+  }
   __syncthreads();
 }
 

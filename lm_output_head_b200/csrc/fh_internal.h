@@ -22,9 +22,8 @@ struct SyncWords {
   uint32_t ticket;        // kernel exit tickets (last CTA finalises)
   uint32_t union_count;   // distinct clusters of the last batched decode
   uint32_t epoch;         // fused B = 1 calls so far (selects the per-call buffers)
-  uint32_t arrive2;       // second barrier (unused by the current kernels)
-  float spec_ratio;       // p-th key / (|h| / sqrt(d)) of the last fused call: speculation prior
-  uint32_t pad;
+  uint32_t ready;         // epoch + 1 once the fused call's cluster selection is published
+  uint32_t pad[2];
 };
 
 struct B1Params {
@@ -38,11 +37,11 @@ struct B1Params {
   int32_t* out_cluster_ids;
   float* out_max_logit;
   uint32_t* keys;         // workspace [c]: order-preserving keys of the clusters
-  float* z_row;           // workspace [nc_max]: candidate logits in queue order (sampling)
-  int32_t* row_queue;     // workspace [2][nc_max]: candidate token ids, -1 until written; alternate calls
+  float* z_row;           // workspace [p*b]: candidate logits in canonical order (sampling)
+  int32_t* sel_list;      // workspace [max_probes]: the chosen cluster ids, ascending
   unsigned long long* best;
   SyncWords* sync;
-  int v, d, c, b, p, nc_max;
+  int v, d, c, b, p;
   int crow_bytes;
   int mode;
   float T;
