@@ -184,6 +184,34 @@ fh_status fh_dense_head(fh_head* head, const void* hidden, int32_t B, float* log
                         int32_t* out_argmax, fh_stream_t stream);
 
 /*
+ * Allocation-free dense head: the same z = E h and argmax as fh_dense_head
+ * (write-up section 1.1), with no handle. The write-up has no counterpart to
+ * this entry point; it serves callers that must not allocate device memory
+ * while they run (a serving process whose allocator already holds the free
+ * HBM; a latency-critical loop, where cudaMalloc / cudaFree may synchronise
+ * the device). It allocates nothing: the kernel's scratch (one word per hidden
+ * row plus an exit ticket) is a fixed 1 KB device array inside this library,
+ * zero between calls.
+ *  E           device bf16 [v, d] row-major, 16-byte aligned; read only.
+ *  v, d        vocabulary size >= 1; hidden size, a multiple of 8, <= 2560.
+ *  hidden      device bf16 [B, d] row-major, 16-byte aligned.
+ *  B           1 .. FH_NOALLOC_MAX_ROWS; a larger B returns FH_ERR_INVALID_ARG
+ *              (the fixed scratch holds FH_NOALLOC_MAX_ROWS rows).
+ *  logits      device fp32 [B, v], or NULL to skip writing them.
+ *  out_argmax  device int32 [B] (lowest token id among equal maxima).
+ * Errors: FH_ERR_INVALID_ARG (null / misaligned pointer, size out of range),
+ * FH_ERR_UNSUPPORTED (d > 2560, or not an sm_100 device), FH_ERR_CUDA.
+ * The first call on each device resolves the scratch's address
+ * (cudaGetSymbolAddress, which may load the module) and sets kernel
+ * attributes: make it before any stream capture begins. All calls on a
+ * device share the scratch: launches that can overlap in time (unordered
+ * streams, concurrent host threads) race and corrupt each other's results.
+ */
+#define FH_NOALLOC_MAX_ROWS 64
+fh_status fh_dense_head_noalloc(const void* E, int32_t v, int32_t d, const void* hidden, int32_t B,
+                                float* logits, int32_t* out_argmax, fh_stream_t stream);
+
+/*
  * Synchronise `stream`, then return and clear the device status word
  * (FH_OK if no kernel recorded an error since the last read).
  */

@@ -34,8 +34,10 @@ FH_QUERY_FUSED_B1 = 3
 EXPORTED = (
     "fh_create", "fh_destroy", "fh_centroid_scores", "fh_select_clusters",
     "fh_candidate_logits", "fh_decode", "fh_dense_head", "fh_get_device_status",
-    "fh_status_string", "fh_set_spin_budget", "fh_query",
+    "fh_status_string", "fh_set_spin_budget", "fh_query", "fh_dense_head_noalloc",
 )
+
+FH_NOALLOC_MAX_ROWS = 64
 
 
 class HeadDesc(ctypes.Structure):
@@ -80,6 +82,8 @@ def load() -> ctypes.CDLL:
     lib.fh_decode.restype = ctypes.c_int
     lib.fh_dense_head.argtypes = [vp, vp, i32, vp, vp, vp]
     lib.fh_dense_head.restype = ctypes.c_int
+    lib.fh_dense_head_noalloc.argtypes = [vp, i32, i32, vp, i32, vp, vp, vp]
+    lib.fh_dense_head_noalloc.restype = ctypes.c_int
     lib.fh_get_device_status.argtypes = [vp, vp]
     lib.fh_get_device_status.restype = ctypes.c_int
     lib.fh_status_string.argtypes = [ctypes.c_int]

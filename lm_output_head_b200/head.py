@@ -186,6 +186,20 @@ class FlashHead:
         return (out_argmax, logits) if want_logits else out_argmax
 
 
+def dense_head_noalloc(E: torch.Tensor, hidden: torch.Tensor, out_argmax: torch.Tensor, *,
+                       logits: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Dense head through ``fh_dense_head_noalloc``: no handle and no device
+    allocation (the caller passes every output). At most
+    ``FH_NOALLOC_MAX_ROWS`` hidden rows per call; calls that may overlap in
+    time share one fixed scratch and must be ordered (e.g. one stream)."""
+    lib = _lib.load()
+    v, d = E.shape
+    B = hidden.shape[0]
+    _check(lib.fh_dense_head_noalloc(_ptr(E), int(v), int(d), _ptr(hidden), int(B), _ptr(logits),
+                                     _ptr(out_argmax), _stream(stream)), "fh_dense_head_noalloc")
+    return out_argmax
+
+
 class HostDecoder:
     """End-to-end decode from pinned host memory: H2D copy of the hidden states
     (and uniforms), ``fh_decode``, D2H copy of the tokens, all on one stream."""
