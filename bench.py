@@ -105,6 +105,13 @@ class ClockSampler:
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
 
+    def wait_first(self, timeout_s: float = 20.0):
+        """Block until nvidia-smi has produced a sample: its start-up must not
+        overlap the warm-up or the timed steps."""
+        t_end = time.time() + timeout_s
+        while self.proc is not None and not self.samples and time.time() < t_end:
+            time.sleep(0.05)
+
     def _read(self):
         for line in self.proc.stdout:
             parts = [x.strip() for x in line.split(",")]
@@ -146,6 +153,29 @@ def dist_setup():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return world, rank, local
+
+
+def rank_states(H, rank):
+    """Replica `rank` decodes the hidden states rotated by 37 rows per rank
+    (rows are independent: no exchange between replicas)."""
+    return np.roll(H, -rank * 37, axis=0)
+
+
+def max_over_ranks(total_ms, world, device):
+    """This rank's device-timed total -> the maximum over all ranks (all_reduce
+    MAX; the tensor lives on the GPU for NCCL, on the host for gloo)."""
+    if world <= 1:
+        return float(total_ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(total_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(total_ms_max, steps, world):
+    """Whole-job tokens/s: every rank decodes `steps` tokens; the job takes the slowest rank's time."""
+    return world * steps / (total_ms_max / 1e3)
 
 
 # ---------------------------------------------------------------------------
@@ -198,7 +228,7 @@ def run_ours(args):
     assert dh.fused_b1, "fused B=1 path unavailable"
     n_states = hid.H.shape[0]
     # each rank decodes its own slice of states (replicas; independent rows)
-    Hdev = fh.bf16_from_bits(np.roll(hid.H, -rank * 37, axis=0), dev)
+    Hdev = fh.bf16_from_bits(rank_states(hid.H, rank), dev)
     out = torch.empty(1, dtype=torch.int32, device=dev)
 
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -243,18 +273,14 @@ def run_ours(args):
 
     sampler = ClockSampler(dev.index)
     sampler.start()
-    time.sleep(0.3)
+    sampler.wait_first()
     ms, w0, w1 = timed_loop(step, args.steps, args.warmup)
     status = dh.device_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed loop")
-    total_ms = sum(ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(ms), world, dev)
     mean_ms = total_ms / args.steps
-    value = world * args.steps / (total_ms / 1e3)
+    value = job_throughput(total_ms, args.steps, world)
 
     # dense comparison (same protocol, fewer steps)
     kd = max(3, min(args.steps, 200))

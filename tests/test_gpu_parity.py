@@ -320,6 +320,51 @@ def test_decode_ragged_hidden_size(fh):
         dh.close()
 
 
+@pytest.mark.parametrize("cfg_id,B", [(0, 1), (0, 4), (1, 1), (1, 3)])
+def test_decode_all_scores_tied(fh, cfg_id, B):
+    """h = 0: every centroid score and every logit is exactly 0, so the order
+    (key desc, id asc) picks clusters 0..p-1 and the lowest candidate token id
+    wins. On the Llama-3.2-1B-shaped head all 8016 keys share one histogram
+    bin, more than the boundary rank takes, so the tie fallback runs."""
+    cfg, head, hid, _, dh = get_cfg(cfg_id, fh)
+    p = cfg.p
+    out_ids = torch.empty((B, p), dtype=torch.int32, device="cuda")
+    tok = dh.decode(hid_dev(np.zeros((B, cfg.d), np.uint16)), p, out_cluster_ids=out_ids).cpu().numpy()
+    assert dh.device_status() == 0
+    ids = out_ids.cpu().numpy()
+    want_tok, _, _ = oracle.decode(head, np.zeros((1, cfg.d), np.uint16), p)
+    for r in range(B):
+        assert np.array_equal(ids[r], np.arange(p))
+        assert tok[r] == int(np.min(head.C2T[:p])) == int(np.asarray(want_tok).ravel()[0])
+
+
+def test_decode_duplicated_centroids(fh):
+    """Centroid rows drawn from three patterns: every key is one of three
+    values, so whole groups tie at the boundary; the chosen set is exact
+    (lowest ids first within the boundary group) on both paths."""
+    cfg, head, hid, _ = synth.make_config(0)
+    rng = np.random.default_rng(77)
+    pat = rng.integers(0, 3, size=cfg.c)
+    C = head.C[np.array([5, 17, 101])[pat]].copy()  # three distinct centroid rows
+    h2 = synth.Head(v=head.v, d=head.d, c=head.c, b=head.b, E=head.E, C=C, C2T=head.C2T)
+    dh = _to_dev(h2, 4, cfg.p, fh, int4=False)
+    H = hid.H[:4]
+    Cw = oracle.centroid_matrix(h2)
+    S = oracle.centroid_scores(Cw, H)
+    for B in (1, 4):
+        out_ids = torch.empty((B, cfg.p), dtype=torch.int32, device="cuda")
+        tok = dh.decode(hid_dev(H[:B]), cfg.p, out_cluster_ids=out_ids).cpu().numpy()
+        assert dh.device_status() == 0
+        ids = out_ids.cpu().numpy()
+        for r in range(B):
+            vals = np.unique(S[r])
+            assert len(vals) == 3 and np.min(np.diff(vals)) > 1e-3  # well separated: fp32 keeps the order
+            assert np.array_equal(ids[r], np.sort(oracle.select_greedy(S[r:r + 1], cfg.p)[0]))
+            rep = parity.check_greedy_token(h2, H[r], ids[r], int(tok[r]))
+            assert rep.tight_mismatch == 0
+    dh.close()
+
+
 def _decode_check_gumbel(cfg, head, hid, uni, dh, rows, B, p, T):
     rep = parity.Report()
     Cw = oracle.centroid_matrix(head)
