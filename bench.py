@@ -5,15 +5,21 @@ d = 2048, c = 8016 balanced clusters of b = 16, p = 512 probes, bf16 E and C
 -- decoding one hidden state per step (B = 1, greedy), cycling through 1024
 seeded planted/flat hidden states. A step is one ``fh_decode`` call: centroid
 scores, top-p selection, C2T gather, candidate logits and argmax, all in the
-library's fused kernel. Before every step (outside the timed events) a buffer
-twice the L2 is written and read back, so C and E come from HBM each time and
-the L2 holds only clean lines.
+library's fused kernel.
+
+Throughput (``value``): K steps issued back to back between one pair of CUDA
+events. The steps rotate over enough copies of the head (E, C, C2T) that a
+step's head was last touched at least 4 x L2 of traffic earlier, so every
+step reads its centroid and token rows from HBM (inputs larger than L2).
+Latency (``isolated_latency_us``): one step between CUDA events with a buffer
+twice the L2 written and read back before it, outside the events.
 
 Reported: head tokens/s (whole job, all ranks), us/token, the HBM roofline of
 the fused kernel (algorithmic bytes = centroid bytes + p*b*d*2 + C2T rows + h +
-output), the dense-head kernel on the same E for comparison, an end-to-end
-number through the public API from pinned host memory, SM clocks sampled
-during the timed region, and the fp64 oracle timed on the host cores.
+output), the dense-head kernel on the same E for comparison (same two
+protocols), an end-to-end number through the public API from pinned host
+memory, SM clocks sampled during the timed region, and the fp64 oracle timed
+on the host cores.
 
 ``--impl reference`` times the fp64 CPU oracle on the same workload instead.
 Under torchrun every rank runs its own replica (the head does not shard:
@@ -215,23 +221,33 @@ def run_ours(args):
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
 
+    import ctypes
     import synth
     import lm_output_head_b200 as fh
     from lm_output_head_b200 import build as fhbuild
     fhbuild.build()
 
     cfg, head, hid, _ = synth.make_config(1)
-    E = fh.bf16_from_bits(head.E, dev)
-    C = fh.bf16_from_bits(head.C, dev)
-    C2T = torch.from_numpy(head.C2T).to(dev)
-    dh = fh.FlashHead(E, C2T, C=C, max_batch=1, max_probes=cfg.p)
+    E0 = fh.bf16_from_bits(head.E, dev)
+    C0 = fh.bf16_from_bits(head.C, dev)
+    T0 = torch.from_numpy(head.C2T).to(dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    # copies of the head, used in rotation: a step's E, C and C2T were last
+    # touched n_copies - 1 steps (>= 2 x L2 of traffic) earlier, so every
+    # step reads its head from HBM although steps run back to back
+    per_step = algorithmic_bytes(cfg.v, cfg.d, cfg.c, cfg.b, cfg.p)
+    n_copies = args.copies or max(3, -(-4 * l2 // per_step) + 1)
+    heads = []
+    for i in range(n_copies):
+        E, C, T = (E0, C0, T0) if i == 0 else (E0.clone(), C0.clone(), T0.clone())
+        heads.append(fh.FlashHead(E, T, C=C, max_batch=1, max_probes=cfg.p))
+    dh = heads[0]
     assert dh.fused_b1, "fused B=1 path unavailable"
     n_states = hid.H.shape[0]
     # each rank decodes its own slice of states (replicas; independent rows)
     Hdev = fh.bf16_from_bits(rank_states(hid.H, rank), dev)
     out = torch.empty(1, dtype=torch.int32, device=dev)
 
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
     flush64 = flush.view(torch.int64)
     stream = torch.cuda.current_stream(dev)
@@ -243,51 +259,97 @@ def run_ours(args):
         flush.fill_(1)
         flush64.sum()
 
-    def step(i):
-        dh.decode(Hdev[i % n_states:i % n_states + 1], cfg.p, out_tokens=out, stream=stream)
+    # the timed loop calls the C ABI directly with prepared arguments, so the
+    # host issues steps faster than the GPU runs them
+    lib = dh._lib
+    sptr = ctypes.c_void_p(stream.cuda_stream)
+    optr = ctypes.c_void_p(out.data_ptr())
+    hptrs = [ctypes.c_void_p(Hdev[i].data_ptr()) for i in range(n_states)]
+    handles = [h._h for h in heads]
 
-    def timed_loop(fn, K, W, flush_first=True):
+    def step(i):
+        st = lib.fh_decode(handles[i % n_copies], hptrs[i % n_states], 1, cfg.p, 0, 1.0, None, None, optr,
+                           None, None, sptr)
+        if st != 0:
+            raise RuntimeError(f"fh_decode returned {st}")
+
+    def back_to_back(fn, K, W):
+        """K steps issued back to back between one pair of events (after W warm-up steps)."""
         for i in range(W):
-            if flush_first:
-                flush_l2()
             fn(i)
         torch.cuda.synchronize(dev)
         if world > 1:
             torch.distributed.barrier()
-        starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-        ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
         torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
         wall0 = time.time()
+        e0.record(stream)
         for i in range(K):
-            if flush_first:
-                flush_l2()
-            starts[i].record(stream)
             fn(W + i)
-            ends[i].record(stream)
+        e1.record(stream)
         torch.cuda.synchronize(dev)
         wall1 = time.time()
         if world > 1:
             torch.distributed.barrier()
-        ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-        return ms, wall0, wall1
+        return e0.elapsed_time(e1), wall0, wall1
+
+    def isolated(fn, K, W):
+        """Per-step events around each step, L2 flushed before every step (outside the events)."""
+        for i in range(W):
+            flush_l2()
+            fn(i)
+        torch.cuda.synchronize(dev)
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        for i in range(K):
+            flush_l2()
+            starts[i].record(stream)
+            fn(W + i)
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+        return [s.elapsed_time(e) for s, e in zip(starts, ends)]
 
     sampler = ClockSampler(dev.index)
     sampler.start()
     sampler.wait_first()
-    ms, w0, w1 = timed_loop(step, args.steps, args.warmup)
-    status = dh.device_status()
-    if status != 0:
-        raise RuntimeError(f"device status {status} after the timed loop")
-    total_ms = max_over_ranks(sum(ms), world, dev)
+    total_ms, w0, w1 = back_to_back(step, args.steps, args.warmup)
+    for h in heads:
+        status = h.device_status()
+        if status != 0:
+            raise RuntimeError(f"device status {status} after the timed loop")
+    sel_stats = [h.last_selection() for h in heads]
+    total_ms = max_over_ranks(total_ms, world, dev)
     mean_ms = total_ms / args.steps
     value = job_throughput(total_ms, args.steps, world)
 
-    # dense comparison (same protocol, fewer steps)
+    if args.only_decode:  # profiling runs: the decode loop alone
+        sampler.stop()
+        for h in heads:
+            h.close()
+        if rank == 0:
+            print(json.dumps({"only_decode": True, "us_per_token": round(mean_ms * 1e3, 3),
+                              "n_copies": n_copies}), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    # the same steps one at a time, L2 flushed before each: latency of one call
+    kl = max(3, min(args.steps, 500))
+    ms_iso = isolated(step, kl, 3)
+
+    # dense comparison, both protocols
     kd = max(3, min(args.steps, 200))
     dense_out = torch.empty(1, dtype=torch.int32, device=dev)
-    ms_d, _, _ = timed_loop(lambda i: dh.dense_head(Hdev[i % n_states:i % n_states + 1], out_argmax=dense_out,
-                                                    stream=stream), kd, 3)
-    dense_ms = statistics.mean(ms_d)
+    dptr = ctypes.c_void_p(dense_out.data_ptr())
+
+    def dense_step(i):
+        st = lib.fh_dense_head(handles[i % n_copies], hptrs[i % n_states], 1, None, dptr, sptr)
+        if st != 0:
+            raise RuntimeError(f"fh_dense_head returned {st}")
+    dense_total, _, _ = back_to_back(dense_step, kd, 3)
+    dense_ms = dense_total / kd
+    dense_iso = isolated(dense_step, kd, 3)
 
     # end to end from pinned host memory through the public API
     host = torch.from_numpy(hid.H.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -306,6 +368,8 @@ def run_ours(args):
             e2e_ms.append(s0.elapsed_time(s1))
     sampler.stop()
     clocks = sampler.summary(w0, w1)
+    for h in heads:
+        h.close()
 
     if world > 1:
         torch.distributed.barrier()
@@ -315,9 +379,10 @@ def run_ours(args):
         return
 
     peak, peak_kind = load_peaks()
-    abytes = algorithmic_bytes(cfg.v, cfg.d, cfg.c, cfg.b, cfg.p)
+    abytes = per_step
     achieved = abytes / (mean_ms * 1e-3) / 1e9
     dense_bytes = cfg.v * cfg.d * 2 + cfg.d * 2 + 4
+    iso_mean = statistics.mean(ms_iso)
     rec = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -333,19 +398,29 @@ def run_ours(args):
         "data": "synthetic (seeded planted-cluster head; 75% planted / 25% flat hidden states)",
         "config": {"workload": WORKLOAD, "global_batch": world, "per_gpu_batch": 1,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "flushed before every step: 2 x L2 buffer written then read, outside the timed events",
+                   "l2": f"inputs larger than L2: steps rotate over {n_copies} copies of the head "
+                         f"({n_copies} x {(cfg.v * cfg.d * 2 + cfg.c * cfg.d * 2 + cfg.v * 4) / 1e6:.0f} MB), "
+                         "so each step reads its head from HBM; steps issued back to back",
                    "states": n_states},
         "us_per_token": round(mean_ms * 1e3, 3),
-        "latency_us": {"p50": round(statistics.median(ms) * 1e3, 3),
-                       "p90": round(float(np.percentile(ms, 90)) * 1e3, 3)},
+        "isolated_latency_us": {"mean": round(iso_mean * 1e3, 3),
+                                "p50": round(statistics.median(ms_iso) * 1e3, 3),
+                                "p90": round(float(np.percentile(ms_iso, 90)) * 1e3, 3),
+                                "protocol": "one call between CUDA events, 2 x L2 written and read back before "
+                                            "each call outside the events (includes launch latency)"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                      "frac_of_8TBps": round(achieved / 8000.0, 4),
                      "algorithmic_bytes": abytes, "kernel": "decode_b1_kernel<8,false>",
                      "traffic": measured_traffic("decode_b1_llama1b")},
+        "selection": {"candidate_list_mean": round(statistics.mean(n for n, _ in sel_stats), 1),
+                      "from_all_keys": sum(1 for _, f in sel_stats if f),
+                      "note": "last call of each head copy: length of the short candidate list the "
+                              "selection read, and how many fell back to all c keys"},
         "dense": {"us_per_token": round(dense_ms * 1e3, 3), "tokens_per_s": round(1e3 / dense_ms, 1),
                   "achieved_GBps": round(dense_bytes / (dense_ms * 1e-3) / 1e9, 1),
                   "frac": round(dense_bytes / (dense_ms * 1e-3) / 1e9 / peak, 4),
+                  "isolated_us": round(statistics.mean(dense_iso) * 1e3, 3),
                   "speedup_flashhead_vs_dense": round(dense_ms / mean_ms, 3)},
         "e2e": {"value": round(1e3 / statistics.mean(e2e_ms), 1), "unit": "tokens/s",
                 "us_per_token": round(statistics.mean(e2e_ms) * 1e3, 3),
@@ -403,6 +478,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--copies", type=int, default=0,
+                    help="head copies the steps rotate over (default: enough to exceed 4 x L2)")
+    ap.add_argument("--only-decode", action="store_true",
+                    help="time the decode loop only (for profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

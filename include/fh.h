@@ -232,13 +232,19 @@ fh_status fh_set_spin_budget(fh_head* head, int64_t cycles);
  * Introspection: FH_QUERY_WORKSPACE_BYTES, FH_QUERY_LAST_UNION (number of
  * distinct clusters gathered by the last batched fh_decode, after
  * fh_get_device_status or a stream sync), FH_QUERY_NUM_SMS,
- * FH_QUERY_FUSED_B1 (1 if B = 1 decodes run the single fused kernel).
+ * FH_QUERY_FUSED_B1 (1 if B = 1 decodes run the single fused kernel),
+ * FH_QUERY_LAST_LIST / FH_QUERY_LAST_FULL (last fused B = 1 decode: keys
+ * that fell in its histogram of the predicted boundary region, and 1 if its
+ * selection fell back to a histogram of all c keys). Queries that read device
+ * counters synchronise the device.
  */
 typedef enum {
   FH_QUERY_WORKSPACE_BYTES = 0,
   FH_QUERY_LAST_UNION = 1,
   FH_QUERY_NUM_SMS = 2,
-  FH_QUERY_FUSED_B1 = 3
+  FH_QUERY_FUSED_B1 = 3,
+  FH_QUERY_LAST_LIST = 4,
+  FH_QUERY_LAST_FULL = 5
 } fh_query_key;
 fh_status fh_query(fh_head* head, int32_t key, int64_t* value);
 

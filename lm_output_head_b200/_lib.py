@@ -29,6 +29,8 @@ FH_QUERY_WORKSPACE_BYTES = 0
 FH_QUERY_LAST_UNION = 1
 FH_QUERY_NUM_SMS = 2
 FH_QUERY_FUSED_B1 = 3
+FH_QUERY_LAST_LIST = 4
+FH_QUERY_LAST_FULL = 5
 
 # every symbol include/fh.h declares
 EXPORTED = (

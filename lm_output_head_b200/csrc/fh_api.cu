@@ -16,6 +16,7 @@ cudaError_t set_attrs_dense(int max_smem);
 int dense_max_rows();
 cudaError_t occupancy_decode_b1(int int4, int nch, size_t smem, int* blocks);
 size_t decode_b1_misc_bytes();
+size_t decode_b1_scratch_bytes(int c, int list_cap);
 cudaError_t occupancy_dense(int nch, size_t smem, int* blocks);
 
 }  // namespace fh
@@ -38,8 +39,11 @@ struct fh_head {
   int32_t* row_ok = nullptr;           // [max_batch]
   uint32_t* c2t_counts = nullptr;      // [v]
   uint32_t* b1_keys = nullptr;         // fused B = 1 state
-  float* b1_z_row = nullptr;
-  int32_t* b1_sel = nullptr;
+  float* b1_z_buf = nullptr;           // [c * b]
+  uint32_t* b1_hist = nullptr;         // [kB1Bins]
+  uint32_t* b1_list_key = nullptr;     // [b1_list_cap]
+  int32_t* b1_list_id = nullptr;       // [b1_list_cap]
+  int b1_list_cap = 0;
   int words = 0;
   int b1_grid = 0;
   int dense_grid = 0;
@@ -238,8 +242,12 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   const size_t o_cnt = take(static_cast<size_t>(D.v) * 4);
   const int words = (D.c + 31) / 32;
   const size_t o_keys1 = take(static_cast<size_t>(D.c) * 4);
-  const size_t o_zrow = take(nc * 4);
-  const size_t o_sel1 = take(static_cast<size_t>(mp) * 4);
+  const size_t o_zbuf = take(static_cast<size_t>(D.v) * 4);
+  const size_t o_hist1 = take(static_cast<size_t>(kB1Bins) * 4);
+  // candidate list of the fused decode: up to 4 p entries (the region aims at ~2 p keys)
+  const int list_cap = static_cast<int>(std::min<size_t>(4 * mp, D.c));
+  const size_t o_lkey = take(static_cast<size_t>(list_cap) * 4);
+  const size_t o_lid = take(static_cast<size_t>(list_cap) * 4);
   const size_t o_crow = D.fmt == FH_CENTROID_INT4_G32 ? take(static_cast<size_t>(D.c) * h->crow_bytes) : 0;
   h->ws_bytes = off;
 
@@ -262,8 +270,11 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   h->row_ok = reinterpret_cast<int32_t*>(h->ws + o_rok);
   h->c2t_counts = reinterpret_cast<uint32_t*>(h->ws + o_cnt);
   h->b1_keys = reinterpret_cast<uint32_t*>(h->ws + o_keys1);
-  h->b1_z_row = reinterpret_cast<float*>(h->ws + o_zrow);
-  h->b1_sel = reinterpret_cast<int32_t*>(h->ws + o_sel1);
+  h->b1_z_buf = reinterpret_cast<float*>(h->ws + o_zbuf);
+  h->b1_hist = reinterpret_cast<uint32_t*>(h->ws + o_hist1);
+  h->b1_list_key = reinterpret_cast<uint32_t*>(h->ws + o_lkey);
+  h->b1_list_id = reinterpret_cast<int32_t*>(h->ws + o_lid);
+  h->b1_list_cap = list_cap;
   h->words = words;
   h->crows = D.fmt == FH_CENTROID_INT4_G32 ? h->ws + o_crow : static_cast<const uint8_t*>(D.C);
 
@@ -317,8 +328,8 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
     h->b1_off_slots = static_cast<int>(o);
     h->b1_slot_bytes = static_cast<int>(up(std::max(static_cast<size_t>(h->crow_bytes), static_cast<size_t>(D.d) * 2), 128));
     // the slots double as the selector's scratch once phase 1 is done
-    o += std::max(std::max(static_cast<size_t>(kWarps) * h->b1_slot_bytes, hist_select_smem_bytes(D.c)),
-                  up(sizeof(RegSelSmem), 128));
+    // the slots double as the selection's scratch between the phases
+    o += std::max(static_cast<size_t>(kWarps) * h->b1_slot_bytes, decode_b1_scratch_bytes(D.c, h->b1_list_cap));
     h->b1_smem = o;
     int blocks = 0;
     e = occupancy_decode_b1(D.fmt == FH_CENTROID_INT4_G32, h->nch, h->b1_smem, &blocks);
@@ -358,6 +369,15 @@ fh_status fh_query(fh_head* h, int32_t key, int64_t* value) {
     case FH_QUERY_LAST_UNION: {
       uint32_t u = 0;
       cudaError_t e = cudaMemcpy(&u, &h->sync->union_count, 4, cudaMemcpyDeviceToHost);
+      if (e != cudaSuccess) return cuda_fail(e);
+      *value = u;
+      return FH_OK;
+    }
+    case FH_QUERY_LAST_LIST:
+    case FH_QUERY_LAST_FULL: {
+      uint32_t u = 0;
+      const uint32_t* src = key == FH_QUERY_LAST_LIST ? &h->sync->last_in_range : &h->sync->last_full;
+      cudaError_t e = cudaMemcpy(&u, src, 4, cudaMemcpyDeviceToHost);
       if (e != cudaSuccess) return cuda_fail(e);
       *value = u;
       return FH_OK;
@@ -464,8 +484,11 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
     P.out_cluster_ids = out_cluster_ids;
     P.out_max_logit = out_max_logit;
     P.keys = h->b1_keys;
-    P.z_row = h->b1_z_row;
-    P.sel_list = h->b1_sel;
+    P.z_buf = h->b1_z_buf;
+    P.hist = h->b1_hist;
+    P.list_key = h->b1_list_key;
+    P.list_id = h->b1_list_id;
+    P.list_cap = h->b1_list_cap;
     P.best = h->best;
     P.sync = h->sync;
     P.v = D.v;

@@ -11,27 +11,36 @@
 //     owns c/G clusters. A warp's first row streams into registers, its
 //     second into a shared-memory slot by one bulk copy, both requested at
 //     kernel start. The key -- the score, or when sampling the Gumbel key
-//     s/T - ln(-ln u) (section 1.2.3) -- goes to global memory.
-//  2. the last CTA to finish phase 1 (one atomic ticket) becomes the
-//     selector: it reads the c keys once, selects the p largest exactly
-//     (key desc, id asc; histogram + exact rank of the boundary bin in shared
-//     memory), publishes the chosen ids in ascending order and raises a
-//     ready flag. Candidate row r is then slot r % b of the (r / b)-th chosen
-//     cluster: the canonical candidate order (section 1.2.1).
-//  3. one thread per CTA polls the flag with backoff; candidate row r belongs
-//     to CTA r mod G, warp (r / G) mod 16, which maps it through C2T (rows
-//     prefetched to L2 in phase 1), streams it (first row in registers,
-//     second into its slot) and keeps a packed (logit, token) maximum
-//     (section 1.2.4, stage 2).
+//     s/T - ln(-ln u) (section 1.2.3) -- goes to global memory. A key that
+//     falls in the region where the p-th key is expected (predicted from the
+//     previous call: from its rank-2p key up to its rank-p key plus twice
+//     their distance, relative to |h| when greedy) also counts in a global
+//     histogram of that region (kB1Bins equal bins; keys above it count in the
+//     top bin) and is appended, (key, id), to a short candidate list (one
+//     reservation per CTA).
+//  2. one grid-wide arrival count (release / acquire); then every CTA
+//     selects the same boundary redundantly from the histogram and the list:
+//     the bin holding the p-th largest key, and an exact rank (key desc, id
+//     asc) of that bin's few entries. Cluster k is chosen iff its (key, id)
+//     reaches the boundary entry, so the chosen set is the list entries that
+//     reach it -- no CTA waits for a published selection. If the region holds
+//     fewer than p keys or the boundary bin is crowded (the first call, a poor
+//     prediction, heavy ties), the CTA runs the general exact selector over
+//     all c keys instead.
+//  3. the chosen clusters in a fixed order (list order, or ascending ids after
+//     the general selector) give the candidate rows: row r is slot r % b of
+//     the (r / b)-th chosen cluster and belongs to CTA r mod G, warp
+//     (r / G) mod 16; it is read through C2T and dotted with h (section 1.2.4,
+//     stage 2), keeping a packed (logit, token) maximum.
 //  4. CTA maxima meet in one 64-bit atomicMax; the last CTA to finish (exit
 //     ticket) writes the token: the argmax, or, when sampling, the inverse-CDF
-//     draw over softmax(z/T) walking the candidates in canonical order.
+//     draw over softmax(z/T) in canonical order (cluster asc, slot asc)
+//     through the per-slot logit buffer. It also stores this call's rank-p
+//     and rank-2p keys for the next call and clears the histogram.
 //
-// Device-wide coordination is two atomic tickets and one flag; no
-// device-wide barrier, no histogram atomics on hot lines, and no CTA but the
-// selector reads all c keys. HBM traffic is the algorithmic
-// minimum: each centroid row once, each selected token row once, plus C2T
-// rows and h.
+// The result does not depend on the prediction: it only decides whether the
+// short list or the general selector finds the boundary.
+#include <algorithm>
 #include <climits>
 
 #include "fh_device.cuh"
@@ -39,14 +48,57 @@
 namespace fh {
 namespace {
 
+#ifdef FH_TIMELINE
+// Development aid (off in the library build): globaltimer stamps per CTA.
+__device__ unsigned long long g_tl[1024 * 16 + 8];
+__device__ __forceinline__ void tl_mark(int i) {
+  if (threadIdx.x == 0) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    g_tl[blockIdx.x * 16 + i] = t;
+  }
+}
+#define FH_TL(i) tl_mark(i)
+#define FH_TLV(i, v) (g_tl[blockIdx.x * 16 + (i)] = (v))
+#else
+#define FH_TL(i)
+#define FH_TLV(i, v)
+#endif
+
+static_assert(kB1Bins == 4 * kThreads, "each thread scans four histogram bins");
+
+constexpr int kNoteMax = kThreads;  // list entries one CTA stages (it owns at most 16 * 32 clusters)
+
 struct B1Misc {
   unsigned long long hbar;
   unsigned long long wbar[kWarps];
   unsigned long long wbest[kWarps];
   float scan[kWarps + 1];
   uint32_t uscan[kWarps + 1];
-  int claim, lastpos, last, selector;
+  int claim, lastpos, last, full;
+  uint32_t t1, above, m1, t2, total;
+  uint32_t bkey;
+  int32_t bid;
+  float edge_2p;
+  uint32_t nnote, base, nlist;
+  int32_t note_k[kNoteMax];
+  uint32_t note_key[kNoteMax];
 };
+
+__device__ __forceinline__ bool chosen(uint32_t key, int32_t id, uint32_t bkey, int32_t bid) {
+  return key > bkey || (key == bkey && id <= bid);
+}
+
+__device__ __forceinline__ size_t up128(size_t x) { return (x + 127) & ~size_t(127); }
+
+// Histogram bin of a key in the predicted region [L, L + kB1Bins / S): -1
+// below it, the top bin above it. Every CTA evaluates it with the same L, S
+// and the same rounding, so all agree on every key's bin.
+__device__ __forceinline__ int region_bin(float key, float L, float S) {
+  if (!(key >= L)) return -1;
+  const float x = __fmul_rn(__fsub_rn(key, L), S);
+  return x >= static_cast<float>(kB1Bins - 1) ? kB1Bins - 1 : static_cast<int>(x);
+}
 
 template <int NCH, bool INT4>
 __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P) {
@@ -57,11 +109,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   const bool gumbel = P.mode == 1;
 
   float* hs = reinterpret_cast<float*>(smem + P.off_h);
-  int32_t* ssel = reinterpret_cast<int32_t*>(smem + P.off_sel);
+  int32_t* ssel = reinterpret_cast<int32_t*>(smem + P.off_sel);  // the chosen clusters, ascending
   B1Misc* misc = reinterpret_cast<B1Misc*>(smem + P.off_misc);
-  uint8_t* slots = smem + P.off_slots;  // per-warp row slots; the selector's scratch after phase 1
+  uint8_t* slots = smem + P.off_slots;  // per-warp row slots; the selection's scratch between phases
 
   const uint32_t epoch = P.sync->epoch;  // calls on one head are stream-ordered
+  FH_TL(0);
 
   // ---------------- phase 1: centroid scores ----------------
   const uint32_t hbar = smem_addr(&misc->hbar);
@@ -73,6 +126,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     fence_mbar_init();
     mbar_expect_tx(hbar, static_cast<uint32_t>(d * 2));
     bulk_g2s(smem_addr(hraw), P.hidden, static_cast<uint32_t>(d * 2), hbar);
+    misc->nnote = 0u;
   }
   const int cw = static_cast<int>(blockIdx.x) + G * warp;  // first cluster of this warp
   const int cstride = G * kWarps;
@@ -97,23 +151,50 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   }
   float ureg = 0.f;  // lane j holds u of item j
   if (gumbel && lane < n1) ureg = __ldg(P.u_clusters + cw + lane * cstride);
-  if (lane < n1) prefetch_l2(P.C2T + static_cast<size_t>(cw + lane * cstride) * b);  // read in phase 3 if chosen
+  const int mi = gumbel ? 1 : 0;
+  const uint32_t prior_ok = P.sync->prior_ok[mi];
+  const float prior_p = P.sync->prior_p[mi];
+  const float prior_2p = P.sync->prior_2p[mi];
   __syncthreads();  // hbar initialised before anyone waits on it
   if (!mbar_wait_bounded(hbar, 0u, kWaitBudget) && lane == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
+  float hnorm;
   {
     // widen h in place (d <= 4 * kThreads: one round, every chunk read before any is written)
     float hv[8];
+    float ss = 0.f;
     if (tid < d / 8) {
       const uint4 x = *reinterpret_cast<const uint4*>(hraw + 8 * tid);
       hv[0] = bf16lo(x.x); hv[1] = bf16hi(x.x); hv[2] = bf16lo(x.y); hv[3] = bf16hi(x.y);
       hv[4] = bf16lo(x.z); hv[5] = bf16hi(x.z); hv[6] = bf16lo(x.w); hv[7] = bf16hi(x.w);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ss = fmaf(hv[i], hv[i], ss);
     }
+    ss = warp_sum(ss);
+    if (lane == 0) misc->scan[warp] = ss;
     __syncthreads();
     if (tid < d / 8) {
       reinterpret_cast<float4*>(hs)[2 * tid] = make_float4(hv[0], hv[1], hv[2], hv[3]);
       reinterpret_cast<float4*>(hs)[2 * tid + 1] = make_float4(hv[4], hv[5], hv[6], hv[7]);
     }
+    float tot = 0.f;
+#pragma unroll
+    for (int i = 0; i < kWarps; ++i) tot += misc->scan[i];
+    hnorm = sqrtf(tot);
     __syncthreads();
+  }
+  FH_TL(1);
+  // the predicted region [L, U): from the last call's rank-2p key up to its
+  // rank-p key plus twice their distance (identical arithmetic in every CTA)
+  const float unit = gumbel ? 1.f : hnorm;
+  float L = 0.f, S = 0.f;
+  bool region = prior_ok != 0u && unit > 0.f;
+  if (region) {
+    const float kp = prior_p * unit, k2 = prior_2p * unit;
+    float span = 3.f * (kp - k2);
+    if (!(span > 0.f)) span = fmaxf(fabsf(kp), 1e-30f) * 0.25f;
+    L = k2;
+    S = static_cast<float>(kB1Bins) / span;
+    region = fabsf(L) < 3.0e38f && S > 0.f && S < 3.0e38f;
   }
   for (int i = 0; i < n1; ++i) {
     const int k = cw + i * cstride;
@@ -132,79 +213,239 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     }
     const float u = __shfl_sync(0xFFFFFFFFu, ureg, i & 31);
     const float key = gumbel ? gumbel_key(s, P.T, u) : s;
-    if (lane == 0) P.keys[k] = f2key(key);
-  }
-
-  // ---------------- phase 2: the last CTA to finish selects ----------------
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    misc->selector = atomicAdd(&P.sync->arrive, 1u) == static_cast<uint32_t>(G - 1);
-  }
-  __syncthreads();
-  const int r_all = P.p * b;
-  if (misc->selector) {
-    __threadfence();
-    if (P.c <= kThreads * 16) {
-      select_reg<16>(P.keys, P.c, P.p, P.off_sel, P.off_slots);
-    } else if (P.c <= kThreads * 32) {
-      select_reg<32>(P.keys, P.c, P.p, P.off_sel, P.off_slots);
-    } else {
-      select_stage_gkeys(P.keys, P.c, slots);
-      select_top_p_staged(P.c, P.p, P.off_sel, P.off_slots);
-    }
-    for (int i = tid; i < P.p; i += kThreads) {
-      P.sel_list[i] = ssel[i];
-      if (P.out_cluster_ids) P.out_cluster_ids[i] = ssel[i];
-    }
-    __syncthreads();
-    if (tid == 0) {
-      __threadfence();
-      st_release_u32(&P.sync->ready, epoch + 1u);  // the selection of this call is published
-    }
-    fence_proxy_async_smem();  // the slots were generic scratch; bulk copies follow
-  } else {
-    // one thread per CTA waits (bounded, with backoff) for the selector's flag
-    if (tid == 0) {
-      int okw = 1;
-      const long long t0 = clock64();
-      while (ld_acquire_u32(&P.sync->ready) != epoch + 1u) {
-        __nanosleep(200);
-        if (clock64() - t0 > P.spin_budget) {
-          okw = 0;
-          break;
+    if (lane == 0) {
+      const uint32_t kk = f2key(key);
+      P.keys[k] = kk;
+      const int bn = region ? region_bin(key, L, S) : -1;
+      if (bn >= 0) {
+        red_relaxed_add_u32(P.hist + bn, 1u);
+        const uint32_t at = atomicAdd(&misc->nnote, 1u);
+        if (at < static_cast<uint32_t>(kNoteMax)) {
+          misc->note_k[at] = k;
+          misc->note_key[at] = kk;
         }
       }
-      misc->claim = okw;
     }
   }
   __syncthreads();
-  const bool sel_ok = misc->selector || misc->claim;
+  FH_TL(2);
+  // append this CTA's region keys to the candidate list
+  const int nnote = min(static_cast<int>(misc->nnote), kNoteMax);
+  if (tid == 0) misc->base = nnote ? atomicAdd(&P.sync->list_count, static_cast<uint32_t>(nnote)) : 0u;
+  __syncthreads();
+  for (int i = tid; i < nnote; i += kThreads) {
+    const uint32_t at = misc->base + static_cast<uint32_t>(i);
+    if (at < static_cast<uint32_t>(P.list_cap)) {
+      P.list_key[at] = misc->note_key[i];
+      P.list_id[at] = misc->note_k[i];
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    red_release_add_u32(&P.sync->arrive, 1u);  // keys, counts and list entries of this CTA are published
+    // wait (bounded, with backoff) until every CTA has arrived
+    int okw = 1;
+    const long long t0 = clock64();
+    while (ld_acquire_u32(&P.sync->arrive) < static_cast<uint32_t>(G)) {
+      __nanosleep(32);
+      if (clock64() - t0 > P.spin_budget) {
+        okw = 0;
+        break;
+      }
+    }
+    misc->claim = okw;
+    misc->nlist = __ldcg(&P.sync->list_count);
+  }
+  __syncthreads();
+  FH_TL(3);
+  bool ok = misc->claim != 0;
+
+  // ---------------- phase 2: the boundary of the top p ----------------
+  // scratch (the slot area): the list's keys and ids, or all c keys; then the selection state
+  const int p = P.p, c = P.c;
+  const int r_2p = min(c, 2 * p);
+  const uint32_t nlist = misc->nlist;
+  const bool use_list = region && nlist >= static_cast<uint32_t>(p) && nlist <= static_cast<uint32_t>(P.list_cap);
+  const int nl = use_list ? static_cast<int>(nlist) : 0;
+  uint32_t* skey = reinterpret_cast<uint32_t*>(slots);
+  int32_t* sid = reinterpret_cast<int32_t*>(slots + up128(static_cast<size_t>(P.list_cap) * 4));
+  const uint32_t bs_off =
+      static_cast<uint32_t>(P.off_slots) +
+      static_cast<uint32_t>(std::max(2 * up128(static_cast<size_t>(P.list_cap) * 4), up128(static_cast<size_t>(c) * 4)));
+  BoundSmem& bs = *reinterpret_cast<BoundSmem*>(smem + bs_off);
+  bool full = true;
+  if (tid == 0) {
+    misc->total = nlist;
+    misc->t2 = 0xFFFFFFFFu;
+  }
+  if (ok) {
+    if (use_list) {
+      const uint4 hq = __ldcg(reinterpret_cast<const uint4*>(P.hist) + (kB1Bins / 4 - 1 - tid));
+      for (int i = tid; i < nl; i += kThreads) {
+        skey[i] = __ldcg(P.list_key + i);
+        sid[i] = __ldcg(P.list_id + i);
+      }
+      FH_TL(8);
+      // bins from the top: thread t owns kB1Bins-1-4t (first) .. kB1Bins-4-4t
+      const uint32_t hv[4] = {hq.w, hq.z, hq.y, hq.x};
+      uint32_t total;
+      uint32_t run = block_scan_excl_u32(hv[0] + hv[1] + hv[2] + hv[3], misc->uscan, &total);
+      if (tid == 0) {
+        misc->total = total;
+        misc->m1 = 0xFFFFFFFFu;
+        misc->t2 = 0xFFFFFFFFu;
+        bs.nc = 0u;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t bin = static_cast<uint32_t>(kB1Bins - 1 - 4 * tid - j);
+        if (run < static_cast<uint32_t>(p) && run + hv[j] >= static_cast<uint32_t>(p)) {
+          misc->t1 = bin;
+          misc->above = run;
+          misc->m1 = hv[j];
+        }
+        if (run < static_cast<uint32_t>(r_2p) && run + hv[j] >= static_cast<uint32_t>(r_2p)) misc->t2 = bin;
+        run += hv[j];
+      }
+      __syncthreads();
+      FH_TL(9);
+      // the list holds every key the histogram counted; a crowded boundary bin takes the general path
+      full = misc->m1 > static_cast<uint32_t>(kBoundEntries) || misc->total != nlist;
+      if (!full) {
+        // gather the boundary bin's entries (their bins agree with phase 1), rank them exactly
+        const int t1 = static_cast<int>(misc->t1);
+        for (int i = tid; i < nl; i += kThreads) {
+          const uint32_t kk = skey[i];
+          if (region_bin(key2f(kk), L, S) == t1) {
+            const uint32_t at = atomicAdd(&bs.nc, 1u);
+            if (at < static_cast<uint32_t>(kBoundEntries)) {
+              bs.ckey[at] = kk;
+              bs.cid[at] = sid[i];
+            }
+          }
+        }
+        __syncthreads();
+        FH_TL(10);
+        const uint32_t m1 = min(bs.nc, static_cast<uint32_t>(kBoundEntries));  // == misc->m1
+        const uint32_t need = static_cast<uint32_t>(p) - misc->above;
+        for (uint32_t a = tid; a < m1; a += kThreads) {
+          const uint32_t ka = bs.ckey[a];
+          const int32_t ia = bs.cid[a];
+          uint32_t r = 0;
+          for (uint32_t bb = 0; bb < m1; ++bb) {
+            const uint32_t kb = bs.ckey[bb];
+            r += (kb > ka || (kb == ka && bs.cid[bb] < ia)) ? 1u : 0u;
+          }
+          if (r + 1u == need) {
+            misc->bkey = ka;
+            misc->bid = ia;
+          }
+        }
+        if (tid == 0) {
+          misc->edge_2p = misc->t2 != 0xFFFFFFFFu ? L + static_cast<float>(misc->t2) / S
+                                                  : __int_as_float(0x7FC00000);
+          if (m1 != misc->m1) misc->m1 = 0xFFFFFFFFu;  // inconsistent counts: take the general path
+        }
+        __syncthreads();
+        FH_TL(11);
+        full = misc->m1 == 0xFFFFFFFFu;
+      }
+    }
+    if (full) {
+      // the general exact selector over all c keys
+      for (int i = tid; i < c / 4; i += kThreads)
+        reinterpret_cast<uint4*>(skey)[i] = __ldcg(reinterpret_cast<const uint4*>(P.keys) + i);
+      for (int i = (c / 4) * 4 + tid; i < c; i += kThreads) skey[i] = __ldcg(P.keys + i);
+      __syncthreads();
+      select_boundary(c, p, p, r_2p, static_cast<uint32_t>(P.off_slots), kImplicitIds, bs_off);
+      if (bs.heavy) {
+        // heavy ties: radix select (ties to the lower id) into ssel, then its worst entry
+        __syncthreads();
+        SelectSmem& rs = *reinterpret_cast<SelectSmem*>(smem + bs_off);
+        block_select_top_p(skey, c, p, ssel, rs);
+        unsigned long long worst = ~0ull;
+        for (int i = tid; i < p; i += kThreads) {
+          const int k = ssel[i];
+          const unsigned long long cmp = (static_cast<unsigned long long>(skey[k]) << 32) |
+                                         static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(k));
+          worst = cmp < worst ? cmp : worst;
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+          const unsigned long long y = __shfl_xor_sync(0xFFFFFFFFu, worst, o);
+          worst = y < worst ? y : worst;
+        }
+        if (lane == 0) misc->wbest[warp] = worst;
+        __syncthreads();
+        if (tid == 0) {
+          unsigned long long m = ~0ull;
+          for (int i = 0; i < kWarps; ++i) m = misc->wbest[i] < m ? misc->wbest[i] : m;
+          misc->bkey = static_cast<uint32_t>(m >> 32);
+          misc->bid = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(m & 0xFFFFFFFFull));
+          misc->edge_2p = __int_as_float(0x7FC00000);
+        }
+      } else if (tid == 0) {
+        misc->bkey = bs.bkey;
+        misc->bid = bs.bid;
+        misc->edge_2p = bs.edge_b;
+      }
+      __syncthreads();
+    }
+    if (tid == 0) misc->full = full;
+    // the chosen clusters in row order (list order, or ascending ids): warp w
+    // owns entries [w * span, w * span + span), 32 consecutive per step (one per
+    // lane: no bank conflicts), one ballot each
+    const uint32_t bkey = misc->bkey;
+    const int32_t bid = misc->bid;
+    const int n = full ? c : nl;
+    const int wspan = ((n + kWarps - 1) / kWarps + 31) & ~31;
+    const int w0 = min(n, warp * wspan), w1 = min(n, w0 + wspan);
+    uint32_t cnt = 0;
+    for (int base = w0; base < w1; base += 32) {
+      const int i = base + lane;
+      const bool ch = i < w1 && chosen(skey[i], full ? i : sid[i], bkey, bid);
+      cnt += __popc(__ballot_sync(0xFFFFFFFFu, ch));
+    }
+    if (lane == 0) misc->uscan[warp] = cnt;
+    __syncthreads();
+    uint32_t pos = 0;
+    for (int i = 0; i < warp; ++i) pos += misc->uscan[i];
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int base = w0; base < w1; base += 32) {
+      const int i = base + lane;
+      const int32_t k = i < w1 ? (full ? i : sid[i]) : 0;
+      const bool ch = i < w1 && chosen(skey[i], k, bkey, bid);
+      const uint32_t m = __ballot_sync(0xFFFFFFFFu, ch);
+      const uint32_t at = pos + __popc(m & lt);
+      if (ch && at < static_cast<uint32_t>(p)) ssel[at] = k;
+      pos += __popc(m);
+    }
+    fence_proxy_async_smem();  // the slots were generic scratch; bulk copies follow
+    __syncthreads();
+  }
+  FH_TL(4);
 
   // ---------------- phase 3: candidate rows ----------------
-  // rows r0 = blockIdx + G * warp, r0 + 16 G, ...: two at a time are polled
-  // together and streamed together (registers, slot).
+  // row r is slot r % b of the (r / b)-th chosen cluster; rows
+  // blockIdx + G * warp + 16 G i belong to this warp, two at a time
   unsigned long long best = 0ull;
-  bool ok = true;
-  if (!sel_ok) ok = false;
-  for (int r0 = cw; sel_ok && r0 < r_all; r0 += 2 * cstride) {
+  const int r_all = p * b;
+  for (int r0 = cw; ok && r0 < r_all; r0 += 2 * cstride) {
     const int r1 = r0 + cstride;
     const bool two = r1 < r_all;
-    // candidate row r is slot r % b of the (r / b)-th chosen cluster (canonical order)
     int t = 0;
     if (lane == 0 || (lane == 1 && two)) {
       const int r = lane == 0 ? r0 : r1;
-      const int k = __ldcg(P.sel_list + r / b);
-      t = (k >= 0 && k < P.c) ? __ldg(P.C2T + static_cast<size_t>(k) * b + r % b) : -1;
+      const int k = ssel[r / b];
+      t = (k >= 0 && k < c) ? __ldg(P.C2T + static_cast<size_t>(k) * b + r % b) : -1;
     }
     const int t0 = __shfl_sync(0xFFFFFFFFu, t, 0);
     const int t1 = two ? __shfl_sync(0xFFFFFFFFu, t, 1) : 0;
-    if (t0 < 0 || t1 < 0) {  // only an inconsistent selection; never read outside E
+    if (t0 < 0 || t1 < 0 || t0 >= P.v || t1 >= P.v) {  // only an inconsistent selection; never read outside E
       ok = false;
       break;
     }
     if (two && lane == 0) {
-      fence_proxy_async_smem();
       mbar_expect_tx(wbar, static_cast<uint32_t>(d * 2));
       bulk_g2s(slot, P.E + static_cast<size_t>(t1) * d, static_cast<uint32_t>(d * 2), wbar);
     }
@@ -213,51 +454,77 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     const float z0 = row_dot_bf16_hs<NCH>(e, hs, d);
     unsigned long long pk = pack_best(z0, t0);
     best = pk > best ? pk : best;
-    if (gumbel && lane == 0) P.z_row[r0] = z0;
+    if (gumbel && lane == 0) P.z_buf[static_cast<size_t>(ssel[r0 / b]) * b + r0 % b] = z0;
     if (two) {
-      if (!mbar_wait_bounded(wbar, wphase, kWaitBudget)) ok = false;
+      const bool got = mbar_wait_bounded(wbar, wphase, kWaitBudget);
       wphase ^= 1u;
+      if (!__all_sync(0xFFFFFFFFu, got)) {
+        mbar_wait_bounded(wbar, wphase ^ 1u, kWaitBudget);  // drain before the slot is released
+        ok = false;
+        break;
+      }
       const float z1 = srow_dot_bf16_hs<NCH>(slot, hs, d);
       pk = pack_best(z1, t1);
       best = pk > best ? pk : best;
-      if (gumbel && lane == 0) P.z_row[r1] = z1;
+      if (gumbel && lane == 0) P.z_buf[static_cast<size_t>(ssel[r1 / b]) * b + r1 % b] = z1;
       __syncwarp();
+      if (lane == 0) fence_proxy_async_smem();
     }
   }
   if (!ok && lane == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
   best = warp_max_u64(best);
   if (lane == 0) misc->wbest[warp] = best;
   __syncthreads();
+  FH_TL(5);
+
+  // ---------------- exit: the last CTA writes the token ----------------
   if (tid == 0) {
     unsigned long long m = 0ull;
     for (int i = 0; i < kWarps; ++i) m = misc->wbest[i] > m ? misc->wbest[i] : m;
     if (m) atomicMax(P.best, m);
-  }
-
-  // ---------------- exit: the last CTA writes the token ----------------
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    const uint32_t tk = atomicAdd(&P.sync->ticket, 1u);
-    misc->last = (tk == static_cast<uint32_t>(G - 1));
+    // acq_rel: this CTA's maximum and logits are published; the last CTA sees everyone's
+    misc->last = atom_acq_rel_add_u32(&P.sync->ticket, 1u) == static_cast<uint32_t>(G - 1);
   }
   __syncthreads();
+  FH_TL(6);
   if (!misc->last) return;
-  __threadfence();
 
-  const unsigned long long bw = *reinterpret_cast<volatile unsigned long long*>(P.best);
-  if (!gumbel) {
-    if (tid == 0) {
-      P.out_tokens[0] = best_token(bw);
-      if (P.out_max_logit) P.out_max_logit[0] = best_logit(bw);
-    }
-  } else {
+  const unsigned long long bw = __ldcg(P.best);
+  if (tid == 0) {
+    if (!gumbel) P.out_tokens[0] = best_token(bw);
+    if (P.out_max_logit) P.out_max_logit[0] = best_logit(bw);
+  }
+  if (ok && (gumbel || P.out_cluster_ids) && !misc->full) {
+    // list order -> ascending ids (canonical order): membership bitmap over the c ids, then a scan
+    const int words = (c + 31) >> 5;
+    uint32_t* bits = reinterpret_cast<uint32_t*>(slots);
+    for (int i = tid; i < words; i += kThreads) bits[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < p; i += kThreads) atomicOr(&bits[ssel[i] >> 5], 1u << (ssel[i] & 31));
+    __syncthreads();
+    const int wpt = (words + kThreads - 1) / kThreads;
+    const int v0 = min(words, tid * wpt), v1 = min(words, v0 + wpt);
+    uint32_t cnt = 0;
+    for (int wi = v0; wi < v1; ++wi) cnt += __popc(bits[wi]);
+    uint32_t pos = block_scan_excl_u32(cnt, misc->uscan, nullptr);
+    __syncthreads();  // every ssel entry is in the bitmap before any is overwritten
+    for (int wi = v0; wi < v1; ++wi)
+      for (uint32_t m = bits[wi]; m; m &= m - 1u) {
+        if (pos < static_cast<uint32_t>(p)) ssel[pos] = wi * 32 + __ffs(m) - 1;
+        ++pos;
+      }
+    __syncthreads();
+  }
+  if (ok && P.out_cluster_ids)
+    for (int i = tid; i < p; i += kThreads) P.out_cluster_ids[i] = ssel[i];
+  if (ok && gumbel) {
     // inverse CDF over softmax(z/T) in canonical order (cluster asc, slot asc)
+    auto zc = [&](int i) -> float { return __ldcg(P.z_buf + static_cast<size_t>(ssel[i / b]) * b + i % b); };
     const float ym = best_logit(bw) / P.T;
     const int qn = (r_all + kThreads - 1) / kThreads;
     const int i0 = min(r_all, tid * qn), i1 = min(r_all, i0 + qn);
     float loc = 0.f;
-    for (int i = i0; i < i1; ++i) loc += expf(__ldcg(P.z_row + i) / P.T - ym);
+    for (int i = i0; i < i1; ++i) loc += expf(zc(i) / P.T - ym);
     if (tid == 0) {
       misc->claim = INT_MAX;
       misc->lastpos = 0;
@@ -269,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     float run = before;
     int claim = INT_MAX, lastpos = -1;
     for (int i = i0; i < i1; ++i) {
-      const float wgt = expf(__ldcg(P.z_row + i) / P.T - ym);
+      const float wgt = expf(zc(i) / P.T - ym);
       if (wgt > 0.f) lastpos = i;
       run += wgt;
       if (run > target) {
@@ -282,17 +549,46 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     __syncthreads();
     if (tid == 0) {
       const int idx = misc->claim != INT_MAX ? misc->claim : misc->lastpos;
-      P.out_tokens[0] = __ldg(P.C2T + static_cast<size_t>(__ldcg(P.sel_list + idx / b)) * b + idx % b);
-      if (P.out_max_logit) P.out_max_logit[0] = best_logit(bw);
+      P.out_tokens[0] = __ldg(P.C2T + static_cast<size_t>(ssel[idx / b]) * b + idx % b);
     }
   }
+#ifdef FH_TIMELINE
   if (tid == 0) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    g_tl[1024 * 16] = t;
+    g_tl[1024 * 16 + 1] = blockIdx.x;
+    g_tl[1024 * 16 + 2] = misc->full;
+    g_tl[1024 * 16 + 3] = misc->total;
+  }
+#endif
+  // clear the histogram for the next call (every CTA has read it)
+  if (region) reinterpret_cast<uint4*>(P.hist)[tid] = make_uint4(0, 0, 0, 0);
+  if (tid == 0) {
+    // this call's keys of rank p and 2p for the next call; past the region's
+    // count the rank-2p key is extrapolated linearly from the region's edge
+    if (ok) {
+      const float kp = key2f(misc->bkey);
+      float k2 = misc->edge_2p;
+      if (!misc->full && misc->t2 == 0xFFFFFFFFu) {
+        const float tot = static_cast<float>(misc->total);
+        k2 = L - (kp - L) * (static_cast<float>(r_2p) - tot) / fmaxf(1.f, tot - static_cast<float>(p));
+      }
+      const float pp = kp / unit, p2 = fminf(k2, kp) / unit;
+      if (pp == pp && p2 == p2 && fabsf(pp) < 3.0e38f && fabsf(p2) < 3.0e38f && unit > 0.f) {
+        P.sync->prior_p[mi] = pp;
+        P.sync->prior_2p[mi] = p2;
+        P.sync->prior_ok[mi] = 1u;
+      }
+      P.sync->last_in_range = region ? misc->total : 0u;
+      P.sync->last_full = misc->full;
+    }
     *P.best = 0ull;
     P.sync->arrive = 0u;
     P.sync->ticket = 0u;
+    P.sync->list_count = 0u;
     P.sync->epoch = epoch + 1u;
   }
-  __threadfence();
 }
 
 template <int NCH>
@@ -314,6 +610,20 @@ cudaError_t launch_nch(const B1Params& P, int grid, size_t smem, int int4, cudaS
 }  // namespace
 
 size_t decode_b1_misc_bytes() { return sizeof(B1Misc); }
+
+// Scratch of the selection phase (in the slot area): the candidate list's
+// keys and ids, or all c keys, then the selection's shared state.
+size_t decode_b1_scratch_bytes(int c, int list_cap) {
+  auto r128 = [](size_t x) { return (x + 127) & ~size_t(127); };
+  const size_t keys = std::max(2 * r128(static_cast<size_t>(list_cap) * 4), r128(static_cast<size_t>(c) * 4));
+  return keys + std::max(sizeof(BoundSmem), sizeof(SelectSmem));
+}
+
+#ifdef FH_TIMELINE
+extern "C" int fh_timeline_read(unsigned long long* host, int n) {
+  return static_cast<int>(cudaMemcpyFromSymbol(host, g_tl, static_cast<size_t>(n) * 8));
+}
+#endif
 
 cudaError_t launch_decode_b1(const B1Params& P, int grid, size_t smem, int int4, int nch, cudaStream_t st) {
   switch (nch) {

@@ -100,6 +100,22 @@ __device__ __forceinline__ void st_release_u32(unsigned* p, uint32_t v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// Release add without a result (orders this thread's earlier memory operations, and
+// those made visible to it by a CTA barrier, before the add).
+__device__ __forceinline__ void red_release_add_u32(unsigned* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void red_relaxed_add_u32(unsigned* p, uint32_t v) {
+  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t atom_acq_rel_add_u32(unsigned* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 __device__ __forceinline__ uint32_t ld_relaxed_u32(const unsigned* p) {
   uint32_t v;
   asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -517,13 +533,6 @@ static __device__ __noinline__ void select_top_p_staged(int c, int p, uint32_t s
   __syncthreads();
 }
 
-// Stage keys: order-preserving u32 keys from global memory (4 in flight per thread).
-__device__ __forceinline__ void select_stage_gkeys(const uint32_t* gkeys, int c, uint8_t* scratch) {
-  uint32_t* key = select_keys_area(scratch);
-#pragma unroll 4
-  for (int k = threadIdx.x; k < c; k += kThreads) key[k] = __ldcg(gkeys + k);
-  __syncthreads();
-}
 
 // Exclusive block scan of one u32 per thread: warp scans by shuffles, one
 // barrier, then every thread adds the totals of the warps before it.
@@ -549,58 +558,48 @@ __device__ __forceinline__ uint32_t block_scan_excl_u32(uint32_t v, uint32_t* ws
   return before + x - v;
 }
 
-// Top-p for one CTA whose c keys (order-preserving u32 in global memory) fit
-// in registers, KPT per thread (c <= kThreads * KPT). Thread t owns ids
-// t*KPT .. t*KPT + KPT - 1, so each thread's keys are in id order and block
-// scans do the gather and the output. One CTA runs it alone, so it is written
-// for few instructions per key: each key's bin is computed once (in the
-// key's register), then two KPT-bit masks (above / in the boundary bin) carry
-// everything after the histogram. Steps: value range (warp reductions), a
-// value-linear 4096-bin histogram in shared memory, a two-level search for
-// the bin holding the p-th largest key, an id-ordered gather (keys reloaded
-// from global memory) and exact all-pairs rank of that bin (key desc, id
-// asc), and one scan that writes the chosen ids ascending to `sel`. More than
-// kBoundaryMax keys in that bin (heavy ties) falls back to the staged
-// selector. `sel_off` / `scratch_off` are byte offsets into the dynamic
-// shared memory; the scratch must hold hist_select_smem_bytes(c) bytes.
-struct RegSelSmem {
+// ---------------------------------------------------------------------------
+// boundary of a top-p set
+// ---------------------------------------------------------------------------
+// For n keys (order-preserving u32) in shared memory with their cluster ids
+// (a shared array, or the key's index when ids_off == kImplicitIds), finds the
+// p-th entry in the order (key desc, id asc): cluster k with key x is among
+// the p best iff x > bkey, or x == bkey and k <= bid. Also returns the lower
+// value edges of the histogram bins holding the ra-th and rb-th largest keys
+// (NaN where the rank exceeds n), used to predict the next call's
+// thresholds. Steps: value range, a value-linear 4096-bin histogram, a
+// two-level search from the top for the bins of ranks p, ra, rb, and an
+// exact rank (key desc, id asc) of the entries of the boundary bin. More than
+// kBoundEntries entries in that bin (heavy ties) sets `heavy` and returns
+// without a boundary. All kThreads threads must call it; every thread sees
+// the result in the struct after it returns.
+constexpr uint32_t kImplicitIds = 0xFFFFFFFFu;
+constexpr int kBoundEntries = 1024;
+
+struct BoundSmem {
   uint32_t hist[kHistBins];
-  uint32_t ckey[kBoundaryMax];
-  uint8_t ctake[kBoundaryMax];
-  uint32_t wmin[kWarps], wmax[kWarps], wtot[kWarps], wa[kWarps], wb[kWarps];
-  uint32_t t1, above, m1;
+  uint32_t ckey[kBoundEntries];
+  int32_t cid[kBoundEntries];
+  uint32_t wmin[kWarps], wmax[kWarps], wtot[kWarps];
+  uint32_t t[3], above, m1, nc;
+  uint32_t bkey;
+  int32_t bid;
+  float lo, scale, edge_a, edge_b;
+  int heavy;
 };
 
-template <int KPT>
-static __device__ __noinline__ void select_reg(const uint32_t* gkeys, int c, int p, uint32_t sel_off,
-                                               uint32_t scratch_off) {
-  static_assert(KPT % 4 == 0 && KPT <= 32, "vector loads of 4 keys; one 32-bit mask per thread");
-  int32_t* sel = reinterpret_cast<int32_t*>(fh_dyn_smem + sel_off);
-  RegSelSmem& sm = *reinterpret_cast<RegSelSmem*>(fh_dyn_smem + scratch_off);
+static __device__ __noinline__ void select_boundary(int n, int p, int ra, int rb, uint32_t keys_off,
+                                                    uint32_t ids_off, uint32_t sm_off) {
+  const uint32_t* key = reinterpret_cast<const uint32_t*>(fh_dyn_smem + keys_off);
+  const int32_t* ids = reinterpret_cast<const int32_t*>(fh_dyn_smem + (ids_off == kImplicitIds ? 0u : ids_off));
+  BoundSmem& sm = *reinterpret_cast<BoundSmem*>(fh_dyn_smem + sm_off);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int id0 = tid * KPT;
-  const int nv = max(0, min(KPT, c - id0));  // valid keys of this thread
-  uint32_t kb[KPT];                          // the keys, then their bins
-  if (nv == KPT && (reinterpret_cast<uintptr_t>(gkeys) & 15) == 0) {
-#pragma unroll
-    for (int j = 0; j < KPT; j += 4) {
-      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(gkeys + id0 + j));
-      kb[j] = v.x;
-      kb[j + 1] = v.y;
-      kb[j + 2] = v.z;
-      kb[j + 3] = v.w;
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < KPT; ++j) kb[j] = j < nv ? __ldcg(gkeys + id0 + j) : 0u;
-  }
+  const bool implicit = ids_off == kImplicitIds;
 
-  // value range
   uint32_t mn = 0xFFFFFFFFu, mx = 0u;
-#pragma unroll
-  for (int j = 0; j < KPT; ++j) {
-    mn = min(mn, j < nv ? kb[j] : 0xFFFFFFFFu);
-    mx = max(mx, kb[j]);  // invalid keys are 0
+  for (int i = tid; i < n; i += kThreads) {
+    mn = min(mn, key[i]);
+    mx = max(mx, key[i]);
   }
   mn = __reduce_min_sync(0xFFFFFFFFu, mn);
   mx = __reduce_max_sync(0xFFFFFFFFu, mx);
@@ -609,6 +608,7 @@ static __device__ __noinline__ void select_reg(const uint32_t* gkeys, int c, int
     sm.wmax[warp] = mx;
   }
   for (int i = tid; i < kHistBins / 4; i += kThreads) reinterpret_cast<uint4*>(sm.hist)[i] = make_uint4(0, 0, 0, 0);
+  if (tid == 0) sm.nc = 0u;
   __syncthreads();
 #pragma unroll
   for (int w = 0; w < kWarps; ++w) {
@@ -617,16 +617,8 @@ static __device__ __noinline__ void select_reg(const uint32_t* gkeys, int c, int
   }
   const float lo = key2f(mn), span = key2f(mx) - lo;
   const float scale = span > 0.f ? static_cast<float>(kHistBins) / span : 0.f;
-
-  // bins (computed once, in place) and the histogram
-#pragma unroll
-  for (int j = 0; j < KPT; ++j) {
-    kb[j] = value_bin(kb[j], lo, scale);
-    if (j < nv) atomicAdd(&sm.hist[kb[j]], 1u);
-  }
+  for (int i = tid; i < n; i += kThreads) atomicAdd(&sm.hist[value_bin(key[i], lo, scale)], 1u);
   __syncthreads();
-
-  // two-level search from the top: warp w owns bins 4095 - 256 w .. 3840 - 256 w
   {
     uint32_t s = 0;
 #pragma unroll
@@ -639,78 +631,72 @@ static __device__ __noinline__ void select_reg(const uint32_t* gkeys, int c, int
     uint32_t above_w = 0;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) above_w += w < warp ? sm.wtot[w] : 0u;
-    const uint32_t pp = static_cast<uint32_t>(p);
-    if (above_w < pp && above_w + sm.wtot[warp] >= pp) {
-      // this warp's 256 bins, descending: lane l owns 8 consecutive bins
-      uint32_t hv[8], s = 0;
+    const uint32_t rk[3] = {static_cast<uint32_t>(p), static_cast<uint32_t>(ra), static_cast<uint32_t>(rb)};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        hv[i] = sm.hist[kHistBins - 1 - 256 * warp - 8 * lane - i];
-        s += hv[i];
-      }
-      uint32_t incl = s;
+    for (int j = 0; j < 3; ++j) {
+      const uint32_t rr = rk[j];
+      if (rr >= 1u && above_w < rr && above_w + sm.wtot[warp] >= rr) {
+        uint32_t hv[8], s = 0;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      uint32_t run = above_w + incl - s;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (run < pp && run + hv[i] >= pp) {
-          sm.t1 = kHistBins - 1 - 256 * warp - 8 * lane - i;
-          sm.above = run;
-          sm.m1 = hv[i];
+        for (int i = 0; i < 8; ++i) {
+          hv[i] = sm.hist[kHistBins - 1 - 256 * warp - 8 * lane - i];
+          s += hv[i];
         }
-        run += hv[i];
+        uint32_t incl = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        uint32_t run = above_w + incl - s;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (run < rr && run + hv[i] >= rr) {
+            sm.t[j] = static_cast<uint32_t>(kHistBins - 1 - 256 * warp - 8 * lane - i);
+            if (j == 0) {
+              sm.above = run;
+              sm.m1 = hv[i];
+            }
+          }
+          run += hv[i];
+        }
       }
     }
   }
   __syncthreads();
-  const uint32_t t1 = sm.t1, m1 = sm.m1, need = static_cast<uint32_t>(p) - sm.above;
-  const bool all_in_bin = m1 == need;
-  if (!all_in_bin && m1 > static_cast<uint32_t>(kBoundaryMax)) {  // heavy ties: exact staged selector
+  const uint32_t t1 = sm.t[0], m1 = sm.m1, need = static_cast<uint32_t>(p) - sm.above;
+  if (tid == 0) {
+    sm.lo = lo;
+    sm.scale = scale;
+    sm.edge_a = ra <= n ? (scale > 0.f ? lo + static_cast<float>(sm.t[1]) / scale : lo) : __int_as_float(0x7FC00000);
+    sm.edge_b = rb <= n ? (scale > 0.f ? lo + static_cast<float>(sm.t[2]) / scale : lo) : __int_as_float(0x7FC00000);
+    sm.heavy = m1 > static_cast<uint32_t>(kBoundEntries) ? 1 : 0;
+  }
+  if (m1 > static_cast<uint32_t>(kBoundEntries)) {
     __syncthreads();
-    select_stage_gkeys(gkeys, c, fh_dyn_smem + scratch_off);
-    select_top_p_staged(c, p, sel_off, scratch_off);
     return;
   }
-
-  uint32_t gt = 0u, eq = 0u;  // bit j: key j above / in the boundary bin
-#pragma unroll
-  for (int j = 0; j < KPT; ++j) {
-    gt |= (j < nv && kb[j] > t1) ? (1u << j) : 0u;
-    eq |= (j < nv && kb[j] == t1) ? (1u << j) : 0u;
-  }
-  if (all_in_bin) {
-    gt |= eq;
-  } else {
-    // id-ordered gather of the boundary bin, exact rank, take flags back
-    const uint32_t boff = block_scan_excl_u32(static_cast<uint32_t>(__popc(eq)), sm.wa, nullptr);
-    uint32_t at = boff;
-    for (uint32_t m = eq; m; m &= m - 1u) sm.ckey[at++] = __ldcg(gkeys + id0 + (__ffs(m) - 1));
-    __syncthreads();
-    for (uint32_t a = tid; a < m1; a += kThreads) {
-      const uint32_t ka = sm.ckey[a];
-      uint32_t r = 0;
-#pragma unroll 8
-      for (uint32_t bb = 0; bb < m1; ++bb) {
-        const uint32_t kbb = sm.ckey[bb];
-        r += (kbb > ka || (kbb == ka && bb < a)) ? 1u : 0u;  // index order is id order
-      }
-      sm.ctake[a] = r < need ? 1 : 0;
+  for (int i = tid; i < n; i += kThreads) {
+    const uint32_t x = key[i];
+    if (value_bin(x, lo, scale) == t1) {
+      const uint32_t at = atomicAdd(&sm.nc, 1u);
+      sm.ckey[at] = x;
+      sm.cid[at] = implicit ? i : (ids[i] & 0x7FFFFFFF);
     }
-    __syncthreads();
-    at = boff;
-    for (uint32_t m = eq; m; m &= m - 1u)
-      if (sm.ctake[at++]) gt |= 1u << (__ffs(m) - 1);
   }
-
-  // ascending-id output
-  uint32_t pos = block_scan_excl_u32(static_cast<uint32_t>(__popc(gt)), sm.wb, nullptr);
-  for (uint32_t m = gt; m; m &= m - 1u) {
-    if (pos < static_cast<uint32_t>(p)) sel[pos] = id0 + (__ffs(m) - 1);
-    ++pos;
+  __syncthreads();
+  for (uint32_t a = tid; a < m1; a += kThreads) {
+    const uint32_t ka = sm.ckey[a];
+    const int32_t ia = sm.cid[a];
+    uint32_t r = 0;
+    for (uint32_t bb = 0; bb < m1; ++bb) {
+      const uint32_t kb = sm.ckey[bb];
+      r += (kb > ka || (kb == ka && sm.cid[bb] < ia)) ? 1u : 0u;
+    }
+    if (r + 1u == need) {
+      sm.bkey = ka;
+      sm.bid = ia;
+    }
   }
   __syncthreads();
 }
@@ -958,25 +944,6 @@ __device__ __forceinline__ bool warp_stream(int n, int nslot, uint32_t ring, uin
   return warp_stream_run(n, nslot, ring, slot_bytes, bars, phase_bits, budget, src, use);
 }
 
-// Load n fp32 values from global memory (L2, bypassing L1) and store their
-// order-preserving keys to shared memory; 16 loads per thread are in flight
-// together instead of one L2 round trip per element.
-__device__ __forceinline__ void load_keys_l2(const float* src, int n, uint32_t* skey) {
-  constexpr int KPT = 16;
-  for (int base = 0; base < n; base += KPT * kThreads) {
-    float v[KPT];
-#pragma unroll
-    for (int j = 0; j < KPT; ++j) {
-      const int k = base + j * kThreads + threadIdx.x;
-      v[j] = k < n ? __ldcg(src + k) : 0.f;
-    }
-#pragma unroll
-    for (int j = 0; j < KPT; ++j) {
-      const int k = base + j * kThreads + threadIdx.x;
-      if (k < n) skey[k] = f2key(v[j]);
-    }
-  }
-}
 
 // Load this lane's slice of a bf16 vector into fp32 registers in the layout
 // of 16-byte chunks: chunk m covers elements (lane + 32 m) * 8 .. + 8.
@@ -995,23 +962,6 @@ __device__ __forceinline__ void load_h_chunks(const uint16_t* h, int d, float* h
   }
 }
 
-// Same for the INT4 layout: half-group g (16 elements) = (lane + 32 m), NQ of them.
-template <int NQ>
-__device__ __forceinline__ void load_h_halfgroups(const uint16_t* h, int d, float* hq) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int m = 0; m < NQ; ++m) {
-    const int e = (lane + 32 * m) * 16;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      uint4 w = make_uint4(0, 0, 0, 0);
-      if (e < d) w = *reinterpret_cast<const uint4*>(h + e + 8 * half);
-      float* o = hq + 16 * m + 8 * half;
-      o[0] = bf16lo(w.x); o[1] = bf16hi(w.x); o[2] = bf16lo(w.y); o[3] = bf16hi(w.y);
-      o[4] = bf16lo(w.z); o[5] = bf16hi(w.z); o[6] = bf16lo(w.w); o[7] = bf16hi(w.w);
-    }
-  }
-}
 
 // Dot of a bf16 row in shared memory with register-resident h (chunk layout), warp-reduced.
 template <int NCH>
@@ -1026,21 +976,5 @@ __device__ __forceinline__ float row_dot_bf16(uint32_t row, int d, const float* 
   return warp_sum(acc);
 }
 
-// Dot of a packed INT4 row ([d/2 code bytes][d/16 scale bytes]) with h in the half-group layout.
-template <int NQ>
-__device__ __forceinline__ float row_dot_int4(uint32_t row, int d, const float* hq) {
-  const int lane = threadIdx.x & 31;
-  float acc = 0.f;
-#pragma unroll
-  for (int m = 0; m < NQ; ++m) {
-    const int g = lane + 32 * m;  // half-group
-    if (g * 16 < d) {
-      const uint2 q = lds64(row + 8u * g);
-      const float sc = bf16f(lds16(row + d / 2 + 2u * (g >> 1)));
-      acc = fmaf(sc, dot16q(q, hq + 16 * m), acc);
-    }
-  }
-  return warp_sum(acc);
-}
 
 }  // namespace fh

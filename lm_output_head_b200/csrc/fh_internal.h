@@ -14,6 +14,7 @@ namespace fh {
 constexpr int kMaxD = 2560;
 constexpr long long kWaitBudget = 4000000000LL;      // bulk-copy waits (~2 s)
 constexpr long long kDefaultSpinBudget = 2000000000LL;  // device-wide waits (~1 s)
+constexpr int kB1Bins = 2048;  // histogram bins of the fused B = 1 selection
 
 // Workspace words at the start of the workspace.
 struct SyncWords {
@@ -21,9 +22,13 @@ struct SyncWords {
   uint32_t arrive;        // grid barrier arrivals
   uint32_t ticket;        // kernel exit tickets (last CTA finalises)
   uint32_t union_count;   // distinct clusters of the last batched decode
-  uint32_t epoch;         // fused B = 1 calls so far (selects the per-call buffers)
-  uint32_t ready;         // epoch + 1 once the fused call's cluster selection is published
-  uint32_t pad[2];
+  uint32_t epoch;         // fused B = 1 calls so far
+  uint32_t last_full;     // 1 if the last fused call selected without its histogram
+  float prior_p[2];       // fused call: keys of rank p and 2p in the last call of each mode
+  float prior_2p[2];      //   [greedy: key / |h|, sampling: key]
+  uint32_t prior_ok[2];   // the predictions of a mode hold values
+  uint32_t last_in_range; // keys the last fused call counted in its histogram
+  uint32_t list_count;    // fused call: entries appended to the candidate list
 };
 
 struct B1Params {
@@ -37,8 +42,11 @@ struct B1Params {
   int32_t* out_cluster_ids;
   float* out_max_logit;
   uint32_t* keys;         // workspace [c]: order-preserving keys of the clusters
-  float* z_row;           // workspace [p*b]: candidate logits in canonical order (sampling)
-  int32_t* sel_list;      // workspace [max_probes]: the chosen cluster ids, ascending
+  float* z_buf;           // workspace [c*b]: logit of slot k*b + j of the chosen clusters (sampling)
+  uint32_t* hist;         // workspace [kB1Bins]: counts of keys per bin near the predicted boundary
+  uint32_t* list_key;     // workspace [list_cap]: keys in the predicted region (candidate list)
+  int32_t* list_id;       // workspace [list_cap]: their cluster ids
+  int list_cap;
   unsigned long long* best;
   SyncWords* sync;
   int v, d, c, b, p;

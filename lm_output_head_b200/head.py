@@ -121,6 +121,11 @@ class FlashHead:
     def fused_b1(self) -> bool:
         return bool(self.query(_lib.FH_QUERY_FUSED_B1))
 
+    def last_selection(self):
+        """(keys counted near the predicted boundary, selected from a histogram of all keys?)
+        of the last fused B = 1 decode."""
+        return self.query(_lib.FH_QUERY_LAST_LIST), bool(self.query(_lib.FH_QUERY_LAST_FULL))
+
     def set_spin_budget(self, cycles: int):
         _check(self._lib.fh_set_spin_budget(self._h, int(cycles)), "fh_set_spin_budget")
 

@@ -389,6 +389,33 @@ def _decode_check_gumbel(cfg, head, hid, uni, dh, rows, B, p, T):
     return rep
 
 
+def test_decode_b1_predicted_thresholds_never_change_results(fh):
+    """The fused B = 1 decode predicts where the p-th key lies from the
+    previous call and selects through a histogram of that region, falling
+    back to a general selector when the prediction misses; results must not
+    depend on the prediction."""
+    cfg, head, hid, _, dh0 = get_cfg(1, fh)
+    dh = fh.FlashHead(dh0.E, dh0.C2T, C=dh0.C, max_batch=1, max_probes=cfg.p)
+    try:
+        rep = _decode_check_greedy(cfg, head, hid, dh, [0], 1, cfg.p)
+        assert dh.last_selection() == (0, True)     # first call: nothing predicted, all keys
+        rep.add(_decode_check_greedy(cfg, head, hid, dh, list(range(1, 13)), 1, cfg.p))
+        in_range, full = dh.last_selection()
+        assert not full and in_range >= cfg.p, (in_range, full)
+        assert rep.tight_mismatch <= 1, rep
+        # sampling at temperatures far apart: the carried prediction is far off
+        # (the region misses the boundary), then recovers
+        rng = np.random.default_rng(77)
+        U = rng.random((16, cfg.c), dtype=np.float32)
+        ut = rng.random(16, dtype=np.float32)
+        for i, T in enumerate((0.7, 0.7, 0.02, 50.0, 0.7)):
+            r = _decode_check_gumbel(cfg, head, hid, (U, ut), dh, [3 * i, 3 * i + 1, 3 * i + 2], 1, cfg.p, T)
+            assert r.tight_mismatch <= 1, (T, r)
+        assert dh.device_status() == 0
+    finally:
+        dh.close()
+
+
 def test_decode_gumbel_b1_tiny(fh):
     cfg, head, hid, _, dh = get_cfg(0, fh, n_states=65, max_batch=65, max_probes=256)
     rng = np.random.default_rng(31)
