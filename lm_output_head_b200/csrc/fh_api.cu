@@ -38,6 +38,12 @@ struct fh_head {
   float* cand_logits = nullptr;        // [max_batch, max_probes * b]
   int32_t* row_ok = nullptr;           // [max_batch]
   uint32_t* c2t_counts = nullptr;      // [v]
+  uint32_t* g_cnt = nullptr;           // de-duplication: [c] counts, [c] cursors, [c + 1] offsets
+  uint32_t* g_cur = nullptr;
+  uint32_t* g_off = nullptr;
+  int32_t* g_ulist = nullptr;          // [c]
+  int32_t* g_rows = nullptr;           // [max_batch * max_probes]
+  uint32_t* g_next = nullptr;
   uint32_t* b1_keys = nullptr;         // fused B = 1 state
   float* b1_z_buf = nullptr;           // [c * b]
   uint32_t* b1_hist = nullptr;         // [kB1Bins]
@@ -161,6 +167,44 @@ fh_status launch_candidates_rows(fh_head* h, const void* hidden, int32_t B, int3
   return e == cudaSuccess ? FH_OK : cuda_fail(e);
 }
 
+// Batches of at least this many hidden rows score centroids (and run the
+// dense head) on the tensor cores; smaller ones stream rows on CUDA cores.
+constexpr int kGemmMinBatch = 64;
+
+// tcgen05 GEMM over blocks of up to 256 hidden rows. epi 0: out[r][k] =
+// scores (mode 0) or Gumbel keys (mode 1) of A = the centroids; epi 1: packed
+// (logit, token) maxima of A = E into h->best[r] (+ optional logits out[r][t]).
+fh_status launch_gemm_rows(fh_head* h, const void* hidden, int32_t B, int epi, int mode, float T, const float* u,
+                           float* out, cudaStream_t st) {
+  const fh_head_desc& D = h->desc;
+  const bool centroids = epi == 0;
+  const bool int4 = centroids && D.fmt == FH_CENTROID_INT4_G32;
+  const int rows = centroids ? D.c : D.v;
+  const long long ldo = rows;
+  for (int r0 = 0; r0 < B; r0 += 256) {
+    GemmParams P{};
+    P.rows = rows;
+    P.d = D.d;
+    P.nb = std::min(256, B - r0);
+    P.int4 = int4 ? 1 : 0;
+    P.epi = epi;
+    P.mode = mode;
+    P.T = T;
+    P.crows = h->crows;
+    P.crow_bytes = h->crow_bytes;
+    P.out = out ? out + static_cast<size_t>(r0) * ldo : nullptr;
+    P.ldo = ldo;
+    P.u = u ? u + static_cast<size_t>(r0) * ldo : nullptr;
+    P.best = h->best + r0;
+    P.status = &h->sync->status;
+    const void* A = centroids ? (int4 ? nullptr : D.C) : D.E;
+    const void* H = static_cast<const uint16_t*>(hidden) + static_cast<size_t>(r0) * D.d;
+    cudaError_t e = launch_gemm(P, A, H, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return FH_OK;
+}
+
 size_t select_smem(const fh_head* h, int32_t p) {
   return up(static_cast<size_t>(p) * 4, 128) + hist_select_smem_bytes(h->desc.c);
 }
@@ -240,6 +284,12 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   const size_t o_log = take(mb * nc * 4);
   const size_t o_rok = take(mb * 4);
   const size_t o_cnt = take(static_cast<size_t>(D.v) * 4);
+  const size_t o_gcnt = take(static_cast<size_t>(D.c) * 4);
+  const size_t o_gcur = take(static_cast<size_t>(D.c) * 4);
+  const size_t o_goff = take(static_cast<size_t>(D.c + 1) * 4);
+  const size_t o_gul = take(static_cast<size_t>(D.c) * 4);
+  const size_t o_grows = take(mb * mp * 4);
+  const size_t o_gnext = take(16);
   const int words = (D.c + 31) / 32;
   const size_t o_keys1 = take(static_cast<size_t>(D.c) * 4);
   const size_t o_zbuf = take(static_cast<size_t>(D.v) * 4);
@@ -269,6 +319,12 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   h->cand_logits = reinterpret_cast<float*>(h->ws + o_log);
   h->row_ok = reinterpret_cast<int32_t*>(h->ws + o_rok);
   h->c2t_counts = reinterpret_cast<uint32_t*>(h->ws + o_cnt);
+  h->g_cnt = reinterpret_cast<uint32_t*>(h->ws + o_gcnt);
+  h->g_cur = reinterpret_cast<uint32_t*>(h->ws + o_gcur);
+  h->g_off = reinterpret_cast<uint32_t*>(h->ws + o_goff);
+  h->g_ulist = reinterpret_cast<int32_t*>(h->ws + o_gul);
+  h->g_rows = reinterpret_cast<int32_t*>(h->ws + o_grows);
+  h->g_next = reinterpret_cast<uint32_t*>(h->ws + o_gnext);
   h->b1_keys = reinterpret_cast<uint32_t*>(h->ws + o_keys1);
   h->b1_z_buf = reinterpret_cast<float*>(h->ws + o_zbuf);
   h->b1_hist = reinterpret_cast<uint32_t*>(h->ws + o_hist1);
@@ -287,6 +343,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
         e = set_attrs_decode_b1(ms);
         if (e == cudaSuccess) e = set_attrs_batched(ms);
         if (e == cudaSuccess) e = set_attrs_dense(ms);
+        if (e == cudaSuccess) e = set_attrs_gemm();
         if (e != cudaSuccess) {
           status = cuda_fail(e);
           break;
@@ -407,6 +464,8 @@ fh_status fh_centroid_scores(fh_head* h, const void* hidden, int32_t B, float* s
   fh_status s = check_call(h, hidden, B);
   if (s != FH_OK) return s;
   if (!scores || !aligned(scores, 4)) return FH_ERR_INVALID_ARG;
+  if (B >= kGemmMinBatch)
+    return launch_gemm_rows(h, hidden, B, 0, 0, 1.f, nullptr, scores, reinterpret_cast<cudaStream_t>(stream));
   return launch_scores_rows(h, hidden, B, 0, 1.f, nullptr, scores, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -510,7 +569,9 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
   }
 
   // batched path: keys -> per-row select -> candidates -> epilogue
-  s = launch_scores_rows(h, hidden, B, gumbel ? 1 : 0, gumbel ? T : 1.f, u_clusters, h->keys, st);
+  s = B >= kGemmMinBatch
+          ? launch_gemm_rows(h, hidden, B, 0, gumbel ? 1 : 0, gumbel ? T : 1.f, u_clusters, h->keys, st)
+          : launch_scores_rows(h, hidden, B, gumbel ? 1 : 0, gumbel ? T : 1.f, u_clusters, h->keys, st);
   if (s != FH_OK) return s;
   SelectParams SP{};
   SP.in = h->keys;
@@ -526,8 +587,33 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
   if (ssm > h->smem_budget) return FH_ERR_UNSUPPORTED;
   cudaError_t e = launch_select(SP, B, ssm, st);
   if (e != cudaSuccess) return cuda_fail(e);
-  s = launch_candidates_rows(h, hidden, B, p, gumbel ? h->cand_logits : nullptr, nullptr, true, false, st);
-  if (s != FH_OK) return s;
+  if (D.b == 16) {
+    // de-duplicated across the batch: every chosen cluster's token rows are read once
+    GroupParams GP{};
+    GP.sel = h->sel;
+    GP.C2T = D.C2T;
+    GP.E = static_cast<const uint16_t*>(D.E);
+    GP.H = static_cast<const uint16_t*>(hidden);
+    GP.cnt = h->g_cnt;
+    GP.cur = h->g_cur;
+    GP.off = h->g_off;
+    GP.ulist = h->g_ulist;
+    GP.rows_of = h->g_rows;
+    GP.union_count = &h->sync->union_count;
+    GP.next = h->g_next;
+    GP.best = h->best;
+    GP.logits = gumbel ? h->cand_logits : nullptr;
+    GP.B = B;
+    GP.p = p;
+    GP.c = D.c;
+    GP.b = D.b;
+    GP.d = D.d;
+    e = launch_group(GP, h->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+  } else {
+    s = launch_candidates_rows(h, hidden, B, p, gumbel ? h->cand_logits : nullptr, nullptr, true, false, st);
+    if (s != FH_OK) return s;
+  }
   EpilogueParams EP{};
   EP.logits = h->cand_logits;
   EP.cand_tok = h->cand_tok;
@@ -554,6 +640,18 @@ fh_status fh_dense_head(fh_head* h, const void* hidden, int32_t B, float* logits
   if (!out_argmax) return FH_ERR_INVALID_ARG;
   const fh_head_desc& D = h->desc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (B >= kGemmMinBatch) {
+    // tensor cores: fused column argmax into h->best, then one word per row out
+    s = launch_gemm_rows(h, hidden, B, 1, 0, 1.f, nullptr, logits, st);
+    if (s != FH_OK) return s;
+    EpilogueParams EP{};
+    EP.best = h->best;
+    EP.out_tokens = out_argmax;
+    EP.mode = 0;
+    EP.T = 1.f;
+    cudaError_t e = launch_epilogue(EP, B, st);
+    return e == cudaSuccess ? FH_OK : cuda_fail(e);
+  }
   const int rmax = dense_max_rows();
   for (int r0 = 0; r0 < B; r0 += rmax) {
     const int rows = B - r0 < rmax ? B - r0 : rmax;

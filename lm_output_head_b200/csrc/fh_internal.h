@@ -123,6 +123,40 @@ struct DenseParams {
   int off_h, off_bar, off_ring;
 };
 
+struct GemmParams {
+  int rows, d;              // streamed operand: rows x d (centroid or token rows), K = d
+  int nb;                   // hidden rows of this launch, 1..256 (two M blocks of 128)
+  int hm, tn, nbuf, stages, tmem_cols;  // set by the launcher
+  int int4;                 // streamed operand given as packed INT4 rows (crows) instead of bf16
+  int epi;                  // 0: store scores / keys, 1: per-hidden-row argmax
+  int mode;                 // epi 0: 0 raw scores, 1 Gumbel keys
+  float T;
+  const uint8_t* crows;
+  int crow_bytes;
+  float* out;               // [nb, ldo]: scores/keys (epi 0) or logits (epi 1, may be null)
+  long long ldo;
+  const float* u;           // [nb, ldo] Gumbel uniforms (epi 0, mode 1)
+  unsigned long long* best; // [nb] packed (logit, token) maxima (epi 1)
+  int* status;
+};
+
+struct GroupParams {
+  const int32_t* sel;       // [B, p] chosen clusters per row, ascending
+  const int32_t* C2T;       // [c, b]
+  const uint16_t* E;        // [v, d]
+  const uint16_t* H;        // [B, d]
+  uint32_t* cnt;            // [c] workspace: rows per cluster
+  uint32_t* cur;            // [c] workspace: fill cursors
+  uint32_t* off;            // [c + 1] workspace: CSR offsets
+  int32_t* ulist;           // [c] workspace: the union of chosen clusters, ascending
+  int32_t* rows_of;         // [B * p] workspace: rows of each cluster, grouped by cluster
+  uint32_t* union_count;    // |union|
+  uint32_t* next;           // work counter of the grouped kernel
+  unsigned long long* best; // [B] packed (logit, token) maxima
+  float* logits;            // [B, p*b] canonical candidate logits (sampling), or null
+  int B, p, c, b, d;
+};
+
 struct C2TCheckParams {
   const int32_t* C2T;
   uint32_t* counts;         // [v]
@@ -150,6 +184,12 @@ cudaError_t launch_epilogue(const EpilogueParams& P, int B, cudaStream_t st);
 cudaError_t launch_dense(const DenseParams& P, int grid, size_t smem, int nch, cudaStream_t st);
 cudaError_t launch_c2t_check(const C2TCheckParams& P, cudaStream_t st);
 cudaError_t launch_repack_int4(const RepackParams& P, cudaStream_t st);
+// tcgen05 GEMM (B >= 64): streamed rows bf16 [rows, d] through TMA, or packed INT4 rows; H bf16 [nb, d].
+cudaError_t launch_gemm(const GemmParams& P, const void* rows_bf16, const void* H, int num_sms, cudaStream_t st);
+cudaError_t set_attrs_gemm();
+// De-duplicated candidate logits of a batch (b == 16): CSR of the selections by cluster, then one
+// pass per distinct cluster on the tensor cores.
+cudaError_t launch_group(const GroupParams& P, int num_sms, cudaStream_t st);
 
 // Opt-in shared memory attribute for every instantiation (called once per device).
 cudaError_t set_kernel_attributes(int max_smem);

@@ -143,8 +143,11 @@ def test_workspace_limit_gives_oom(fh, monkeypatch):
 # ---------------------------------------------------------------------------
 # stage 1: centroid scores
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("cfg_id,B", [(0, 1), (0, 32), (1, 1), (2, 1), (2, 4), (2, 16), (3, 32), (4, 256)])
+@pytest.mark.parametrize("cfg_id,B", [(0, 1), (0, 32), (0, 64), (0, 65), (1, 1), (2, 1), (2, 4), (2, 16), (3, 32),
+                                      (4, 256)])
 def test_centroid_scores(fh, cfg_id, B):
+    """B >= 64 runs the tcgen05 tile GEMM (bf16, or INT4 dequantised as exact hi + lo
+    bf16 pairs); smaller batches stream centroid rows on CUDA cores."""
     cfg, head, hid, _, dh = get_cfg(cfg_id, fh)
     H = hid.H[:B]
     s = dh.centroid_scores(hid_dev(H)).cpu().numpy()
@@ -416,6 +419,25 @@ def test_decode_b1_predicted_thresholds_never_change_results(fh):
         dh.close()
 
 
+def test_decode_batch_deduplicates_shared_clusters(fh):
+    """Batched decodes group the chosen (row, cluster) pairs by cluster and read each
+    distinct cluster's token rows once: a batch of one repeated hidden state gathers
+    exactly p clusters, and every row gets the single-row answer."""
+    cfg, head, hid, _, dh = get_cfg(0, fh, n_states=65, max_batch=65, max_probes=256)
+    H = np.repeat(hid.H[3:4], 64, axis=0)
+    tok = dh.decode(hid_dev(H), cfg.p).cpu().numpy()
+    assert dh.device_status() == 0
+    assert dh.query(1) == cfg.p              # FH_QUERY_LAST_UNION
+    ref, _, _ = oracle.decode(head, H[:1], cfg.p)
+    assert np.all(tok == tok[0])
+    assert parity.check_greedy_token(head, H[0], oracle.select_greedy(
+        oracle.centroid_scores(oracle.centroid_matrix(head), H[:1]), cfg.p)[0], int(tok[0])).tight_mismatch == 0
+    # distinct rows: the union lies between p and min(c, B p)
+    dh.decode(hid_dev(hid.H[:64]), cfg.p)
+    u = dh.query(1)
+    assert cfg.p <= u <= min(cfg.c, 64 * cfg.p)
+
+
 def test_decode_gumbel_b1_tiny(fh):
     cfg, head, hid, _, dh = get_cfg(0, fh, n_states=65, max_batch=65, max_probes=256)
     rng = np.random.default_rng(31)
@@ -433,8 +455,9 @@ def test_decode_gumbel_qwen_b32(fh):
 # ---------------------------------------------------------------------------
 # dense head
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("cfg_id,B", [(0, 1), (0, 33), (1, 1), (1, 4), (3, 2)])
+@pytest.mark.parametrize("cfg_id,B", [(0, 1), (0, 33), (0, 65), (1, 1), (1, 4), (3, 2), (4, 64)])
 def test_dense_head(fh, cfg_id, B):
+    """B >= 64 runs the tcgen05 tile GEMM with the fused column argmax."""
     cfg, head, hid, _, dh = get_cfg(cfg_id, fh) if cfg_id else get_cfg(0, fh, n_states=65, max_batch=65,
                                                                        max_probes=256)
     H = hid.H[:B]
