@@ -514,21 +514,31 @@ static __device__ __noinline__ void select_top_p_staged(int c, int p, uint32_t s
     __syncthreads();
   }
 
-  // ascending-id compaction: thread t owns ids [t*kpt, t*kpt + kpt); one block scan
-  const int kpt = (c + kThreads - 1) / kThreads;
-  const int id0 = min(c, tid * kpt), id1 = min(c, id0 + kpt);
+  // ascending-id compaction: warp w owns ids [w * span, w * span + span), 32
+  // consecutive ids per step (one per lane: no shared-memory bank conflicts)
+  const int span = ((c + kWarps - 1) / kWarps + 31) & ~31;
+  const int w0 = min(c, warp * span), w1 = min(c, w0 + span);
+  auto taken = [&](int k) {
+    const uint32_t bn = value_bin(key[k], lo, scale);
+    return bn > t1 || (bn == t1 && (all_in_bin || flag[k]));
+  };
   uint32_t cnt = 0;
-  for (int k = id0; k < id1; ++k) {
-    const uint32_t bn = value_bin(key[k], lo, scale);
-    cnt += (bn > t1 || (bn == t1 && (all_in_bin || flag[k]))) ? 1u : 0u;
+  for (int base = w0; base < w1; base += 32) {
+    const int k = base + lane;
+    cnt += __popc(__ballot_sync(0xFFFFFFFFu, k < w1 && taken(k)));
   }
-  uint32_t pos = block_exclusive_scan<kThreads, uint32_t>(cnt, sm.scan, nullptr);
-  for (int k = id0; k < id1; ++k) {
-    const uint32_t bn = value_bin(key[k], lo, scale);
-    if (bn > t1 || (bn == t1 && (all_in_bin || flag[k]))) {
-      if (pos < static_cast<uint32_t>(p)) sel[pos] = k;
-      ++pos;
-    }
+  if (lane == 0) sm.scan[warp] = cnt;
+  __syncthreads();
+  uint32_t pos = 0;
+  for (int w = 0; w < warp; ++w) pos += sm.scan[w];
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int base = w0; base < w1; base += 32) {
+    const int k = base + lane;
+    const bool tk = k < w1 && taken(k);
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, tk);
+    const uint32_t at = pos + __popc(m & lt);
+    if (tk && at < static_cast<uint32_t>(p)) sel[at] = k;
+    pos += __popc(m);
   }
   __syncthreads();
 }

@@ -13,7 +13,7 @@
 //   - warp 5 (one lane) loads H blocks, and the streamed rows when they are
 //     bf16, with TMA (cp.async.bulk.tensor, 128-byte swizzle, no multicast)
 //     into a ring of shared-memory stages of 64 K-elements;
-//   - INT4 centroids: warps 8..11 read the packed codes and bf16 scales and
+//   - INT4 centroids: warps 8..15 read the packed codes and bf16 scales and
 //     write code * scale into the stage as an exact pair of bf16 tiles
 //     hi + lo (hi = bf16(code * scale), lo = the rest, exact in bf16), in the
 //     same swizzled layout, so two MMAs give the exact products;
@@ -28,6 +28,7 @@
 // Every wait is bounded; one that runs out records FH_ERR_TIMEOUT, the CTA
 // drains its copies and MMAs, frees its tensor memory and returns.
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -38,13 +39,13 @@
 namespace fh {
 namespace {
 
-constexpr int kGemmThreads = 384;  // 12 warps
+constexpr int kGemmThreads = 512;  // 16 warps
 constexpr int kTileM = 128;
 constexpr int kTileK = 64;         // bf16 elements per stage row: 128 bytes, one swizzle span
 constexpr int kMaxN = 256;
 constexpr long long kGemmBudget = 4000000000LL;
 
-constexpr int kDequantThreads = 128;  // warps 8..11
+constexpr int kDequantThreads = 256;  // warps 8..15
 
 struct GemmSmem {  // after the stages
   unsigned long long full[4], empty[4], tfull[2], tempty[2], done;
@@ -119,11 +120,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// bf16 bits of x, round to nearest even (x finite)
-__device__ __forceinline__ uint32_t bf16_rn_bits(float x) {
-  const uint32_t u = __float_as_uint(x);
-  return (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
-}
 
 template <bool B_INT4>
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -202,51 +198,58 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (B_INT4 && warp >= 8) {
     // ---------------- INT4 dequantisation of the streamed rows (hi + lo bf16) ----------------
-    const int r0 = tid - 8 * 32;  // rows r0, r0 + 128, ... of the tile
+    // thread pair (2r, 2r + 1) handles row r of the tile, 32 elements each; the
+    // codes of a stage are loaded before its slot is free
+    const int dt = tid - 8 * 32;  // 0 .. kDequantThreads-1
+    const int half = dt & 1;
     int g = 0;
     bool ok = true;
     for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
       for (int ks = 0; ks < kst; ++ks, ++g) {
         const int s = g % S;
         const uint32_t ph = static_cast<uint32_t>(g / S) & 1u;
+        const int e0 = ks * kTileK + 32 * half;  // this thread's 32 elements (one scale group)
+        constexpr int kRowsPerPass = kDequantThreads / 2;
+        const int nrow = tn / kRowsPerPass;  // 2 (tn 128) or 4 (tn 256)
+        uint4 q[4];
+        uint32_t scw[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          q[i] = make_uint4(0, 0, 0, 0);
+          scw[i] = 0u;
+          const int r = (dt >> 1) + i * kRowsPerPass;
+          const int row = t * tn + r;
+          if (i < nrow && row < P.rows && e0 < P.d) {
+            const uint8_t* src = P.crows + static_cast<size_t>(row) * P.crow_bytes;
+            q[i] = *reinterpret_cast<const uint4*>(src + e0 / 2);
+            scw[i] = *reinterpret_cast<const unsigned short*>(src + P.d / 2 + 2 * (e0 / 32));
+          }
+        }
         if (!wait_parity(bar(sm.empty[s]), ph ^ 1u, abort_flag, kGemmBudget)) {
           ok = false;
           break;
         }
-        const int e0 = ks * kTileK;
-        for (int r = r0; r < tn; r += kDequantThreads) {
-          const int row = t * tn + r;
-          // codes and scales of elements e0 .. e0+63 (two groups of 32)
-          uint4 q0 = make_uint4(0, 0, 0, 0), q1 = make_uint4(0, 0, 0, 0);
-          uint32_t scw = 0;
-          if (row < P.rows) {
-            const uint8_t* src = P.crows + static_cast<size_t>(row) * P.crow_bytes;
-            q0 = *reinterpret_cast<const uint4*>(src + e0 / 2);
-            if (e0 + 32 < P.d) {
-              q1 = *reinterpret_cast<const uint4*>(src + e0 / 2 + 16);
-              scw = *reinterpret_cast<const uint32_t*>(src + P.d / 2 + 2 * (e0 / 32));
-            } else {
-              scw = *reinterpret_cast<const unsigned short*>(src + P.d / 2 + 2 * (e0 / 32));
-            }
-          }
-          const float sc0 = __uint_as_float(scw << 16), sc1 = __uint_as_float(scw & 0xFFFF0000u);
-          const uint32_t qw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (i >= nrow) break;
+          const int r = (dt >> 1) + i * kRowsPerPass;
+          const float scl = __uint_as_float(scw[i] << 16);
+          const uint32_t qw[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
           uint8_t* hi = gbase + (b_hi(s) - base) + r * 128;
           uint8_t* lo = gbase + (b_lo(s) - base) + r * 128;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {  // 16-byte chunk j: elements 8j .. 8j+7
-            const float scl = j < 4 ? sc0 : sc1;
+          for (int j = 0; j < 4; ++j) {  // 16-byte chunk 4 half + j: elements 8j .. 8j+7 of the half
             uint32_t h[4], l[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float v0 = nib(qw[j], 2 * e) * scl, v1 = nib(qw[j], 2 * e + 1) * scl;
-              const uint32_t h0 = bf16_rn_bits(v0), h1 = bf16_rn_bits(v1);
-              const uint32_t l0 = bf16_rn_bits(v0 - __uint_as_float(h0 << 16));
-              const uint32_t l1 = bf16_rn_bits(v1 - __uint_as_float(h1 << 16));
-              h[e] = h0 | (h1 << 16);
-              l[e] = l0 | (l1 << 16);
+              const __nv_bfloat162 hb = __floats2bfloat162_rn(v0, v1);
+              const float2 hf = __bfloat1622float2(hb);
+              const __nv_bfloat162 lb = __floats2bfloat162_rn(v0 - hf.x, v1 - hf.y);  // exact rest
+              h[e] = *reinterpret_cast<const uint32_t*>(&hb);
+              l[e] = *reinterpret_cast<const uint32_t*>(&lb);
             }
-            const int pc = (j ^ (r & 7)) * 16;  // 128-byte swizzle of chunk j in row r
+            const int pc = ((4 * half + j) ^ (r & 7)) * 16;  // 128-byte swizzle of the chunk in row r
             *reinterpret_cast<uint4*>(hi + pc) = make_uint4(h[0], h[1], h[2], h[3]);
             *reinterpret_cast<uint4*>(lo + pc) = make_uint4(l[0], l[1], l[2], l[3]);
           }

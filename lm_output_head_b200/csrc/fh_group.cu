@@ -36,28 +36,53 @@ __global__ void csr_count_kernel(const GroupParams P) {
 }
 
 // One CTA: exclusive scan of the c counts into off[0..c], the union list
-// (clusters with a nonzero count, ascending) and its length.
+// (clusters with a nonzero count, ascending) and its length. Thread t owns
+// 32 consecutive ids, read and written as 16-byte vectors (c % 4 == 0), or
+// one by one otherwise.
 __global__ void __launch_bounds__(kThreads, 1) csr_scan_kernel(const GroupParams P) {
   __shared__ uint32_t wsum[kWarps], wsum2[kWarps];
   const int tid = threadIdx.x;
-  const int per = (P.c + kThreads - 1) / kThreads;
-  const int k0 = min(P.c, tid * per), k1 = min(P.c, k0 + per);
-  uint32_t tot = 0, nz = 0;
-  for (int k = k0; k < k1; ++k) {
-    const uint32_t v = P.cnt[k];
-    tot += v;
-    nz += v ? 1u : 0u;
+  constexpr int kPer = 32;
+  uint32_t all_tot = 0, all_nz = 0, carry_o = 0, carry_u = 0;
+  const bool vec = (P.c & 3) == 0;
+  for (int base = 0; base < P.c; base += kPer * kThreads) {  // one pass for c <= 16384
+    const int k0 = base + tid * kPer;
+    uint32_t v[kPer];
+    if (vec && k0 + kPer <= P.c) {
+#pragma unroll
+      for (int j = 0; j < kPer; j += 4) {
+        const uint4 x = *reinterpret_cast<const uint4*>(P.cnt + k0 + j);
+        v[j] = x.x; v[j + 1] = x.y; v[j + 2] = x.z; v[j + 3] = x.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) v[j] = k0 + j < P.c ? P.cnt[k0 + j] : 0u;
+    }
+    uint32_t tot = 0, nz = 0;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      tot += v[j];
+      nz += v[j] ? 1u : 0u;
+    }
+    uint32_t ptot, pnz;
+    uint32_t o = carry_o + block_scan_excl_u32(tot, wsum, &ptot);
+    uint32_t u = carry_u + block_scan_excl_u32(nz, wsum2, &pnz);
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int k = k0 + j;
+      if (k < P.c) {
+        P.off[k] = o;
+        if (v[j]) P.ulist[u++] = k;
+      }
+      o += v[j];
+    }
+    carry_o += ptot;
+    carry_u += pnz;
+    __syncthreads();
   }
-  uint32_t all_tot, all_nz;
-  uint32_t o = block_scan_excl_u32(tot, wsum, &all_tot);
-  uint32_t u = block_scan_excl_u32(nz, wsum2, &all_nz);
-  for (int k = k0; k < k1; ++k) {
-    const uint32_t v = P.cnt[k];
-    P.off[k] = o;
-    P.cur[k] = 0u;
-    o += v;
-    if (v) P.ulist[u++] = k;
-  }
+  all_tot = carry_o;
+  all_nz = carry_u;
+  for (int k = tid; k < P.c; k += kThreads) P.cur[k] = 0u;
   if (tid == 0) {
     P.off[P.c] = all_tot;
     *P.union_count = all_nz;
@@ -87,8 +112,10 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4],
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t ld_pair(const uint16_t* p, int k, int d) {
-  return k < d ? __ldg(reinterpret_cast<const uint32_t*>(p + k)) : 0u;  // k even, d even: pairs never straddle d
+// Eight consecutive bf16 of a row from element k (k % 8 == 0, d % 8 == 0: a
+// chunk never straddles d); zeros past the row's end.
+__device__ __forceinline__ uint4 ld_chunk(const uint16_t* p, int k, int d) {
+  return k < d ? __ldg(reinterpret_cast<const uint4*>(p + k)) : make_uint4(0, 0, 0, 0);
 }
 
 // Position of cluster k among the row's ascending clusters (binary search).
@@ -133,13 +160,26 @@ __global__ void __launch_bounds__(256) group_kernel(const GroupParams P) {
       float acc[kChunks][4];
 #pragma unroll
       for (int ch = 0; ch < kChunks; ++ch) acc[ch][0] = acc[ch][1] = acc[ch][2] = acc[ch][3] = 0.f;
-#pragma unroll 4
-      for (int k0 = 0; k0 < d; k0 += 16) {
-        const int ka = k0 + 2 * t, kb = k0 + 8 + 2 * t;
-        const uint32_t a[4] = {ld_pair(ea, ka, d), ld_pair(eb, ka, d), ld_pair(ea, kb, d), ld_pair(eb, kb, d)};
+      // The dot product over K is order-free, so two MMA K-steps take 32
+      // elements in a lane-friendly order: lane t of a fragment row loads the
+      // 8 contiguous elements [k0 + 8t, k0 + 8t + 8); the first K-step uses
+      // elements 8t..8t+3 (as its columns 2t, 2t+1, 2t+8, 2t+9), the second
+      // 8t+4..8t+7. A and B use the same order, so the sums are unchanged.
+#pragma unroll 2
+      for (int k0 = 0; k0 < d; k0 += 32) {
+        const int kk = k0 + 8 * t;
+        const uint4 xa = ld_chunk(ea, kk, d), xb = ld_chunk(eb, kk, d);
+        uint4 xh[kChunks];
+#pragma unroll
+        for (int ch = 0; ch < kChunks; ++ch) xh[ch] = ch < nch ? ld_chunk(hrow[ch], kk, d) : make_uint4(0, 0, 0, 0);
+        const uint32_t a0[4] = {xa.x, xb.x, xa.y, xb.y};
+        const uint32_t a1[4] = {xa.z, xb.z, xa.w, xb.w};
 #pragma unroll
         for (int ch = 0; ch < kChunks; ++ch) {
-          if (ch < nch) mma_16816(acc[ch], a, ld_pair(hrow[ch], ka, d), ld_pair(hrow[ch], kb, d));
+          if (ch < nch) {
+            mma_16816(acc[ch], a0, xh[ch].x, xh[ch].y);
+            mma_16816(acc[ch], a1, xh[ch].z, xh[ch].w);
+          }
         }
       }
       // acc[ch]: (slot g, col 2t), (slot g, col 2t+1), (slot g+8, col 2t), (slot g+8, col 2t+1)
