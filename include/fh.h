@@ -107,10 +107,13 @@ typedef struct fh_head fh_head;
 /*
  * Create a head. Validates the description, checks on the device that C2T
  * is a permutation of 0..v-1 (FH_ERR_INVALID_C2T otherwise), allocates the
- * workspace, and for INT4 packs each centroid row with its scales into a
- * library-owned copy (row = d/2 code bytes, then d/16 scale bytes, padded to
- * 16 bytes) so that one bulk copy moves a row. Synchronises `stream` once.
- * On success *out owns the workspace; release it with fh_destroy.
+ * workspace, and fills two library-owned copies inside it: the token rows of
+ * E in cluster-major order (row k*b + j = E[C2T[k][j]], v*d*2 bytes; a
+ * cluster's b rows are one contiguous block, read without a C2T lookup), and,
+ * for INT4, each centroid row packed with its scales (row = d/2 code bytes,
+ * then d/16 scale bytes, padded to 16 bytes) so that one bulk copy moves a
+ * row. Synchronises `stream`. On success *out owns the workspace; release it
+ * with fh_destroy. E itself is still read by the dense head.
  */
 fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out);
 

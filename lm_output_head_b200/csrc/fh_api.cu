@@ -38,6 +38,7 @@ struct fh_head {
   float* cand_logits = nullptr;        // [max_batch, max_probes * b]
   int32_t* row_ok = nullptr;           // [max_batch]
   uint32_t* c2t_counts = nullptr;      // [v]
+  uint16_t* Ecm = nullptr;             // [v, d] cluster-major copy of the token rows
   uint32_t* g_cnt = nullptr;           // de-duplication: [c] counts, [c] cursors, [c + 1] offsets
   uint32_t* g_cur = nullptr;
   uint32_t* g_off = nullptr;
@@ -284,6 +285,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   const size_t o_log = take(mb * nc * 4);
   const size_t o_rok = take(mb * 4);
   const size_t o_cnt = take(static_cast<size_t>(D.v) * 4);
+  const size_t o_ecm = take(static_cast<size_t>(D.v) * D.d * 2);
   const size_t o_gcnt = take(static_cast<size_t>(D.c) * 4);
   const size_t o_gcur = take(static_cast<size_t>(D.c) * 4);
   const size_t o_goff = take(static_cast<size_t>(D.c + 1) * 4);
@@ -319,6 +321,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   h->cand_logits = reinterpret_cast<float*>(h->ws + o_log);
   h->row_ok = reinterpret_cast<int32_t*>(h->ws + o_rok);
   h->c2t_counts = reinterpret_cast<uint32_t*>(h->ws + o_cnt);
+  h->Ecm = reinterpret_cast<uint16_t*>(h->ws + o_ecm);
   h->g_cnt = reinterpret_cast<uint32_t*>(h->ws + o_gcnt);
   h->g_cur = reinterpret_cast<uint32_t*>(h->ws + o_gcur);
   h->g_off = reinterpret_cast<uint32_t*>(h->ws + o_goff);
@@ -344,6 +347,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
         if (e == cudaSuccess) e = set_attrs_batched(ms);
         if (e == cudaSuccess) e = set_attrs_dense(ms);
         if (e == cudaSuccess) e = set_attrs_gemm();
+        if (e == cudaSuccess) e = set_attrs_group();
         if (e != cudaSuccess) {
           status = cuda_fail(e);
           break;
@@ -366,6 +370,10 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) { status = cuda_fail(e); break; }
     if (bad) { status = FH_ERR_INVALID_C2T; break; }
+    // token rows in cluster-major order (C2T is a permutation: every read is in range)
+    e = launch_gather_cluster_major(static_cast<const uint16_t*>(D.E), D.C2T, h->Ecm, D.v, D.d, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) { status = cuda_fail(e); break; }
   } while (false);
   if (status != FH_OK) {
     cudaFree(h->ws);
@@ -534,6 +542,7 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
   if (B == 1 && h->fused_ok) {
     B1Params P{};
     P.E = static_cast<const uint16_t*>(D.E);
+    P.Ecm = h->Ecm;
     P.Crows = h->crows;
     P.C2T = D.C2T;
     P.hidden = static_cast<const uint16_t*>(hidden);
@@ -592,7 +601,7 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
     GroupParams GP{};
     GP.sel = h->sel;
     GP.C2T = D.C2T;
-    GP.E = static_cast<const uint16_t*>(D.E);
+    GP.Ecm = h->Ecm;
     GP.H = static_cast<const uint16_t*>(hidden);
     GP.cnt = h->g_cnt;
     GP.cur = h->g_cur;

@@ -30,8 +30,10 @@
 //  3. the chosen clusters in a fixed order (list order, or ascending ids after
 //     the general selector) give the candidate rows: row r is slot r % b of
 //     the (r / b)-th chosen cluster and belongs to CTA r mod G, warp
-//     (r / G) mod 16; it is read through C2T and dotted with h (section 1.2.4,
-//     stage 2), keeping a packed (logit, token) maximum.
+//     (r / G) mod 16; it is read from the head's cluster-major copy of E (row
+//     k*b + j holds token C2T[k][j], so no C2T lookup precedes the row load)
+//     and dotted with h (section 1.2.4, stage 2), keeping a packed (logit,
+//     token) maximum.
 //  4. CTA maxima meet in one 64-bit atomicMax; the last CTA to finish (exit
 //     ticket) writes the token: the argmax, or, when sampling, the inverse-CDF
 //     draw over softmax(z/T) in canonical order (cluster asc, slot asc)
@@ -433,24 +435,25 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   for (int r0 = cw; ok && r0 < r_all; r0 += 2 * cstride) {
     const int r1 = r0 + cstride;
     const bool two = r1 < r_all;
-    int t = 0;
-    if (lane == 0 || (lane == 1 && two)) {
-      const int r = lane == 0 ? r0 : r1;
-      const int k = ssel[r / b];
-      t = (k >= 0 && k < c) ? __ldg(P.C2T + static_cast<size_t>(k) * b + r % b) : -1;
-    }
-    const int t0 = __shfl_sync(0xFFFFFFFFu, t, 0);
-    const int t1 = two ? __shfl_sync(0xFFFFFFFFu, t, 1) : 0;
-    if (t0 < 0 || t1 < 0 || t0 >= P.v || t1 >= P.v) {  // only an inconsistent selection; never read outside E
+    // the rows sit at k*b + j of the cluster-major copy: their loads do not wait for C2T,
+    // whose entries (the token ids of the output) are read alongside
+    const int k0 = ssel[r0 / b], k1 = two ? ssel[r1 / b] : k0;
+    if (k0 < 0 || k0 >= c || k1 < 0 || k1 >= c) {  // only an inconsistent selection; never read outside E
       ok = false;
       break;
     }
+    const size_t q0 = static_cast<size_t>(k0) * b + r0 % b, q1 = static_cast<size_t>(k1) * b + r1 % b;
     if (two && lane == 0) {
       mbar_expect_tx(wbar, static_cast<uint32_t>(d * 2));
-      bulk_g2s(slot, P.E + static_cast<size_t>(t1) * d, static_cast<uint32_t>(d * 2), wbar);
+      bulk_g2s(slot, P.Ecm + q1 * d, static_cast<uint32_t>(d * 2), wbar);
     }
     uint4 e[NCH];
-    row_load_bf16<NCH>(P.E + static_cast<size_t>(t0) * d, d, e);
+    row_load_bf16<NCH>(P.Ecm + q0 * d, d, e);
+    int t = 0;
+    if (lane == 0) t = __ldg(P.C2T + q0);
+    else if (lane == 1 && two) t = __ldg(P.C2T + q1);
+    const int t0 = __shfl_sync(0xFFFFFFFFu, t, 0);
+    const int t1 = two ? __shfl_sync(0xFFFFFFFFu, t, 1) : 0;
     const float z0 = row_dot_bf16_hs<NCH>(e, hs, d);
     unsigned long long pk = pack_best(z0, t0);
     best = pk > best ? pk : best;

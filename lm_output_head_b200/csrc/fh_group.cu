@@ -11,8 +11,10 @@
 // (mma.sync m16n8k16, bf16 in, fp32 accumulate: 16 token slots x 8 hidden
 // rows per tile, K = d). A cluster's tile is a handful of hidden rows, far
 // below the 64- or 128-row minimum of a tcgen05 MMA, so the warp-level MMA
-// keeps the work exact instead of padding it 4-8x. Fragments are loaded
-// straight from global memory (token rows once, hidden rows from L2).
+// keeps the work exact instead of padding it 4-8x. Token rows are read once,
+// from the head's cluster-major copy (a cluster's 16 rows are one contiguous
+// block); hidden rows come from L2; both are staged through a per-warp
+// cp.async ring in shared memory.
 // Outputs: the packed (logit, token) maximum of every row (64-bit
 // atomicMax), and, when sampling, every logit at its canonical position in
 // the row (rank of k among the row's ascending clusters, then slot).
@@ -112,12 +114,6 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4],
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Eight consecutive bf16 of a row from element k (k % 8 == 0, d % 8 == 0: a
-// chunk never straddles d); zeros past the row's end.
-__device__ __forceinline__ uint4 ld_chunk(const uint16_t* p, int k, int d) {
-  return k < d ? __ldg(reinterpret_cast<const uint4*>(p + k)) : make_uint4(0, 0, 0, 0);
-}
-
 // Position of cluster k among the row's ascending clusters (binary search).
 __device__ __forceinline__ int rank_in_row(const int32_t* sel, int p, int k) {
   int lo = 0, hi = p - 1;
@@ -129,12 +125,39 @@ __device__ __forceinline__ int rank_in_row(const int32_t* sel, int p, int k) {
   return lo;
 }
 
-constexpr int kChunks = 4;  // 8-row chunks of R_k per pass (32 hidden rows)
+constexpr int kChunks = 4;          // 8-row chunks of R_k per pass (32 hidden rows)
+constexpr int kRing = 4;            // cp.async stages per warp
+constexpr int kSlice = 32;          // K elements per stage: 64 bytes of every row
+constexpr int kStageBytes = (16 + 8 * kChunks) * kSlice * 2;  // 16 token rows + 32 hidden rows: 3 KB
+constexpr int kGroupWarps = 16;     // warps per CTA (one CTA per SM)
+constexpr int kGroupSmem = kGroupWarps * kRing * kStageBytes;  // 192 KB
 
-__global__ void __launch_bounds__(256) group_kernel(const GroupParams P) {
-  const int lane = threadIdx.x & 31;
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// One warp per distinct cluster (dynamic). For each pass over up to 32 of the
+// hidden rows that chose it, K is streamed in slices of 32 elements through a
+// per-warp ring of kRing shared-memory stages filled with 16-byte cp.async
+// copies (the cluster's 16 token rows, contiguous in the cluster-major copy,
+// and the pass's hidden rows, zero-filled past the row list): every warp keeps
+// several KB in flight without holding them in registers. Fragments are read
+// back with 16-byte shared loads (conflict-free: 64-byte rows) in the permuted
+// K order described below and fed to mma.sync m16n8k16.
+__global__ void __launch_bounds__(kGroupWarps * 32, 1) group_kernel(const GroupParams P) {
+  extern __shared__ __align__(128) uint8_t gsm[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;  // mma fragment coordinates
   const int d = P.d, b = P.b;
+  const int nsl = (d + kSlice - 1) / kSlice;
+  const uint32_t ring = static_cast<uint32_t>(__cvta_generic_to_shared(gsm)) +
+                        static_cast<uint32_t>(warp * kRing * kStageBytes);
   const uint32_t nu = *P.union_count;
   for (;;) {
     uint32_t ui = 0;
@@ -143,45 +166,67 @@ __global__ void __launch_bounds__(256) group_kernel(const GroupParams P) {
     if (ui >= nu) break;
     const int k = P.ulist[ui];
     const int r0 = static_cast<int>(P.off[k]), r1 = static_cast<int>(P.off[k + 1]);
-    // token slots g and g + 8 of cluster k (b == 16: one m16 tile)
+    const uint16_t* ek = P.Ecm + static_cast<size_t>(k) * b * d;  // the cluster's 16 rows, contiguous
     const int tok_a = __ldg(P.C2T + static_cast<size_t>(k) * b + g);
     const int tok_b = __ldg(P.C2T + static_cast<size_t>(k) * b + g + 8);
-    const uint16_t* ea = P.E + static_cast<size_t>(tok_a) * d;
-    const uint16_t* eb = P.E + static_cast<size_t>(tok_b) * d;
     for (int rb = r0; rb < r1; rb += 8 * kChunks) {
-      const int nch = min(kChunks, (r1 - rb + 7) / 8);
-      // hidden row of fragment column g in each chunk (rows past the cluster's list repeat a valid row)
-      const uint16_t* hrow[kChunks];
+      const int nrows = min(8 * kChunks, r1 - rb);
+      const int nch = (nrows + 7) / 8;
+      const int hl = P.rows_of[rb + min(lane, nrows - 1)];  // hidden row of pass row `lane`
+      auto issue = [&](int sl) {
+        const uint32_t st = ring + static_cast<uint32_t>((sl % kRing) * kStageBytes);
+        const int e0 = sl * kSlice;
 #pragma unroll
-      for (int ch = 0; ch < kChunks; ++ch) {
-        const int idx = min(rb + ch * 8 + g, r1 - 1);
-        hrow[ch] = P.H + static_cast<size_t>(P.rows_of[idx]) * d;
+        for (int i = 0; i < 2; ++i) {  // token rows: 16 rows x 4 chunks
+          const int c = lane + 32 * i, row = c >> 2, ch = c & 3;
+          const bool ok = e0 + 8 * ch < d;
+          cp_async16(st + static_cast<uint32_t>(row * 64 + ch * 16), ek + static_cast<size_t>(row) * d + (ok ? e0 + 8 * ch : 0), ok);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {  // hidden rows: 32 rows x 4 chunks
+          const int c = lane + 32 * i, row = c >> 2, ch = c & 3;
+          const int hr = __shfl_sync(0xFFFFFFFFu, hl, row);
+          const bool ok = row < nrows && e0 + 8 * ch < d;
+          cp_async16(st + static_cast<uint32_t>((16 + row) * 64 + ch * 16),
+                     P.H + static_cast<size_t>(hr) * d + (ok ? e0 + 8 * ch : 0), ok);
+        }
+        cp_async_commit();
+      };
+#pragma unroll
+      for (int sl = 0; sl < kRing - 1; ++sl) {
+        if (sl < nsl) issue(sl);
+        else cp_async_commit();  // empty group: keeps the group count uniform
       }
       float acc[kChunks][4];
 #pragma unroll
       for (int ch = 0; ch < kChunks; ++ch) acc[ch][0] = acc[ch][1] = acc[ch][2] = acc[ch][3] = 0.f;
-      // The dot product over K is order-free, so two MMA K-steps take 32
-      // elements in a lane-friendly order: lane t of a fragment row loads the
-      // 8 contiguous elements [k0 + 8t, k0 + 8t + 8); the first K-step uses
-      // elements 8t..8t+3 (as its columns 2t, 2t+1, 2t+8, 2t+9), the second
-      // 8t+4..8t+7. A and B use the same order, so the sums are unchanged.
-#pragma unroll 2
-      for (int k0 = 0; k0 < d; k0 += 32) {
-        const int kk = k0 + 8 * t;
-        const uint4 xa = ld_chunk(ea, kk, d), xb = ld_chunk(eb, kk, d);
-        uint4 xh[kChunks];
-#pragma unroll
-        for (int ch = 0; ch < kChunks; ++ch) xh[ch] = ch < nch ? ld_chunk(hrow[ch], kk, d) : make_uint4(0, 0, 0, 0);
+      for (int sl = 0; sl < nsl; ++sl) {
+        cp_async_wait<kRing - 2>();
+        __syncwarp();
+        const uint32_t st = ring + static_cast<uint32_t>((sl % kRing) * kStageBytes);
+        // The dot product over K is order-free, so the slice's 32 elements feed
+        // two MMA K-steps in a lane-friendly order: lane t of a fragment row
+        // takes the 8 contiguous elements 8t..8t+7 of the slice; the first
+        // K-step uses 8t..8t+3 (as its columns 2t, 2t+1, 2t+8, 2t+9), the second
+        // 8t+4..8t+7. A and B use the same order, so the sums are unchanged.
+        const uint4 xa = lds128(st + static_cast<uint32_t>(g * 64 + t * 16));
+        const uint4 xb = lds128(st + static_cast<uint32_t>((g + 8) * 64 + t * 16));
         const uint32_t a0[4] = {xa.x, xb.x, xa.y, xb.y};
         const uint32_t a1[4] = {xa.z, xb.z, xa.w, xb.w};
 #pragma unroll
         for (int ch = 0; ch < kChunks; ++ch) {
           if (ch < nch) {
-            mma_16816(acc[ch], a0, xh[ch].x, xh[ch].y);
-            mma_16816(acc[ch], a1, xh[ch].z, xh[ch].w);
+            const uint4 xh = lds128(st + static_cast<uint32_t>((16 + 8 * ch + g) * 64 + t * 16));
+            mma_16816(acc[ch], a0, xh.x, xh.y);
+            mma_16816(acc[ch], a1, xh.z, xh.w);
           }
         }
+        __syncwarp();  // the stage is read before it is refilled
+        if (sl + kRing - 1 < nsl) issue(sl + kRing - 1);
+        else cp_async_commit();
       }
+      cp_async_wait<0>();
+      __syncwarp();
       // acc[ch]: (slot g, col 2t), (slot g, col 2t+1), (slot g+8, col 2t), (slot g+8, col 2t+1)
 #pragma unroll
       for (int ch = 0; ch < kChunks; ++ch) {
@@ -214,6 +259,10 @@ __global__ void __launch_bounds__(256) group_kernel(const GroupParams P) {
 
 }  // namespace
 
+cudaError_t set_attrs_group() {
+  return cudaFuncSetAttribute(group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGroupSmem);
+}
+
 cudaError_t launch_group(const GroupParams& P, int num_sms, cudaStream_t st) {
   const long long n = static_cast<long long>(P.B) * P.p;
   const int gsz = static_cast<int>(std::min<long long>((n + 255) / 256, 4LL * num_sms));
@@ -222,7 +271,7 @@ cudaError_t launch_group(const GroupParams& P, int num_sms, cudaStream_t st) {
   csr_count_kernel<<<gsz, 256, 0, st>>>(P);
   csr_scan_kernel<<<1, kThreads, 0, st>>>(P);
   csr_fill_kernel<<<gsz, 256, 0, st>>>(P);
-  group_kernel<<<num_sms * 8, 256, 0, st>>>(P);
+  group_kernel<<<num_sms, kGroupWarps * 32, kGroupSmem, st>>>(P);
   return cudaGetLastError();
 }
 

@@ -33,6 +33,7 @@ struct SyncWords {
 
 struct B1Params {
   const uint16_t* E;
+  const uint16_t* Ecm;    // cluster-major token rows: row k*b + j = E[C2T[k][j]]
   const uint8_t* Crows;   // bf16 rows (d*2 bytes) or packed INT4 rows (crow_bytes)
   const int32_t* C2T;
   const uint16_t* hidden;
@@ -143,7 +144,7 @@ struct GemmParams {
 struct GroupParams {
   const int32_t* sel;       // [B, p] chosen clusters per row, ascending
   const int32_t* C2T;       // [c, b]
-  const uint16_t* E;        // [v, d]
+  const uint16_t* Ecm;      // [v, d] cluster-major token rows: row k*b + j = E[C2T[k][j]]
   const uint16_t* H;        // [B, d]
   uint32_t* cnt;            // [c] workspace: rows per cluster
   uint32_t* cur;            // [c] workspace: fill cursors
@@ -184,12 +185,16 @@ cudaError_t launch_epilogue(const EpilogueParams& P, int B, cudaStream_t st);
 cudaError_t launch_dense(const DenseParams& P, int grid, size_t smem, int nch, cudaStream_t st);
 cudaError_t launch_c2t_check(const C2TCheckParams& P, cudaStream_t st);
 cudaError_t launch_repack_int4(const RepackParams& P, cudaStream_t st);
+// Cluster-major copy of the token rows: out[k*b + j] = E[C2T[k][j]].
+cudaError_t launch_gather_cluster_major(const uint16_t* E, const int32_t* C2T, uint16_t* out, int v, int d,
+                                        cudaStream_t st);
 // tcgen05 GEMM (B >= 64): streamed rows bf16 [rows, d] through TMA, or packed INT4 rows; H bf16 [nb, d].
 cudaError_t launch_gemm(const GemmParams& P, const void* rows_bf16, const void* H, int num_sms, cudaStream_t st);
 cudaError_t set_attrs_gemm();
 // De-duplicated candidate logits of a batch (b == 16): CSR of the selections by cluster, then one
 // pass per distinct cluster on the tensor cores.
 cudaError_t launch_group(const GroupParams& P, int num_sms, cudaStream_t st);
+cudaError_t set_attrs_group();
 
 // Opt-in shared memory attribute for every instantiation (called once per device).
 cudaError_t set_kernel_attributes(int max_smem);

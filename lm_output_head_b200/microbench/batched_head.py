@@ -1,11 +1,15 @@
-"""Timing of the batched path on the Gemma-3-shaped head (v 262144, d 1152,
-c 16384 balanced clusters of 16, p 1024, INT4 centroids, bf16 tokens, B 256
-planted hidden states): the tcgen05 centroid GEMM, the tcgen05 dense head
-(fused argmax), and the whole batched decode (GEMM keys, per-row top-p,
-de-duplicated candidate logits, argmax). CUDA events on the launching
-stream, median of the timed repeats; prints one JSON line.
+"""Timing of the batched path (B > 1).
 
-    python -m lm_output_head_b200.microbench.batched_head [--repeats N]
+For each requested head shape and batch: the whole batched decode (centroid
+keys -- tcgen05 GEMM at B >= 64, CUDA cores below --, per-row top-p,
+de-duplicated candidate logits, argmax or inverse-CDF draw), its algorithmic
+bytes (centroid bytes once + every distinct chosen cluster's token rows and
+C2T row once + hidden rows + uniforms + outputs) and achieved GB/s; at
+B >= 64 also the tcgen05 centroid GEMM and the tcgen05 dense head (fused
+argmax) with their TFLOP/s. CUDA events on the launching stream, median of the
+timed repeats; one JSON line per case.
+
+    python -m lm_output_head_b200.microbench.batched_head [--repeats N] [--cases 4:256,3:32,2:16,2:4]
 """
 from __future__ import annotations
 
@@ -20,30 +24,47 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--repeats", type=int, default=20)
-    ap.add_argument("--batch", type=int, default=256)
-    args = ap.parse_args()
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def run_case(cfg_id, B, repeats):
+    import numpy as np
     import torch
     import synth
     import lm_output_head_b200 as fh
-    cfg, head, hid, _ = synth.make_config(4, n_states=args.batch)
+    cfg, head, hid, uni = synth.make_config(cfg_id, n_states=max(B, 64))
     dev = "cuda"
     E = fh.bf16_from_bits(head.E, dev)
     C2T = torch.from_numpy(head.C2T).to(dev)
-    Cq = torch.from_numpy(head.C_q).to(dev)
-    Cs = fh.bf16_from_bits(head.C_scales, dev)
-    dh = fh.FlashHead(E, C2T, C_q=Cq, C_scales=Cs, max_batch=args.batch, max_probes=cfg.p)
-    H = fh.bf16_from_bits(hid.H[:args.batch], dev)
-    B = args.batch
+    if head.C_q is not None:
+        dh = fh.FlashHead(E, C2T, C_q=torch.from_numpy(head.C_q).to(dev),
+                          C_scales=fh.bf16_from_bits(head.C_scales, dev), max_batch=B, max_probes=cfg.p)
+        cbytes = head.C_q.nbytes + head.C_scales.nbytes
+    else:
+        dh = fh.FlashHead(E, C2T, C=fh.bf16_from_bits(head.C, dev), max_batch=B, max_probes=cfg.p)
+        cbytes = head.C.nbytes
+    H = fh.bf16_from_bits(hid.H[:B], dev)
+    gumbel = cfg.mode == "gumbel"
+    kw = {}
+    ubytes = 0
+    if gumbel:
+        rng = np.random.default_rng(5)
+        kw = dict(mode="gumbel", T=cfg.temperature,
+                  u_clusters=torch.from_numpy(rng.random((B, cfg.c), dtype=np.float32)).to(dev),
+                  u_token=torch.from_numpy(rng.random(B, dtype=np.float32)).to(dev))
+        ubytes = B * cfg.c * 4 + B * 4
 
     def timeit(fn):
         for _ in range(3):
             fn()
         torch.cuda.synchronize()
         ts = []
-        for _ in range(args.repeats):
+        for _ in range(repeats):
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record()
@@ -53,24 +74,40 @@ def main():
             ts.append(a.elapsed_time(b) * 1e3)
         return statistics.median(ts)
 
-    scores = torch.empty((B, cfg.c), dtype=torch.float32, device=dev)
-    am = torch.empty(B, dtype=torch.int32, device=dev)
     tok = torch.empty(B, dtype=torch.int32, device=dev)
-    t_c = timeit(lambda: dh.centroid_scores(H, out=scores))
-    t_d = timeit(lambda: dh.dense_head(H, out_argmax=am))
-    t_x = timeit(lambda: dh.decode(H, cfg.p, out_tokens=tok))
+    t_x = timeit(lambda: dh.decode(H, cfg.p, out_tokens=tok, **kw))
     union = dh.query(1)
-    status = dh.device_status()
-    fl_c = 2.0 * B * cfg.c * cfg.d
-    fl_d = 2.0 * B * cfg.v * cfg.d
-    print(json.dumps({
-        "workload": f"Gemma-3-shaped head v{cfg.v} d{cfg.d} c{cfg.c} b{cfg.b} p{cfg.p} INT4 centroids, B={B}",
-        "centroid_gemm_us": round(t_c, 2), "centroid_gemm_tflops": round(fl_c / t_c / 1e6, 1),
-        "dense_gemm_us": round(t_d, 2), "dense_gemm_tflops": round(fl_d / t_d / 1e6, 1),
-        "decode_us": round(t_x, 2), "decode_tokens_per_s": round(B / t_x * 1e6, 1),
-        "union_clusters": union, "union_of_possible": round(union / min(cfg.c, B * cfg.p), 4),
-        "device_status": status}), flush=True)
+    abytes = cbytes + union * (cfg.b * cfg.d * 2 + cfg.b * 4) + B * cfg.d * 2 + ubytes + B * 4
+    peak, kind = measured_hbm_peak()
+    rec = {"workload": f"config {cfg_id}: v{cfg.v} d{cfg.d} c{cfg.c} b{cfg.b} p{cfg.p} "
+                       f"{'INT4' if head.C_q is not None else 'bf16'} centroids, B={B}, {cfg.mode}",
+           "decode_us": round(t_x, 2), "decode_tokens_per_s": round(B / t_x * 1e6, 1),
+           "union_clusters": union, "union_of_possible": round(union / min(cfg.c, B * cfg.p), 4),
+           "algorithmic_bytes": int(abytes), "achieved_GBps": round(abytes / t_x / 1e3, 1),
+           "frac_of_hbm_peak": round(abytes / t_x / 1e3 / peak, 4), "peak_kind": kind}
+    if B >= 64:
+        scores = torch.empty((B, cfg.c), dtype=torch.float32, device=dev)
+        am = torch.empty(B, dtype=torch.int32, device=dev)
+        t_c = timeit(lambda: dh.centroid_scores(H, out=scores))
+        t_d = timeit(lambda: dh.dense_head(H, out_argmax=am))
+        rec.update({"centroid_gemm_us": round(t_c, 2),
+                    "centroid_gemm_tflops": round(2.0 * B * cfg.c * cfg.d / t_c / 1e6, 1),
+                    "dense_gemm_us": round(t_d, 2),
+                    "dense_gemm_tflops": round(2.0 * B * cfg.v * cfg.d / t_d / 1e6, 1)})
+    rec["device_status"] = dh.device_status()
     dh.close()
+    print(json.dumps(rec), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--repeats", type=int, default=20)
+    ap.add_argument("--cases", default="4:256,3:32,2:16,2:4",
+                    help="comma-separated config:batch pairs")
+    args = ap.parse_args()
+    for case in args.cases.split(","):
+        cfg_id, B = (int(x) for x in case.split(":"))
+        run_case(cfg_id, B, args.repeats)
 
 
 if __name__ == "__main__":
