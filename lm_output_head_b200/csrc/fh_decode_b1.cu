@@ -143,12 +143,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
                wbar);
     }
   }
-  constexpr int NQ = (NCH + 1) / 2;
   uint4 w[NCH];
-  uint2 q[NQ];
-  uint32_t sc[NQ];
+  uint32_t q[NCH], sc[NCH];
   if (n1 > 0) {
-    if constexpr (INT4) row_load_int4<NQ>(P.Crows + static_cast<size_t>(cw) * P.crow_bytes, d, q, sc);
+    if constexpr (INT4) row_load_int4<NCH>(P.Crows + static_cast<size_t>(cw) * P.crow_bytes, d, q, sc);
     else row_load_bf16<NCH>(reinterpret_cast<const uint16_t*>(P.Crows + static_cast<size_t>(cw) * P.crow_bytes), d, w);
   }
   float ureg = 0.f;  // lane j holds u of item j
@@ -204,11 +202,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     if (i == 1) {  // the row that landed in the slot
       if (!mbar_wait_bounded(wbar, wphase, kWaitBudget) && lane == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
       wphase ^= 1u;
-      if constexpr (INT4) s = srow_dot_int4_hs<NQ>(slot, hs, d);
+      if constexpr (INT4) s = srow_dot_int4_hs<NCH>(slot, hs, d);
       else s = srow_dot_bf16_hs<NCH>(slot, hs, d);
     } else if constexpr (INT4) {
-      if (i > 0) row_load_int4<NQ>(P.Crows + static_cast<size_t>(k) * P.crow_bytes, d, q, sc);
-      s = row_dot_int4_hs<NQ>(q, sc, hs, d);
+      if (i > 0) row_load_int4<NCH>(P.Crows + static_cast<size_t>(k) * P.crow_bytes, d, q, sc);
+      s = row_dot_int4_hs<NCH>(q, sc, hs, d);
     } else {
       if (i > 0) row_load_bf16<NCH>(reinterpret_cast<const uint16_t*>(P.Crows + static_cast<size_t>(k) * P.crow_bytes), d, w);
       s = row_dot_bf16_hs<NCH>(w, hs, d);

@@ -740,12 +740,6 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   return v;
 }
 
-__device__ __forceinline__ uint2 ldg_stream64(const void* p) {
-  uint2 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-  return v;
-}
-
 // bf16 row: chunk m of lane l covers elements (l + 32 m) * 8 .. + 8.
 template <int NCH>
 __device__ __forceinline__ void row_load_bf16(const uint16_t* row, int d, uint4 (&w)[NCH]) {
@@ -780,39 +774,52 @@ __device__ __forceinline__ float row_dot_bf16_hs(const uint4 (&w)[NCH], const fl
   return warp_sum(acc);
 }
 
-// Packed INT4 row ([d/2 code bytes][d/16 scale bytes]): half-group g = l + 32 m
-// (16 codes, 8 bytes) and the bf16 scale of its group g/2.
-template <int NQ>
-__device__ __forceinline__ void row_load_int4(const uint8_t* row, int d, uint2 (&q)[NQ], uint32_t (&sc)[NQ]) {
+// Packed INT4 row ([d/2 code bytes][d/16 scale bytes]) in the same chunk
+// layout as a bf16 row: for chunk m, lane l holds the 4 code bytes of
+// elements (l + 32 m) * 8 .. + 8 (one 32-bit word) and the bf16 scale of their
+// group of 32, so the codes load coalesced and h is read as two float4 per
+// chunk at a 32-byte lane stride (no shared-memory bank conflicts).
+__device__ __forceinline__ uint32_t ldg_stream32(const void* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
+template <int NCH>
+__device__ __forceinline__ void row_load_int4(const uint8_t* row, int d, uint32_t (&q)[NCH], uint32_t (&sc)[NCH]) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int m = 0; m < NQ; ++m) {
-    const int g = lane + 32 * m;
-    if (g * 16 < d) {
-      q[m] = ldg_stream64(row + 8 * g);
-      sc[m] = __ldg(reinterpret_cast<const unsigned short*>(row + d / 2) + (g >> 1));
+  for (int m = 0; m < NCH; ++m) {
+    const int e = (lane + 32 * m) * 8;
+    if (e < d) {
+      q[m] = ldg_stream32(row + e / 2);
+      sc[m] = __ldg(reinterpret_cast<const unsigned short*>(row + d / 2) + (e >> 5));
     } else {
-      q[m] = make_uint2(0u, 0u);
+      q[m] = 0u;
       sc[m] = 0u;
     }
   }
 }
 
-template <int NQ>
-__device__ __forceinline__ float row_dot_int4_hs(const uint2 (&q)[NQ], const uint32_t (&sc)[NQ], const float* hs,
+template <int NCH>
+__device__ __forceinline__ float row_dot_int4_hs(const uint32_t (&q)[NCH], const uint32_t (&sc)[NCH], const float* hs,
                                                  int d) {
   const int lane = threadIdx.x & 31;
   float acc = 0.f;
 #pragma unroll
-  for (int m = 0; m < NQ; ++m) {
-    const int g = lane + 32 * m;
-    if (g * 16 < d) {
-      const float* h = hs + 16 * g;
-      float part = 0.f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) part = fmaf(nib(q[m].x, i), h[i], part);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) part = fmaf(nib(q[m].y, i), h[8 + i], part);
+  for (int m = 0; m < NCH; ++m) {
+    const int e = (lane + 32 * m) * 8;
+    if (e < d) {
+      const float4 a = *reinterpret_cast<const float4*>(hs + e);
+      const float4 b = *reinterpret_cast<const float4*>(hs + e + 4);
+      float part = nib(q[m], 0) * a.x;
+      part = fmaf(nib(q[m], 1), a.y, part);
+      part = fmaf(nib(q[m], 2), a.z, part);
+      part = fmaf(nib(q[m], 3), a.w, part);
+      part = fmaf(nib(q[m], 4), b.x, part);
+      part = fmaf(nib(q[m], 5), b.y, part);
+      part = fmaf(nib(q[m], 6), b.z, part);
+      part = fmaf(nib(q[m], 7), b.w, part);
       acc = fmaf(__uint_as_float(sc[m] << 16), part, acc);
     }
   }
@@ -844,23 +851,24 @@ __device__ __forceinline__ float srow_dot_bf16_hs(uint32_t row, const float* hs,
   return warp_sum(acc);
 }
 
-template <int NQ>
+template <int NCH>
 __device__ __forceinline__ float srow_dot_int4_hs(uint32_t row, const float* hs, int d) {
-  uint2 q[NQ];
-  uint32_t sc[NQ];
+  uint32_t q[NCH], sc[NCH];
   const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int m = 0; m < NQ; ++m) {
-    const int g = lane + 32 * m;
-    if (g * 16 < d) {
-      q[m] = lds64(row + 8u * g);
-      sc[m] = lds16(row + d / 2 + 2u * (g >> 1));
+  for (int m = 0; m < NCH; ++m) {
+    const int e = (lane + 32 * m) * 8;
+    if (e < d) {
+      uint32_t w;
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w) : "r"(row + static_cast<uint32_t>(e / 2)));
+      q[m] = w;
+      sc[m] = lds16(row + static_cast<uint32_t>(d / 2 + 2 * (e >> 5)));
     } else {
-      q[m] = make_uint2(0u, 0u);
+      q[m] = 0u;
       sc[m] = 0u;
     }
   }
-  return row_dot_int4_hs<NQ>(q, sc, hs, d);
+  return row_dot_int4_hs<NCH>(q, sc, hs, d);
 }
 
 // Stage a bf16 vector of d elements (d % 8 == 0) into shared memory as fp32.

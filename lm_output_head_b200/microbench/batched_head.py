@@ -1,4 +1,5 @@
-"""Timing of the batched path (B > 1).
+"""Timing of the batched path (B > 1), and of the fused kernel at B = 1 for
+the INT4-centroid head.
 
 For each requested head shape and batch: the whole batched decode (centroid
 keys -- tcgen05 GEMM at B >= 64, CUDA cores below --, per-row top-p,
@@ -9,7 +10,7 @@ B >= 64 also the tcgen05 centroid GEMM and the tcgen05 dense head (fused
 argmax) with their TFLOP/s. CUDA events on the launching stream, median of the
 timed repeats; one JSON line per case.
 
-    python -m lm_output_head_b200.microbench.batched_head [--repeats N] [--cases 4:256,3:32,2:16,2:4]
+    python -m lm_output_head_b200.microbench.batched_head [--repeats N] [--cases 4:256,3:32,2:16,2:4,2:1]
 """
 from __future__ import annotations
 
@@ -99,15 +100,81 @@ def run_case(cfg_id, B, repeats):
     print(json.dumps(rec), flush=True)
 
 
+def run_b1(cfg_id, steps):
+    """One hidden state per step through the fused kernel, steps issued back to
+    back and rotated over enough head copies that every step reads its
+    centroid and token rows from HBM (the protocol of bench.py)."""
+    import ctypes
+    import torch
+    import synth
+    import lm_output_head_b200 as fh
+    cfg, head, hid, _ = synth.make_config(cfg_id)
+    dev = torch.device("cuda", 0)
+    int4 = head.C_q is not None
+    cbytes = head.C_q.nbytes + head.C_scales.nbytes if int4 else head.C.nbytes
+    abytes = cbytes + cfg.p * cfg.b * cfg.d * 2 + cfg.p * cfg.b * 4 + cfg.d * 2 + 4
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    n_copies = max(3, -(-4 * l2 // abytes) + 1)
+    E0 = fh.bf16_from_bits(head.E, dev)
+    T0 = torch.from_numpy(head.C2T).to(dev)
+    heads = []
+    for i in range(n_copies):
+        E, T = (E0, T0) if i == 0 else (E0.clone(), T0.clone())
+        if int4:
+            heads.append(fh.FlashHead(E, T, C_q=torch.from_numpy(head.C_q).to(dev),
+                                      C_scales=fh.bf16_from_bits(head.C_scales, dev), max_batch=1,
+                                      max_probes=cfg.p))
+        else:
+            heads.append(fh.FlashHead(E, T, C=fh.bf16_from_bits(head.C, dev), max_batch=1, max_probes=cfg.p))
+    Hd = fh.bf16_from_bits(hid.H, dev)
+    out = torch.empty(1, dtype=torch.int32, device=dev)
+    lib = heads[0]._lib
+    sptr = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    optr = ctypes.c_void_p(out.data_ptr())
+    hptrs = [ctypes.c_void_p(Hd[i].data_ptr()) for i in range(Hd.shape[0])]
+    handles = [h._h for h in heads]
+
+    def step(i):
+        st = lib.fh_decode(handles[i % n_copies], hptrs[i % len(hptrs)], 1, cfg.p, 0, 1.0, None, None, optr,
+                           None, None, sptr)
+        if st != 0:
+            raise RuntimeError(f"fh_decode returned {st}")
+    for i in range(20):
+        step(i)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        step(20 + i)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    us = e0.elapsed_time(e1) * 1e3 / steps
+    peak, kind = measured_hbm_peak()
+    status = max(h.device_status() for h in heads)
+    for h in heads:
+        h.close()
+    print(json.dumps({
+        "workload": f"config {cfg_id}: v{cfg.v} d{cfg.d} c{cfg.c} b{cfg.b} p{cfg.p} "
+                    f"{'INT4' if int4 else 'bf16'} centroids, B=1 greedy, fused kernel",
+        "us_per_token": round(us, 3), "tokens_per_s": round(1e6 / us, 1), "algorithmic_bytes": int(abytes),
+        "achieved_GBps": round(abytes / us / 1e3, 1), "frac_of_hbm_peak": round(abytes / us / 1e3 / peak, 4),
+        "peak_kind": kind, "head_copies": n_copies, "device_status": status}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--repeats", type=int, default=20)
-    ap.add_argument("--cases", default="4:256,3:32,2:16,2:4",
-                    help="comma-separated config:batch pairs")
+    ap.add_argument("--cases", default="4:256,3:32,2:16,2:4,2:1",
+                    help="comma-separated config:batch pairs (batch 1: the fused kernel, back to back)")
+    ap.add_argument("--b1-steps", type=int, default=1000)
     args = ap.parse_args()
     for case in args.cases.split(","):
         cfg_id, B = (int(x) for x in case.split(":"))
-        run_case(cfg_id, B, args.repeats)
+        if B == 1:
+            run_b1(cfg_id, args.b1_steps)
+        else:
+            run_case(cfg_id, B, args.repeats)
 
 
 if __name__ == "__main__":
