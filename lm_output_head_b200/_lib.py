@@ -37,6 +37,10 @@ EXPORTED = (
     "fh_create", "fh_destroy", "fh_centroid_scores", "fh_select_clusters",
     "fh_candidate_logits", "fh_decode", "fh_dense_head", "fh_get_device_status",
     "fh_status_string", "fh_set_spin_budget", "fh_query", "fh_dense_head_noalloc",
+    # include/fh_cluster.h
+    "fh_cluster_create", "fh_cluster_destroy", "fh_cluster_normalize", "fh_cluster_seed",
+    "fh_cluster_gather", "fh_cluster_similarities", "fh_cluster_assign", "fh_cluster_update",
+    "fh_cluster_build", "fh_cluster_get_device_status",
 )
 
 FH_NOALLOC_MAX_ROWS = 64
@@ -94,6 +98,22 @@ def load() -> ctypes.CDLL:
     lib.fh_set_spin_budget.restype = ctypes.c_int
     lib.fh_query.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_int64)]
     lib.fh_query.restype = ctypes.c_int
+    pi32 = ctypes.POINTER(ctypes.c_int32)
+    lib.fh_cluster_create.argtypes = [i32, i32, i32, vp, ctypes.POINTER(vp)]
+    lib.fh_cluster_destroy.argtypes = [vp]
+    lib.fh_cluster_destroy.restype = None
+    lib.fh_cluster_normalize.argtypes = [vp, vp, vp, vp]
+    lib.fh_cluster_seed.argtypes = [vp, vp, vp, vp, vp]
+    lib.fh_cluster_gather.argtypes = [vp, vp, vp, vp, vp]
+    lib.fh_cluster_similarities.argtypes = [vp, vp, vp, vp, vp]
+    lib.fh_cluster_assign.argtypes = [vp, vp, vp, vp, pi32, vp]
+    lib.fh_cluster_update.argtypes = [vp, vp, vp, vp, vp]
+    lib.fh_cluster_build.argtypes = [vp, vp, vp, vp, i32, vp, vp, pi32, vp]
+    lib.fh_cluster_get_device_status.argtypes = [vp, vp]
+    for name in ("fh_cluster_create", "fh_cluster_normalize", "fh_cluster_seed", "fh_cluster_gather",
+                 "fh_cluster_similarities", "fh_cluster_assign", "fh_cluster_update", "fh_cluster_build",
+                 "fh_cluster_get_device_status"):
+        getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
 

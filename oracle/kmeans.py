@@ -84,6 +84,17 @@ def kmeanspp_seeds(En: np.ndarray, c: int, u: np.ndarray) -> np.ndarray:
     return chosen
 
 
+def seed_weights(En: np.ndarray, chosen) -> np.ndarray:
+    """k-means++ weights ``D(x)^2``: squared Euclidean distance of every row to the
+    nearest of the rows ``chosen`` (section 2.1, initialisation)."""
+    En = np.asarray(En, dtype=np.float64)
+    d2 = np.full(En.shape[0], np.inf)
+    for i in chosen:
+        diff = En - En[int(i)]
+        d2 = np.minimum(d2, np.sum(diff * diff, axis=1))
+    return d2
+
+
 def balanced_assign(S: np.ndarray, b: int) -> np.ndarray:
     """Cluster of every token under the balance rule, from similarities ``S [v, c]`` (section 1.2.1).
 

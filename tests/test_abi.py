@@ -1,4 +1,4 @@
-"""The C-ABI library loads and exports every entry point include/fh.h declares (no GPU needed)."""
+"""The C-ABI library loads and exports every entry point the headers under include/ declare (no GPU needed)."""
 import ctypes
 import os
 import re
@@ -9,7 +9,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _declared():
-    src = open(os.path.join(ROOT, "include", "fh.h")).read()
+    inc = os.path.join(ROOT, "include")
+    src = "".join(open(os.path.join(inc, f)).read() for f in sorted(os.listdir(inc)) if f.endswith(".h"))
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     names = set(re.findall(r"\b(fh_[a-z_0-9]+)\s*\(", src))
     return sorted(names)

@@ -52,6 +52,22 @@ def test_golden_kmeanspp_edges():
     assert seeds.tolist() == g["seeds"]
 
 
+def test_seed_weights_match_the_worked_seeding():
+    g = _fixture()["kmeanspp"]
+    En = np.array(g["points"], dtype=np.float64)
+    assert kmeans.seed_weights(En, [0]).tolist() == [0.0, 2.0, 4.0, 2.0]
+    assert kmeans.seed_weights(En, [0, 2]).tolist() == [0.0, 2.0, 0.0, 2.0]
+    # the seeding's own draws follow the inverse CDF of these weights
+    rng = np.random.default_rng(4)
+    X = kmeans.normalize_rows(rng.standard_normal((40, 5)))
+    u = rng.uniform(size=8)
+    seeds = kmeans.kmeanspp_seeds(X, 8, u)
+    for j in range(1, 8):
+        cdf = np.cumsum(kmeans.seed_weights(X, seeds[:j]))
+        t = seeds[j]
+        assert cdf[t] > u[j] * cdf[-1] >= (cdf[t - 1] if t > 0 else 0.0)
+
+
 def test_golden_balanced_steps():
     g = _fixture()["balanced"]
     E = np.array([_unit(a) for a in g["angles_deg"]])
@@ -236,3 +252,54 @@ def test_stops_at_the_first_repeated_assignment(seed):
 def test_builder_rejects_unbalanced_sizes():
     with pytest.raises(ValueError):
         kmeans.build_clusters(np.ones((10, 4)), 3, init_ids=np.array([0, 1, 2]))
+
+
+# ---------------------------------------------------------------------------
+# the parallel round structure the assignment kernels use
+# ---------------------------------------------------------------------------
+def _deferred_acceptance(S, b):
+    """Rounds of proposals: every unassigned token proposes to its best cluster
+    (similarity desc, cluster asc) among those whose b-th held pair it beats at
+    the start of the round (or that still have room); every cluster keeps the
+    best b of its held tokens and its proposers (similarity desc, token asc)."""
+    v, c = S.shape
+    held = [[] for _ in range(c)]          # (s, t), best first
+    assign = np.full(v, -1)
+    rounds = 0
+    while np.any(assign < 0):
+        rounds += 1
+        props = [[] for _ in range(c)]
+        for t in np.flatnonzero(assign < 0):
+            best = None
+            for k in range(c):
+                h = held[k]
+                if len(h) == b:
+                    ws, wt = h[-1]
+                    if not (S[t, k] > ws or (S[t, k] == ws and t < wt)):
+                        continue
+                if best is None or S[t, k] > S[t, best]:
+                    best = k
+            props[best].append((S[t, best], t))
+        for k in range(c):
+            if not props[k]:
+                continue
+            cand = sorted(held[k] + props[k], key=lambda e: (-e[0], e[1]))
+            for s_, t in cand[b:]:
+                assign[t] = -1
+            held[k] = cand[:b]
+            for s_, t in held[k]:
+                assign[t] = k
+    return assign, rounds
+
+
+@pytest.mark.parametrize("v,c,levels,seed", [(12, 3, 0, 0), (40, 5, 0, 1), (40, 5, 3, 2), (64, 8, 2, 3),
+                                             (96, 6, 0, 4), (60, 4, 1, 5)])
+def test_round_structure_of_the_kernels_gives_the_greedy_assignment(v, c, levels, seed):
+    # levels > 0 quantises the similarities to a few values, so ties decide most pairs
+    rng = np.random.default_rng(seed)
+    S = rng.standard_normal((v, c))
+    if levels:
+        S = np.round(S * levels) / levels
+    got, rounds = _deferred_acceptance(S, v // c)
+    assert got.tolist() == kmeans.balanced_assign(S, v // c).tolist()
+    assert rounds >= 1
