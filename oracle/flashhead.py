@@ -84,8 +84,26 @@ def dequantize_int4(C_q: np.ndarray, C_scales: np.ndarray) -> np.ndarray:
     return codes.astype(np.float64) * np.repeat(scale, INT4_GROUP, axis=1)
 
 
+def dequantize_int8(C_q: np.ndarray, C_scales: np.ndarray) -> np.ndarray:
+    """INT8 group-32 centroids -> exact float64 ``[c, d]``.
+
+    The W8A16 row of the write-up's parameter table (section 5.2) with the
+    stage-1 quantisation of section 1.2.4: one two's-complement byte per
+    element and one bf16 scale per 32 elements; value = code * scale, exact in
+    fp64 (and in fp32: at most 7 + 8 significant bits).
+    """
+    q = np.asarray(C_q).view(np.int8) if np.asarray(C_q).dtype == np.uint8 else np.asarray(C_q, dtype=np.int8)
+    c, d = q.shape
+    scale = widen_bf16(C_scales)
+    if scale.shape != (c, d // INT4_GROUP) or d % INT4_GROUP:
+        raise ValueError("scales must be [c, d/32]")
+    return q.astype(np.float64) * np.repeat(scale, INT4_GROUP, axis=1)
+
+
 def centroid_matrix(head) -> np.ndarray:
-    """The stage-1 centroid matrix in fp64: INT4 dequantised if present, else bf16 C."""
+    """The stage-1 centroid matrix in fp64: INT8 or INT4 dequantised if present, else bf16 C."""
+    if getattr(head, "C_q8", None) is not None:
+        return dequantize_int8(head.C_q8, head.C_scales8)
     if getattr(head, "C_q", None) is not None:
         return dequantize_int4(head.C_q, head.C_scales)
     return widen_bf16(head.C)

@@ -12,6 +12,8 @@ bytes:
 * INT4 centroids as ``uint8`` arrays, two signed nibbles per byte, element
   ``2i`` in the low nibble of byte ``i`` and element ``2i+1`` in the high one,
   with one bf16 scale per group of 32 elements,
+* INT8 centroids as ``int8`` arrays, one two's-complement code per element,
+  with one bf16 scale per group of 32 elements,
 * the cluster-to-token map ``C2T`` as ``int32 [c, b]``.
 
 Recipe (the planted-cluster head of the FlashHead write-up's shape table):
@@ -23,7 +25,8 @@ Recipe (the planted-cluster head of the FlashHead write-up's shape table):
   the balanced-clustering invariant of FlashHead section 1.2.1);
 * centroids: ``C_k = bf16(normalise(fp64 mean of the cluster's bf16 rows))``;
   the INT4 variant quantises that C symmetrically (codes -7..7, one bf16
-  scale ``max|x|/7`` per group of 32);
+  scale ``max|x|/7`` per group of 32), the INT8 variant likewise with codes
+  -127..127 and scale ``max|x|/127``;
 * hidden states: planted ``bf16(6*mu_j + N(0, 1/d))`` with ``j`` uniform over
   the clusters, or pure ``bf16(N(0, 1/d))`` for flat rows;
 * uniforms for Gumbel cluster selection ``[n, c]`` and for the token draw ``[n]``,
@@ -126,6 +129,8 @@ class Head:
     C2T: np.ndarray                 # int32 [c, b]
     C_q: Optional[np.ndarray] = None        # uint8 [c, d/2] packed signed nibbles
     C_scales: Optional[np.ndarray] = None   # uint16 [c, d/32] bf16 bits
+    C_q8: Optional[np.ndarray] = None       # int8 [c, d] codes (INT8 variant)
+    C_scales8: Optional[np.ndarray] = None  # uint16 [c, d/32] bf16 bits (INT8 variant)
     mu: Optional[np.ndarray] = None         # float64 [c, d] planted directions
     seed_base: int = 0
 
@@ -162,7 +167,36 @@ def quantize_int4_g32(C_bits: np.ndarray):
     return np.ascontiguousarray(packed), np.ascontiguousarray(scale_bits)
 
 
-def make_head(v: int, d: int, c: int, *, seed_base: int = 0, int4: bool = False,
+def _quantize_sym_g32(C_bits: np.ndarray, qmax: int):
+    """Symmetric codes -qmax..qmax with one bf16 scale ``max|x|/qmax`` per 32 elements.
+
+    Returns ``(codes int8 [c, d], scale bits uint16 [c, d/32])``. A group that
+    is all zero gets scale 0 and codes 0.
+    """
+    c, d = C_bits.shape
+    if d % INT4_GROUP:
+        raise ValueError("group-32 centroids need d % 32 == 0")
+    x = bf16_bits_to_f32(C_bits).astype(np.float64).reshape(c, d // INT4_GROUP, INT4_GROUP)
+    amax = np.abs(x).max(axis=2)
+    scale_bits = to_bf16_bits((amax / float(qmax)).astype(np.float32))
+    scale = bf16_bits_to_f32(scale_bits).astype(np.float64)
+    safe = np.where(scale > 0, scale, 1.0)
+    q = np.rint(x / safe[:, :, None])
+    q = np.where(scale[:, :, None] > 0, q, 0.0)
+    q = np.clip(q, -qmax, qmax).astype(np.int8).reshape(c, d)
+    return q, np.ascontiguousarray(scale_bits)
+
+
+def quantize_int8_g32(C_bits: np.ndarray):
+    """Symmetric INT8 with one bf16 scale per 32 elements (codes -127..127).
+
+    Returns ``(C_q int8 [c, d], C_scales uint16 [c, d/32])``.
+    """
+    q, scale_bits = _quantize_sym_g32(C_bits, 127)
+    return np.ascontiguousarray(q), scale_bits
+
+
+def make_head(v: int, d: int, c: int, *, seed_base: int = 0, int4: bool = False, int8: bool = False,
               keep_mu: bool = True, chunk_clusters: int = 512) -> Head:
     """Draw a balanced planted-cluster head with ``b = v/c`` tokens per cluster."""
     if v % c:
@@ -204,6 +238,8 @@ def make_head(v: int, d: int, c: int, *, seed_base: int = 0, int4: bool = False,
                 seed_base=seed_base)
     if int4:
         head.C_q, head.C_scales = quantize_int4_g32(C)
+    if int8:
+        head.C_q8, head.C_scales8 = quantize_int8_g32(C)
     return head
 
 

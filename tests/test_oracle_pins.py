@@ -119,6 +119,69 @@ def test_int4_roundtrip_within_half_step():
 
 
 # ---------------------------------------------------------------------------
+# INT8 (W8A16) centroids
+# ---------------------------------------------------------------------------
+def test_golden_int8_codes():
+    g = _load("int8_codes.json")
+    d = g["d"]
+    q = np.zeros((1, d), dtype=np.uint8)
+    q[0, :8] = g["bytes_first"]
+    q[0, 32:34] = g["group1_first_bytes"]
+    sc = np.array([g["scale_bits"]], dtype=np.uint16)
+    deq = oracle.dequantize_int8(q, sc)[0]
+    assert deq[:8].tolist() == g["expected_first_values"]
+    assert deq[32:34].tolist() == g["expected_group1_first_values"]
+    assert np.all(deq[8:32] == 0) and np.all(deq[34:] == 0)
+    # the same bytes given as int8 codes dequantise identically
+    assert np.array_equal(oracle.dequantize_int8(q.view(np.int8), sc)[0], deq)
+
+
+def test_int8_roundtrip_within_half_step():
+    rng = np.random.default_rng(8)
+    C = _bf16(rng.standard_normal((64, 256)) * 0.05)
+    C[5, 64:96] = 0  # an all-zero group
+    q, sc = synth.quantize_int8_g32(C)
+    assert q.dtype == np.int8 and q.shape == (64, 256) and sc.shape == (64, 8)
+    deq = oracle.dequantize_int8(q, sc)
+    x = oracle.widen_bf16(C)
+    scale = np.repeat(oracle.widen_bf16(sc), 32, axis=1)
+    err = np.abs(deq - x)
+    assert np.all(err <= 0.5 * scale * (1 + 2 ** -7) + 1e-300)
+    assert np.all(deq[5, 64:96] == 0)
+    assert q.min() >= -127 and q.max() <= 127
+    # INT8 is the finer grid: its error is far below the INT4 one on the same rows
+    q4, sc4 = synth.quantize_int4_g32(C)
+    assert np.abs(deq - x).mean() < 0.1 * np.abs(oracle.dequantize_int4(q4, sc4) - x).mean()
+
+
+def test_int8_values_are_exact_in_fp32_and_split_into_two_bf16():
+    # code * scale carries at most 7 + 8 significant bits: exact in fp32, and
+    # exactly hi + lo with hi = bf16(x) and lo = x - hi itself a bf16 value
+    rng = np.random.default_rng(9)
+    C = _bf16(rng.standard_normal((32, 128)))
+    q, sc = synth.quantize_int8_g32(C)
+    deq = oracle.dequantize_int8(q, sc)
+    f32 = deq.astype(np.float32)
+    assert np.array_equal(f32.astype(np.float64), deq)
+    hi = oracle.widen_bf16(_bf16(f32))
+    lo = deq - hi
+    assert np.array_equal(oracle.widen_bf16(_bf16(lo.astype(np.float32))), lo)
+
+
+def test_int8_head_selects_on_its_dequantised_centres():
+    # the oracle's INT8 path is the fp64 two-stage head over the dequantised centres
+    cfg, head, hid, _ = synth.make_config(0)
+    q, sc = synth.quantize_int8_g32(head.C)
+    h8 = _H(head.E, head.C, head.C2T)
+    h8.C_q8, h8.C_scales8 = q, sc
+    Cw = oracle.dequantize_int8(q, sc)
+    S = oracle.centroid_scores(Cw, hid.H[:4])
+    assert np.array_equal(oracle.centroid_scores(oracle.centroid_matrix(h8), hid.H[:4]), S)
+    toks, ids, _ = oracle.decode(h8, hid.H[:4], cfg.p)
+    assert np.array_equal(ids, oracle.select_greedy(S, cfg.p))
+
+
+# ---------------------------------------------------------------------------
 # C2T invariant
 # ---------------------------------------------------------------------------
 def test_c2t_permutation_invariant():
