@@ -392,7 +392,6 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
     o += up(decode_b1_misc_bytes(), 128);
     h->b1_off_slots = static_cast<int>(o);
     h->b1_slot_bytes = static_cast<int>(up(std::max(static_cast<size_t>(h->crow_bytes), static_cast<size_t>(D.d) * 2), 128));
-    // the slots double as the selector's scratch once phase 1 is done
     // the slots double as the selection's scratch between the phases
     o += std::max(static_cast<size_t>(kWarps) * h->b1_slot_bytes, decode_b1_scratch_bytes(D.c, h->b1_list_cap));
     h->b1_smem = o;

@@ -173,6 +173,33 @@ def select_sampled(S: np.ndarray, U: np.ndarray, p: int, T: float) -> np.ndarray
     return np.stack([_top_p_by_key(K[r], p) for r in range(K.shape[0])])
 
 
+def adaptive_probe_count(S: np.ndarray, tau: float, p_min: int, p_max: int, T: float = 1.0) -> np.ndarray:
+    """Probes per row adapted to the spread of its centroid scores (section 1.2.2, "dynamic adjustment").
+
+    The write-up lets the number of probes follow the distribution of the
+    hidden state's centroid scores, with fewer probes where it is peaked
+    (section 4.2: frequent tokens need fewer). Read here as: the smallest
+    ``p`` in ``[p_min, p_max]`` whose top-``p`` clusters hold at least a
+    fraction ``tau`` of ``softmax(s / T)`` over all c clusters. The mass of
+    the top p depends only on the p largest values, not on how ties among
+    them are ordered.
+    """
+    if not 0.0 < tau <= 1.0 or not 1 <= p_min <= p_max:
+        raise ValueError("need 0 < tau <= 1 and 1 <= p_min <= p_max")
+    if not T > 0:
+        raise ValueError("temperature must be > 0")
+    S = np.atleast_2d(np.asarray(S, dtype=np.float64))
+    p_max = min(p_max, S.shape[1])
+    out = np.empty(S.shape[0], dtype=np.int32)
+    for r in range(S.shape[0]):
+        y = np.sort(S[r] / T)[::-1]
+        w = np.exp(y - y[0])
+        mass = np.cumsum(w) / w.sum()
+        p = int(np.searchsorted(mass, tau, side="left")) + 1   # first p with mass >= tau
+        out[r] = min(max(p, p_min), p_max)
+    return out
+
+
 # ---------------------------------------------------------------------------
 # gather + stage 2 candidate logits
 # ---------------------------------------------------------------------------

@@ -119,6 +119,48 @@ def test_int4_roundtrip_within_half_step():
 
 
 # ---------------------------------------------------------------------------
+# adaptive probe count (reading: smallest p whose top-p softmax mass reaches tau)
+# ---------------------------------------------------------------------------
+def test_adaptive_probes_closed_forms():
+    # equal scores: the top p hold p/c of the mass
+    assert oracle.adaptive_probe_count(np.zeros((1, 100)), 0.305, 1, 100)[0] == 31
+    assert oracle.adaptive_probe_count(np.zeros((1, 100)), 0.295, 1, 100)[0] == 30
+    # "at least tau": a mass of exactly tau (0.5 = 2/4, exact in binary) stops at that p
+    assert oracle.adaptive_probe_count(np.zeros((1, 4)), 0.5, 1, 4)[0] == 2
+    # ten clusters at ln 9, ninety at 0: weights 9 and 1, mass of the top p = p/20 up to p = 10,
+    # then (90 + p - 10) / 180
+    S = np.r_[np.full(10, math.log(9.0)), np.zeros(90)][None, :]
+    rng = np.random.default_rng(3)
+    S = S[:, rng.permutation(100)]
+    assert oracle.adaptive_probe_count(S, 0.41, 1, 100)[0] == 9
+    assert oracle.adaptive_probe_count(S, 0.61, 1, 100)[0] == 30
+    # one dominant cluster: p_min
+    D = np.zeros((1, 1000))
+    D[0, 17] = 50.0
+    assert oracle.adaptive_probe_count(D, 0.99, 4, 512)[0] == 4
+    # everything: clamped to p_max
+    assert oracle.adaptive_probe_count(np.zeros((1, 100)), 1.0, 1, 64)[0] == 64
+
+
+def test_adaptive_probes_temperature_and_monotonicity():
+    rng = np.random.default_rng(4)
+    S = rng.standard_normal((6, 300))
+    a = oracle.adaptive_probe_count(S, 0.5, 1, 300, T=0.7)
+    assert np.array_equal(a, oracle.adaptive_probe_count(2.0 * S, 0.5, 1, 300, T=1.4))   # depends on s/T only
+    assert np.array_equal(a, oracle.adaptive_probe_count(S + 3.0, 0.5, 1, 300, T=0.7))   # shift invariant
+    prev = np.zeros(6, dtype=np.int32)
+    for tau in (0.1, 0.3, 0.5, 0.7, 0.9, 0.99):
+        cur = oracle.adaptive_probe_count(S, tau, 1, 300)
+        assert np.all(cur >= prev)
+        prev = cur
+    # a very high temperature flattens the law: p -> ceil(tau c) within one
+    hot = oracle.adaptive_probe_count(S, 0.5, 1, 300, T=1e6)
+    assert np.all(np.abs(hot - 150) <= 1)
+    # colder is more peaked: never more probes
+    assert np.all(oracle.adaptive_probe_count(S, 0.5, 1, 300, T=0.3) <= a)
+
+
+# ---------------------------------------------------------------------------
 # INT8 (W8A16) centroids
 # ---------------------------------------------------------------------------
 def test_golden_int8_codes():
