@@ -253,6 +253,44 @@ def sample_token(tokens: np.ndarray, z: np.ndarray, T: float, u_tok: float) -> i
     return int(tokens[min(i, len(tokens) - 1)])
 
 
+def speculative_verify(z_full: np.ndarray, cand_tokens: np.ndarray, T: float, draft: int,
+                       u_accept: float, u_resample: float) -> int:
+    """Check a FlashHead draft token against the dense head (section 4.2, speculative decoding).
+
+    The write-up drafts with FlashHead sampling and accepts or rejects with
+    the original head's probabilities. Read as standard speculative
+    sampling with the draft law taken given the chosen clusters: ``q`` =
+    ``softmax(z/T)`` over the candidate tokens (zero elsewhere), ``p`` =
+    ``softmax(z/T)`` over the whole vocabulary. The draft is kept when
+    ``u_accept < p(x) / q(x)``; otherwise the token is drawn by inverse CDF
+    (token id order, first running sum above ``u_resample`` times the total)
+    from ``max(0, p - q)``. For every cluster set the result follows ``p``
+    exactly, so the two-stage head's approximation disappears at the cost of
+    one dense pass.
+    """
+    if not T > 0:
+        raise ValueError("temperature must be > 0")
+    z = np.asarray(z_full, dtype=np.float64) / T
+    p = np.exp(z - z.max())
+    p /= p.sum()
+    toks = np.asarray(cand_tokens, dtype=np.int64)
+    zc = z[toks]
+    qc = np.exp(zc - zc.max())
+    qc /= qc.sum()
+    q = np.zeros_like(p)
+    q[toks] = qc
+    x = int(draft)
+    if q[x] <= 0.0:
+        raise ValueError("the draft must be one of the candidates")
+    if u_accept < p[x] / q[x]:
+        return x
+    r = np.maximum(p - q, 0.0)
+    cdf = np.cumsum(r)
+    u = min(max(float(u_resample), 0.0), U_MAX)
+    i = int(np.searchsorted(cdf, u * cdf[-1], side="right"))
+    return min(i, len(r) - 1)
+
+
 # ---------------------------------------------------------------------------
 # whole path
 # ---------------------------------------------------------------------------

@@ -161,6 +161,56 @@ def test_adaptive_probes_temperature_and_monotonicity():
 
 
 # ---------------------------------------------------------------------------
+# speculative drafting: FlashHead draft, dense-head verification
+# ---------------------------------------------------------------------------
+def _softmax(x):
+    from scipy.special import softmax
+    return softmax(np.asarray(x, dtype=np.float64))
+
+
+def test_speculative_verify_output_follows_the_dense_softmax():
+    # draft x ~ q (softmax over the candidates only), then verify: the output
+    # law must be softmax(z/T) over the whole vocabulary (chi-square, fixed seed)
+    rng = np.random.default_rng(12)
+    v, T = 10, 0.8
+    z = rng.standard_normal(v) * 1.5
+    cand = np.array([1, 4, 7, 8])
+    p = _softmax(z / T)
+    q = _softmax(z[cand] / T)
+    n = 60000
+    xs = cand[np.searchsorted(np.cumsum(q), rng.random(n), side="right").clip(0, len(cand) - 1)]
+    ua, ur = rng.random(n), rng.random(n)
+    out = np.array([oracle.speculative_verify(z, cand, T, int(xs[i]), ua[i], ur[i]) for i in range(n)])
+    obs = np.bincount(out, minlength=v)
+    chi2, pval = stats.chisquare(obs, p * n)
+    assert pval > 1e-3, (obs, p * n)
+
+
+def test_speculative_verify_accepts_and_resamples_as_defined():
+    rng = np.random.default_rng(13)
+    v, T = 12, 1.3
+    z = rng.standard_normal(v)
+    # every token a candidate: q = p, every draft is kept
+    for x in range(v):
+        assert oracle.speculative_verify(z, np.arange(v), T, x, 0.999999, 0.5) == x
+    cand = np.array([0, 2, 3, 9, 11])
+    p = _softmax(z / T)
+    q = np.zeros(v)
+    q[cand] = _softmax(z[cand] / T)
+    for x in cand:
+        assert oracle.speculative_verify(z, cand, T, int(x), 0.0, 0.5) == x     # u = 0 always keeps
+    # a rejected draft is replaced from max(0, p - q): its law on a fine u grid
+    x = int(cand[np.argmax(q[cand] - p[cand])])   # the draft most over-weighted by q: ratio < 1
+    assert p[x] / q[x] < 1
+    M = 20000
+    outs = np.array([oracle.speculative_verify(z, cand, T, x, 0.9999999, (i + 0.5) / M) for i in range(M)])
+    r = np.maximum(p - q, 0.0)
+    r /= r.sum()
+    assert np.all(np.abs(np.bincount(outs, minlength=v) / M - r) <= 2.0 / M)
+    assert np.all(r[np.bincount(outs, minlength=v) > 0] > 0)
+
+
+# ---------------------------------------------------------------------------
 # INT8 (W8A16) centroids
 # ---------------------------------------------------------------------------
 def test_golden_int8_codes():
