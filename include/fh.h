@@ -7,7 +7,7 @@
  * token_scores):
  *
  *   1. centroid scores  s = C h over c balanced clusters (section 1.2.2),
- *      C in bf16 or in INT4 with one bf16 scale per 32 elements
+ *      C in bf16, or in INT4 or INT8 with one bf16 scale per 32 elements
  *      (selective quantisation, section 1.2.4);
  *   2. probe selection: the p best clusters (multi-probe retrieval,
  *      section 1.2.2), or p clusters drawn by multinomial sampling at
@@ -65,7 +65,8 @@ typedef enum {
 
 typedef enum {
   FH_CENTROID_BF16 = 0,     /* C: bf16 [c, d] */
-  FH_CENTROID_INT4_G32 = 1  /* C_q: uint8 [c, d/2], C_scales: bf16 [c, d/32] */
+  FH_CENTROID_INT4_G32 = 1, /* C_q: uint8 [c, d/2], C_scales: bf16 [c, d/32] */
+  FH_CENTROID_INT8_G32 = 2  /* C_q: int8 [c, d], C_scales: bf16 [c, d/32] (W8A16) */
 } fh_centroid_format;
 
 typedef enum {
@@ -79,12 +80,15 @@ typedef enum {
  * cluster k, so slot k*b + j of the flattened map names one token).
  *
  *  v, d, c, b   vocabulary, hidden size, clusters, tokens per cluster;
- *               v == c*b, d % 8 == 0 (d % 32 == 0 for INT4), 1 <= c.
+ *               v == c*b, d % 8 == 0 (d % 32 == 0 for INT4 / INT8), 1 <= c.
  *  E            device bf16 [v, d], 16-byte aligned.
  *  C            device bf16 [c, d], 16-byte aligned (BF16 format, else NULL).
  *  C_q          device uint8 [c, d/2] (INT4 format): element 2i in the low
- *               nibble of byte i, 2i+1 in the high nibble, two's complement.
- *  C_scales     device bf16 [c, d/32] (INT4 format): value = code * scale.
+ *               nibble of byte i, 2i+1 in the high nibble, two's complement;
+ *               or device int8 [c, d] (INT8 format): one two's-complement
+ *               byte per element (the W8A16 row of the write-up's parameter
+ *               table, section 5.2).
+ *  C_scales     device bf16 [c, d/32] (INT4 and INT8 formats): value = code * scale.
  *  C2T          device int32 [c, b].
  *  fmt          fh_centroid_format.
  *  max_batch    largest B any call will pass (>= 1).
@@ -110,9 +114,9 @@ typedef struct fh_head fh_head;
  * workspace, and fills two library-owned copies inside it: the token rows of
  * E in cluster-major order (row k*b + j = E[C2T[k][j]], v*d*2 bytes; a
  * cluster's b rows are one contiguous block, read without a C2T lookup), and,
- * for INT4, each centroid row packed with its scales (row = d/2 code bytes,
- * then d/16 scale bytes, padded to 16 bytes) so that one bulk copy moves a
- * row. Synchronises `stream`. On success *out owns the workspace; release it
+ * for INT4 / INT8, each centroid row packed with its scales (row = d/2 or
+ * d code bytes, then d/16 scale bytes, padded to 16 bytes) so that one bulk
+ * copy moves a row. Synchronises `stream`. On success *out owns the workspace; release it
  * with fh_destroy. E itself is still read by the dense head.
  */
 fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out);
@@ -122,7 +126,7 @@ void fh_destroy(fh_head* head);
 
 /*
  * Stage 1 (write-up section 1.2.2): scores[r][k] = sum_i C[k][i] * hidden[r][i]
- * for r < B, k < c (INT4: C dequantised exactly, code * scale).
+ * for r < B, k < c (INT4 / INT8: C dequantised exactly, code * scale).
  *  hidden  device bf16 [B, d], 16-byte aligned.
  *  scores  device fp32 [B, c].
  */

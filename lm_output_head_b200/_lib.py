@@ -22,6 +22,7 @@ FH_ERR_TIMEOUT = 7
 
 FH_CENTROID_BF16 = 0
 FH_CENTROID_INT4_G32 = 1
+FH_CENTROID_INT8_G32 = 2
 FH_GREEDY = 0
 FH_SAMPLE_GUMBEL = 1
 

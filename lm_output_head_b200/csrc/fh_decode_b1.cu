@@ -6,7 +6,7 @@
 // The pages' pipeline (FlashHead write-up, section 2.2.2: h -> centroid_scores
 // -> top_p_clusters -> token_scores) runs as phases of one kernel:
 //
-//  1. centroid scores (section 1.2.2; INT4 centroids per section 1.2.4):
+//  1. centroid scores (section 1.2.2; INT4 or INT8 centroids per section 1.2.4):
 //     cluster k belongs to CTA k mod G (warp (k / G) mod 16), so every CTA
 //     owns c/G clusters. A warp's first row streams into registers, its
 //     second into a shared-memory slot by one bulk copy, both requested at
@@ -102,8 +102,9 @@ __device__ __forceinline__ int region_bin(float key, float L, float S) {
   return x >= static_cast<float>(kB1Bins - 1) ? kB1Bins - 1 : static_cast<int>(x);
 }
 
-template <int NCH, bool INT4>
+template <int NCH, int FMT>
 __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P) {
+  constexpr bool INT4 = FMT == kFmtInt4, INT8 = FMT == kFmtInt8;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = gridDim.x;
@@ -145,8 +146,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   }
   uint4 w[NCH];
   uint32_t q[NCH], sc[NCH];
+  uint2 q8[NCH];
+  uint32_t sw8[int8_scale_words<NCH>()];
   if (n1 > 0) {
     if constexpr (INT4) row_load_int4<NCH>(P.Crows + static_cast<size_t>(cw) * P.crow_bytes, d, q, sc);
+    else if constexpr (INT8) row_load_int8<NCH>(P.Crows + static_cast<size_t>(cw) * P.crow_bytes, d, q8, sw8);
     else row_load_bf16<NCH>(reinterpret_cast<const uint16_t*>(P.Crows + static_cast<size_t>(cw) * P.crow_bytes), d, w);
   }
   float ureg = 0.f;  // lane j holds u of item j
@@ -203,10 +207,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
       if (!mbar_wait_bounded(wbar, wphase, kWaitBudget) && lane == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
       wphase ^= 1u;
       if constexpr (INT4) s = srow_dot_int4_hs<NCH>(slot, hs, d);
+      else if constexpr (INT8) s = srow_dot_int8_hs<NCH>(slot, hs, d);
       else s = srow_dot_bf16_hs<NCH>(slot, hs, d);
     } else if constexpr (INT4) {
       if (i > 0) row_load_int4<NCH>(P.Crows + static_cast<size_t>(k) * P.crow_bytes, d, q, sc);
       s = row_dot_int4_hs<NCH>(q, sc, hs, d);
+    } else if constexpr (INT8) {
+      if (i > 0) row_load_int8<NCH>(P.Crows + static_cast<size_t>(k) * P.crow_bytes, d, q8, sw8);
+      s = row_dot_int8_hs<NCH>(q8, sw8, hs, d);
     } else {
       if (i > 0) row_load_bf16<NCH>(reinterpret_cast<const uint16_t*>(P.Crows + static_cast<size_t>(k) * P.crow_bytes), d, w);
       s = row_dot_bf16_hs<NCH>(w, hs, d);
@@ -593,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
 }
 
 template <int NCH>
-cudaError_t launch_nch(const B1Params& P, int grid, size_t smem, int int4, cudaStream_t st) {
+cudaError_t launch_nch(const B1Params& P, int grid, size_t smem, int cfmt, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
@@ -604,8 +612,9 @@ cudaError_t launch_nch(const B1Params& P, int grid, size_t smem, int int4, cudaS
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (int4) return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, true>, P);
-  return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, false>, P);
+  if (cfmt == kFmtInt4) return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, kFmtInt4>, P);
+  if (cfmt == kFmtInt8) return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, kFmtInt8>, P);
+  return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, kFmtBf16>, P);
 }
 
 }  // namespace
@@ -626,24 +635,27 @@ extern "C" int fh_timeline_read(unsigned long long* host, int n) {
 }
 #endif
 
-cudaError_t launch_decode_b1(const B1Params& P, int grid, size_t smem, int int4, int nch, cudaStream_t st) {
+cudaError_t launch_decode_b1(const B1Params& P, int grid, size_t smem, int cfmt, int nch, cudaStream_t st) {
   switch (nch) {
-    case 1: return launch_nch<1>(P, grid, smem, int4, st);
-    case 2: return launch_nch<2>(P, grid, smem, int4, st);
-    case 3: return launch_nch<3>(P, grid, smem, int4, st);
-    case 4: return launch_nch<4>(P, grid, smem, int4, st);
-    case 5: return launch_nch<5>(P, grid, smem, int4, st);
-    case 6: return launch_nch<6>(P, grid, smem, int4, st);
-    case 8: return launch_nch<8>(P, grid, smem, int4, st);
-    case 10: return launch_nch<10>(P, grid, smem, int4, st);
+    case 1: return launch_nch<1>(P, grid, smem, cfmt, st);
+    case 2: return launch_nch<2>(P, grid, smem, cfmt, st);
+    case 3: return launch_nch<3>(P, grid, smem, cfmt, st);
+    case 4: return launch_nch<4>(P, grid, smem, cfmt, st);
+    case 5: return launch_nch<5>(P, grid, smem, cfmt, st);
+    case 6: return launch_nch<6>(P, grid, smem, cfmt, st);
+    case 8: return launch_nch<8>(P, grid, smem, cfmt, st);
+    case 10: return launch_nch<10>(P, grid, smem, cfmt, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
-cudaError_t occupancy_decode_b1(int int4, int nch, size_t smem, int* blocks) {
-#define FH_O(N)                                                                                      \
-  return int4 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, decode_b1_kernel<N, true>, kThreads, smem) \
-              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, decode_b1_kernel<N, false>, kThreads, smem);
+cudaError_t occupancy_decode_b1(int cfmt, int nch, size_t smem, int* blocks) {
+#define FH_O(N)                                                                                           \
+  return cfmt == kFmtInt4                                                                                 \
+             ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, decode_b1_kernel<N, kFmtInt4>, kThreads, smem) \
+         : cfmt == kFmtInt8                                                                               \
+             ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, decode_b1_kernel<N, kFmtInt8>, kThreads, smem) \
+             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, decode_b1_kernel<N, kFmtBf16>, kThreads, smem);
   switch (nch) {
     case 1: FH_O(1)
     case 2: FH_O(2)
@@ -662,9 +674,11 @@ cudaError_t set_attrs_decode_b1(int max_smem) {
   cudaError_t e = cudaSuccess;
 #define FH_SET(N)                                                                                         \
   if (e == cudaSuccess)                                                                                   \
-    e = cudaFuncSetAttribute(decode_b1_kernel<N, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem); \
+    e = cudaFuncSetAttribute(decode_b1_kernel<N, kFmtBf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem); \
   if (e == cudaSuccess)                                                                                   \
-    e = cudaFuncSetAttribute(decode_b1_kernel<N, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+    e = cudaFuncSetAttribute(decode_b1_kernel<N, kFmtInt4>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem); \
+  if (e == cudaSuccess)                                                                                   \
+    e = cudaFuncSetAttribute(decode_b1_kernel<N, kFmtInt8>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
   FH_SET(1) FH_SET(2) FH_SET(3) FH_SET(4) FH_SET(5) FH_SET(6) FH_SET(8) FH_SET(10)
 #undef FH_SET
   return e;

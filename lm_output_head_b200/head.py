@@ -51,8 +51,9 @@ def bf16_from_bits(bits: np.ndarray, device="cuda") -> torch.Tensor:
 class FlashHead:
     """A FlashHead retrieval head bound to device tensors (borrowed, kept alive here).
 
-    ``E`` bf16 [v, d]; ``C2T`` int32 [c, b]; centroids either ``C`` bf16 [c, d]
-    or ``C_q`` uint8 [c, d/2] with ``C_scales`` bf16 [c, d/32].
+    ``E`` bf16 [v, d]; ``C2T`` int32 [c, b]; centroids either ``C`` bf16 [c, d],
+    or ``C_q`` with ``C_scales`` bf16 [c, d/32]: uint8 [c, d/2] packed INT4
+    codes, or int8 [c, d] INT8 codes (the dtype picks the format).
     """
 
     def __init__(self, E: torch.Tensor, C2T: torch.Tensor, *, C: Optional[torch.Tensor] = None,
@@ -68,11 +69,11 @@ class FlashHead:
             C = _dev(C, "C", _BF16, 2)
             fmt = _lib.FH_CENTROID_BF16
         elif C_q is not None and C_scales is not None:
-            C_q = _dev(C_q, "C_q", (torch.uint8,), 2)
+            C_q = _dev(C_q, "C_q", (torch.uint8, torch.int8), 2)
             C_scales = _dev(C_scales, "C_scales", _BF16, 2)
-            fmt = _lib.FH_CENTROID_INT4_G32
+            fmt = _lib.FH_CENTROID_INT8_G32 if C_q.dtype == torch.int8 else _lib.FH_CENTROID_INT4_G32
         else:
-            raise ValueError("give C (bf16) or C_q and C_scales (INT4)")
+            raise ValueError("give C (bf16) or C_q and C_scales (INT4 uint8 / INT8 int8 codes)")
         self.E, self.C2T, self.C, self.C_q, self.C_scales = E, C2T, C, C_q, C_scales
         self.v, self.d, self.c, self.b = v, d, c, b
         self.fmt = fmt
