@@ -207,3 +207,45 @@ def test_create_rejects_bad_shapes(fh):
     assert lib.fh_cluster_create(100, 256, 3, None, ctypes.byref(h)) == _lib.FH_ERR_INVALID_ARG
     assert lib.fh_cluster_create(4096, 250, 64, None, ctypes.byref(h)) == _lib.FH_ERR_INVALID_ARG
     assert lib.fh_cluster_create(4096, 256, 64, None, ctypes.byref(h)) == _lib.FH_ERR_UNSUPPORTED  # b = 64
+
+
+def test_assign_at_the_llama_shape_has_no_blocking_pair(fh):
+    """v 128256, c 8016, d 2048 from k-means++ seeds: the assignment is balanced and,
+    on the same fp32 similarities, no token prefers a cluster whose weakest member
+    it beats -- the property that makes it the global greedy (unique under the
+    order similarity desc, token asc, cluster asc)."""
+    from lm_output_head_b200.cluster import ClusterBuilder
+    cfg, head, _, _ = synth.make_config(1, n_states=1)
+    v, d, c, b = head.v, head.d, head.c, head.b
+    cbl = ClusterBuilder(v, d, c)
+    try:
+        En = cbl.normalize(fh.bf16_from_bits(head.E, "cuda"))
+        u = np.random.default_rng(21).uniform(size=c).astype(np.float32)
+        ids = cbl.seed(En, torch.from_numpy(u).cuda())
+        assert cbl.device_status() == 0
+        idh = ids.cpu().numpy()
+        assert idh[0] == min(int(math.floor(float(u[0]) * v)), v - 1) and len(set(idh.tolist())) == c
+        S = cbl.similarities(En, cbl.gather(En, ids))
+        a, m, rounds = cbl.assign(S)
+        assert cbl.device_status() == 0
+        mh = m.cpu().numpy()
+        assert oracle.check_c2t(mh, v) and np.all(np.diff(mh, axis=1) > 0)
+        a = a.long()
+        t_all = torch.arange(v, device="cuda")
+        sa = S[a, t_all]                                    # every token's similarity to its cluster
+        ms = S.gather(1, m.long())                          # [c, b] members' similarities
+        # weakest member of every cluster: lowest similarity, then highest token id
+        ws = ms.min(dim=1).values
+        wt = torch.where(ms == ws[:, None], m.long(), torch.full_like(m.long(), -1)).max(dim=1).values
+        blocking = 0
+        for k0 in range(0, c, 512):
+            k1 = min(c, k0 + 512)
+            Sc = S[k0:k1]
+            kk = torch.arange(k0, k1, device="cuda")[:, None]
+            pref = (Sc > sa[None, :]) | ((Sc == sa[None, :]) & (kk < a[None, :]))
+            beats = (Sc > ws[k0:k1, None]) | ((Sc == ws[k0:k1, None]) & (t_all[None, :] < wt[k0:k1, None]))
+            blocking += int((pref & beats & (kk != a[None, :])).sum().item())
+        assert blocking == 0
+        assert rounds >= 1
+    finally:
+        cbl.close()
