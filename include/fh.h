@@ -255,6 +255,29 @@ typedef enum {
 } fh_query_key;
 fh_status fh_query(fh_head* head, int32_t key, int64_t* value);
 
+/*
+ * Speculative drafting (write-up section 4.2): check FlashHead draft tokens
+ * against the dense head. For row r, p = softmax(z/T) over the vocabulary
+ * (z = logits[r], the dense head's logits) and q = softmax(z/T) over the
+ * draft's candidate tokens cand_tokens[r][0..n) (the tokens of the clusters
+ * it was drawn from, e.g. fh_candidate_logits' token ids). The draft x =
+ * draft[r] is kept when u_accept[r] < p(x) / q(x); otherwise the token is the
+ * inverse-CDF draw (token id order) at u_resample[r] from max(0, p - q). For
+ * every cluster set the result follows p exactly (standard speculative
+ * sampling with the draft law taken given the chosen clusters).
+ *  logits       device fp32 [B, v].
+ *  cand_tokens  device int32 [B, n], distinct ids in [0, v) per row.
+ *  draft        device int32 [B], one of the row's candidates.
+ *  u_accept, u_resample  device fp32 [B], uniforms in [0, 1).
+ *  out_tokens   device int32 [B]; -1 and FH_ERR_OUT_OF_RANGE in the device
+ *               status when a candidate or the draft is out of range or the
+ *               draft is not a candidate.
+ * FH_ERR_UNSUPPORTED when the candidate bitmap (v bits) exceeds shared memory.
+ */
+fh_status fh_speculative_verify(fh_head* head, const float* logits, const int32_t* cand_tokens, int32_t n,
+                                int32_t B, const int32_t* draft, float T, const float* u_accept,
+                                const float* u_resample, int32_t* out_tokens, fh_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

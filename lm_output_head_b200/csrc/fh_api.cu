@@ -685,4 +685,18 @@ fh_status fh_dense_head(fh_head* h, const void* hidden, int32_t B, float* logits
   return FH_OK;
 }
 
+fh_status fh_speculative_verify(fh_head* h, const float* logits, const int32_t* cand_tokens, int32_t n, int32_t B,
+                                const int32_t* draft, float T, const float* u_accept, const float* u_resample,
+                                int32_t* out_tokens, fh_stream_t stream) {
+  if (!h || !logits || !cand_tokens || !draft || !u_accept || !u_resample || !out_tokens) return FH_ERR_INVALID_ARG;
+  if (B < 1 || n < 1 || n > h->desc.v || !(T > 0.f && T < 3.0e38f)) return FH_ERR_INVALID_ARG;
+  cudaError_t e = launch_spec_verify(logits, h->desc.v, cand_tokens, n, B, draft, T, u_accept, u_resample, out_tokens,
+                                     &h->sync->status, reinterpret_cast<cudaStream_t>(stream));
+  if (e == cudaErrorInvalidValue) {
+    (void)cudaGetLastError();
+    return FH_ERR_UNSUPPORTED;
+  }
+  return e == cudaSuccess ? FH_OK : cuda_fail(e);
+}
+
 }  // extern "C"

@@ -201,6 +201,10 @@ cudaError_t set_attrs_gemm();
 // pass per distinct cluster on the tensor cores.
 cudaError_t launch_group(const GroupParams& P, int num_sms, cudaStream_t st);
 cudaError_t set_attrs_group();
+// Speculative verification of draft tokens against dense logits (one CTA per row).
+cudaError_t launch_spec_verify(const float* logits, int v, const int32_t* cand, int n, int B, const int32_t* draft,
+                               float T, const float* u_accept, const float* u_resample, int32_t* out, int* status,
+                               cudaStream_t st);
 
 // Opt-in shared memory attribute for every instantiation (called once per device).
 cudaError_t set_kernel_attributes(int max_smem);

@@ -192,6 +192,21 @@ class FlashHead:
         return (out_argmax, logits) if want_logits else out_argmax
 
 
+def speculative_verify(head: FlashHead, logits: torch.Tensor, cand_tokens: torch.Tensor, draft: torch.Tensor,
+                       T: float, u_accept: torch.Tensor, u_resample: torch.Tensor, stream=None) -> torch.Tensor:
+    """Check FlashHead drafts against the dense logits (``fh_speculative_verify``)."""
+    logits = _dev(logits, "logits", (torch.float32,), 2)
+    cand_tokens = _dev(cand_tokens, "cand_tokens", (torch.int32,), 2)
+    B, n = cand_tokens.shape
+    if logits.shape != (B, head.v):
+        raise ValueError("logits must be [B, v]")
+    out = torch.empty(B, dtype=torch.int32, device=logits.device)
+    _check(head._lib.fh_speculative_verify(head._h, _ptr(logits), _ptr(cand_tokens), int(n), int(B), _ptr(draft),
+                                           float(T), _ptr(u_accept), _ptr(u_resample), _ptr(out), _stream(stream)),
+           "fh_speculative_verify")
+    return out
+
+
 def dense_head_noalloc(E: torch.Tensor, hidden: torch.Tensor, out_argmax: torch.Tensor, *,
                        logits: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Dense head through ``fh_dense_head_noalloc``: no handle and no device
