@@ -195,6 +195,9 @@ cudaError_t set_attrs_gemm();
 // pass per distinct cluster on the tensor cores.
 cudaError_t launch_group(const GroupParams& P, int num_sms, cudaStream_t st);
 cudaError_t set_attrs_group();
+// Adaptive probe count per row of centroid scores (one CTA per row).
+cudaError_t launch_adaptive_probes(const float* scores, int B, int c, float tau, int p_min, int p_max, float T,
+                                   int32_t* out_p, cudaStream_t st);
 
 // Opt-in shared memory attribute for every instantiation (called once per device).
 cudaError_t set_kernel_attributes(int max_smem);
