@@ -278,6 +278,21 @@ fh_status fh_speculative_verify(fh_head* head, const float* logits, const int32_
                                 int32_t B, const int32_t* draft, float T, const float* u_accept,
                                 const float* u_resample, int32_t* out_tokens, fh_stream_t stream);
 
+/*
+ * Adaptive probe count (write-up section 1.2.2, "dynamic adjustment"; section
+ * 4.2: fewer probes for frequent tokens). For each row r of scores, out_p[r]
+ * = the smallest p in [p_min, p_max] whose top-p clusters hold at least a
+ * fraction tau of softmax(scores[r] / T) over all c clusters (the mass of the
+ * top p depends only on the p largest scores, not on the order of ties).
+ * Use it with fh_decode / fh_select_clusters row by row.
+ *  scores  device fp32 [B, c] (fh_centroid_scores' output).
+ *  out_p   device int32 [B].
+ * 0 < tau <= 1, 1 <= p_min <= p_max <= c, T finite and > 0.
+ * FH_ERR_UNSUPPORTED when a row's scores (next power of two of c, fp32) exceed shared memory.
+ */
+fh_status fh_adaptive_probes(fh_head* head, const float* scores, int32_t B, float tau, int32_t p_min,
+                             int32_t p_max, float T, int32_t* out_p, fh_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

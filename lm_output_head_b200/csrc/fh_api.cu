@@ -699,4 +699,18 @@ fh_status fh_speculative_verify(fh_head* h, const float* logits, const int32_t* 
   return e == cudaSuccess ? FH_OK : cuda_fail(e);
 }
 
+fh_status fh_adaptive_probes(fh_head* h, const float* scores, int32_t B, float tau, int32_t p_min, int32_t p_max,
+                             float T, int32_t* out_p, fh_stream_t stream) {
+  if (!h || !scores || !out_p || B < 1) return FH_ERR_INVALID_ARG;
+  if (!(tau > 0.f && tau <= 1.f) || p_min < 1 || p_min > p_max || p_max > h->desc.c) return FH_ERR_INVALID_ARG;
+  if (!(T > 0.f && T < 3.0e38f)) return FH_ERR_INVALID_ARG;
+  cudaError_t e = launch_adaptive_probes(scores, B, h->desc.c, tau, p_min, p_max, T, out_p,
+                                         reinterpret_cast<cudaStream_t>(stream));
+  if (e == cudaErrorInvalidValue) {
+    (void)cudaGetLastError();
+    return FH_ERR_UNSUPPORTED;
+  }
+  return e == cudaSuccess ? FH_OK : cuda_fail(e);
+}
+
 }  // extern "C"

@@ -205,6 +205,9 @@ cudaError_t set_attrs_group();
 cudaError_t launch_spec_verify(const float* logits, int v, const int32_t* cand, int n, int B, const int32_t* draft,
                                float T, const float* u_accept, const float* u_resample, int32_t* out, int* status,
                                cudaStream_t st);
+// Adaptive probe count per row of centroid scores (one CTA per row).
+cudaError_t launch_adaptive_probes(const float* scores, int B, int c, float tau, int p_min, int p_max, float T,
+                                   int32_t* out_p, cudaStream_t st);
 
 // Opt-in shared memory attribute for every instantiation (called once per device).
 cudaError_t set_kernel_attributes(int max_smem);

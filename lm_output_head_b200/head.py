@@ -166,6 +166,17 @@ class FlashHead:
                                              _ptr(logits), _stream(stream)), "fh_candidate_logits")
         return toks, logits
 
+    def adaptive_probes(self, scores: torch.Tensor, tau: float, p_min: int, p_max: int, *, T: float = 1.0,
+                        stream=None) -> torch.Tensor:
+        """Probes per row: the smallest p in [p_min, p_max] whose top-p clusters hold a fraction tau
+        of softmax(scores / T)."""
+        scores = _dev(scores, "scores", (torch.float32,), 2)
+        B = scores.shape[0]
+        out = torch.empty(B, dtype=torch.int32, device=self.device)
+        _check(self._lib.fh_adaptive_probes(self._h, _ptr(scores), B, float(tau), int(p_min), int(p_max), float(T),
+                                            _ptr(out), _stream(stream)), "fh_adaptive_probes")
+        return out
+
     def decode(self, hidden: torch.Tensor, p: int, *, mode: str = "greedy", T: float = 1.0,
                u_clusters: Optional[torch.Tensor] = None, u_token: Optional[torch.Tensor] = None,
                out_tokens: Optional[torch.Tensor] = None, out_cluster_ids: Optional[torch.Tensor] = None,
