@@ -144,6 +144,15 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     if constexpr (INT4) row_load_int4<NCH>(P.Crows + static_cast<size_t>(cw) * P.crow_bytes, d, q, sc);
     else row_load_bf16<NCH>(reinterpret_cast<const uint16_t*>(P.Crows + static_cast<size_t>(cw) * P.crow_bytes), d, w);
   }
+  // Phase 3 reads the chosen clusters' rows, scattered over all of Ecm: touch
+  // every 2 MB page of it once now (one L2 prefetch per page across the grid)
+  // so that their address translations are warm by then.
+  {
+    constexpr size_t kPage = size_t(2) << 20;
+    const size_t npages = (static_cast<size_t>(P.v) * d * 2 + kPage - 1) / kPage;
+    for (size_t pg = blockIdx.x + static_cast<size_t>(G) * tid; pg < npages; pg += static_cast<size_t>(G) * kThreads)
+      prefetch_l2(reinterpret_cast<const uint8_t*>(P.Ecm) + pg * kPage);
+  }
   // h, the uniforms and the head's workspace state may come from the preceding grid
   asm volatile("griddepcontrol.wait;" ::: "memory");
   if (tid == 0) {
