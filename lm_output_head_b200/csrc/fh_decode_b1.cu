@@ -649,9 +649,23 @@ cudaError_t launch_nch(const B1Params& P, int grid, size_t smem, int int4, cudaS
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  if (int4) return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, true>, P);
-  return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, false>, P);
+  // programmatic dependent launch with the cooperative attribute; if a driver
+  // refuses the pair, launch cooperatively alone from then on (the kernel's
+  // griddepcontrol instructions are no-ops without the attribute)
+  static bool pdl_ok = true;
+  cfg.numAttrs = pdl_ok ? 2 : 1;
+  auto go = [&]() {
+    return int4 ? cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, true>, P)
+                : cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, false>, P);
+  };
+  cudaError_t e = go();
+  if (e != cudaSuccess && cfg.numAttrs == 2 && e != cudaErrorLaunchOutOfResources) {
+    (void)cudaGetLastError();
+    pdl_ok = false;
+    cfg.numAttrs = 1;
+    e = go();
+  }
+  return e;
 }
 
 }  // namespace
