@@ -657,10 +657,24 @@ cudaError_t launch_nch(const B1Params& P, int grid, size_t smem, int cfmt, cudaS
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  if (cfmt == kFmtInt4) return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, kFmtInt4>, P);
-  if (cfmt == kFmtInt8) return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, kFmtInt8>, P);
-  return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, kFmtBf16>, P);
+  // programmatic dependent launch with the cooperative attribute; if a driver
+  // refuses the pair, launch cooperatively alone from then on (the kernel's
+  // griddepcontrol instructions are no-ops without the attribute)
+  static bool pdl_ok = true;
+  cfg.numAttrs = pdl_ok ? 2 : 1;
+  auto go = [&]() {
+    if (cfmt == kFmtInt4) return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, kFmtInt4>, P);
+    if (cfmt == kFmtInt8) return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, kFmtInt8>, P);
+    return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, kFmtBf16>, P);
+  };
+  cudaError_t e = go();
+  if (e != cudaSuccess && cfg.numAttrs == 2 && e != cudaErrorLaunchOutOfResources) {
+    (void)cudaGetLastError();
+    pdl_ok = false;
+    cfg.numAttrs = 1;
+    e = go();
+  }
+  return e;
 }
 
 }  // namespace
