@@ -249,3 +249,41 @@ def test_assign_at_the_llama_shape_has_no_blocking_pair(fh):
         assert rounds >= 1
     finally:
         cbl.close()
+
+
+def test_built_clusters_serve_as_a_head(fh):
+    """Cluster a planted vocabulary on the GPU, build a FlashHead from the result (E, C_out,
+    C2T_out) and decode: the tokens match the oracle's two-stage head on the same arrays."""
+    from lm_output_head_b200.cluster import ClusterBuilder
+    from tests import parity
+    bits, truth = _planted(15, noise=0.3)
+    rng = np.random.default_rng(16)
+    u = rng.uniform(size=C).astype(np.float32)
+    cbl = ClusterBuilder(V, D, C)
+    try:
+        E = fh.bf16_from_bits(bits, "cuda")
+        Cout, m, it = cbl.build(E, u_init=torch.from_numpy(u).cuda(), max_iter=100)
+        assert cbl.device_status() == 0
+    finally:
+        cbl.close()
+    head = synth.Head(v=V, d=D, c=C, b=B, E=bits, C=_bits(Cout), C2T=m.cpu().numpy())
+    assert oracle.check_c2t(head.C2T, V)
+    dh = fh.FlashHead(E, m, C=Cout, max_batch=4, max_probes=8)
+    try:
+        Hx = synth.to_bf16_bits((rng.standard_normal((8, D)) * 0.5).astype(np.float32))
+        rep = parity.Report()
+        for r in range(8):
+            tok = int(dh.decode(torch.from_numpy(Hx[r:r + 1].view(np.int16)).view(torch.bfloat16).cuda(), 8).item())
+            ids = torch.empty((1, 8), dtype=torch.int32, device="cuda")
+            dh.decode(torch.from_numpy(Hx[r:r + 1].view(np.int16)).view(torch.bfloat16).cuda(), 8,
+                      out_cluster_ids=ids)
+            Cw = oracle.centroid_matrix(head)
+            S = oracle.centroid_scores(Cw, Hx[r:r + 1])[0]
+            hw = oracle.widen_bf16(Hx[r])
+            rep.add(parity.check_cluster_set(ids.cpu().numpy()[0], S, 8, parity.loose_bound(Cw, hw),
+                                             parity.tight_bound(Cw, hw)))
+            rep.add(parity.check_greedy_token(head, Hx[r], ids.cpu().numpy()[0], tok))
+        assert rep.tight_mismatch == 0, rep
+        assert dh.device_status() == 0
+    finally:
+        dh.close()
