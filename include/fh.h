@@ -7,7 +7,7 @@
  * token_scores):
  *
  *   1. centroid scores  s = C h over c balanced clusters (section 1.2.2),
- *      C in bf16 or in INT4 with one bf16 scale per 32 elements
+ *      C in bf16, or in INT4 or INT8 with one bf16 scale per 32 elements
  *      (selective quantisation, section 1.2.4);
  *   2. probe selection: the p best clusters (multi-probe retrieval,
  *      section 1.2.2), or p clusters drawn by multinomial sampling at
@@ -65,7 +65,8 @@ typedef enum {
 
 typedef enum {
   FH_CENTROID_BF16 = 0,     /* C: bf16 [c, d] */
-  FH_CENTROID_INT4_G32 = 1  /* C_q: uint8 [c, d/2], C_scales: bf16 [c, d/32] */
+  FH_CENTROID_INT4_G32 = 1, /* C_q: uint8 [c, d/2], C_scales: bf16 [c, d/32] */
+  FH_CENTROID_INT8_G32 = 2  /* C_q: int8 [c, d], C_scales: bf16 [c, d/32] (W8A16) */
 } fh_centroid_format;
 
 typedef enum {
@@ -79,12 +80,15 @@ typedef enum {
  * cluster k, so slot k*b + j of the flattened map names one token).
  *
  *  v, d, c, b   vocabulary, hidden size, clusters, tokens per cluster;
- *               v == c*b, d % 8 == 0 (d % 32 == 0 for INT4), 1 <= c.
+ *               v == c*b, d % 8 == 0 (d % 32 == 0 for INT4 / INT8), 1 <= c.
  *  E            device bf16 [v, d], 16-byte aligned.
  *  C            device bf16 [c, d], 16-byte aligned (BF16 format, else NULL).
  *  C_q          device uint8 [c, d/2] (INT4 format): element 2i in the low
- *               nibble of byte i, 2i+1 in the high nibble, two's complement.
- *  C_scales     device bf16 [c, d/32] (INT4 format): value = code * scale.
+ *               nibble of byte i, 2i+1 in the high nibble, two's complement;
+ *               or device int8 [c, d] (INT8 format): one two's-complement
+ *               byte per element (the W8A16 row of the write-up's parameter
+ *               table, section 5.2).
+ *  C_scales     device bf16 [c, d/32] (INT4 and INT8 formats): value = code * scale.
  *  C2T          device int32 [c, b].
  *  fmt          fh_centroid_format.
  *  max_batch    largest B any call will pass (>= 1).
@@ -110,9 +114,9 @@ typedef struct fh_head fh_head;
  * workspace, and fills two library-owned copies inside it: the token rows of
  * E in cluster-major order (row k*b + j = E[C2T[k][j]], v*d*2 bytes; a
  * cluster's b rows are one contiguous block, read without a C2T lookup), and,
- * for INT4, each centroid row packed with its scales (row = d/2 code bytes,
- * then d/16 scale bytes, padded to 16 bytes) so that one bulk copy moves a
- * row. Synchronises `stream`. On success *out owns the workspace; release it
+ * for INT4 / INT8, each centroid row packed with its scales (row = d/2 or
+ * d code bytes, then d/16 scale bytes, padded to 16 bytes) so that one bulk
+ * copy moves a row. Synchronises `stream`. On success *out owns the workspace; release it
  * with fh_destroy. E itself is still read by the dense head.
  */
 fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out);
@@ -122,7 +126,7 @@ void fh_destroy(fh_head* head);
 
 /*
  * Stage 1 (write-up section 1.2.2): scores[r][k] = sum_i C[k][i] * hidden[r][i]
- * for r < B, k < c (INT4: C dequantised exactly, code * scale).
+ * for r < B, k < c (INT4 / INT8: C dequantised exactly, code * scale).
  *  hidden  device bf16 [B, d], 16-byte aligned.
  *  scores  device fp32 [B, c].
  */
@@ -250,6 +254,44 @@ typedef enum {
   FH_QUERY_LAST_FULL = 5
 } fh_query_key;
 fh_status fh_query(fh_head* head, int32_t key, int64_t* value);
+
+/*
+ * Speculative drafting (write-up section 4.2): check FlashHead draft tokens
+ * against the dense head. For row r, p = softmax(z/T) over the vocabulary
+ * (z = logits[r], the dense head's logits) and q = softmax(z/T) over the
+ * draft's candidate tokens cand_tokens[r][0..n) (the tokens of the clusters
+ * it was drawn from, e.g. fh_candidate_logits' token ids). The draft x =
+ * draft[r] is kept when u_accept[r] < p(x) / q(x); otherwise the token is the
+ * inverse-CDF draw (token id order) at u_resample[r] from max(0, p - q). For
+ * every cluster set the result follows p exactly (standard speculative
+ * sampling with the draft law taken given the chosen clusters).
+ *  logits       device fp32 [B, v].
+ *  cand_tokens  device int32 [B, n], distinct ids in [0, v) per row.
+ *  draft        device int32 [B], one of the row's candidates.
+ *  u_accept, u_resample  device fp32 [B], uniforms in [0, 1).
+ *  out_tokens   device int32 [B]; -1 and FH_ERR_OUT_OF_RANGE in the device
+ *               status when a candidate or the draft is out of range or the
+ *               draft is not a candidate.
+ * FH_ERR_UNSUPPORTED when the candidate bitmap (v bits) exceeds shared memory.
+ */
+fh_status fh_speculative_verify(fh_head* head, const float* logits, const int32_t* cand_tokens, int32_t n,
+                                int32_t B, const int32_t* draft, float T, const float* u_accept,
+                                const float* u_resample, int32_t* out_tokens, fh_stream_t stream);
+
+/*
+ * Adaptive probe count (write-up section 1.2.2, "dynamic adjustment"; section
+ * 4.2: fewer probes for frequent tokens). For each row r of scores, out_p[r]
+ * = the smallest p in [p_min, p_max] whose top-p clusters hold at least a
+ * fraction tau of softmax(scores[r] / T) over all c clusters (the mass of the
+ * top p depends only on the p largest scores, not on the order of ties).
+ * Use it with fh_decode / fh_select_clusters row by row.
+ *  scores  device fp32 [B, c] (fh_centroid_scores' output).
+ *  out_p   device int32 [B].
+ * 0 < tau <= 1, 1 <= p_min <= p_max <= c, T finite and > 0.
+ * FH_ERR_UNSUPPORTED when a row's scores (next power of two of c, fp32) exceed shared memory.
+ */
+fh_status fh_adaptive_probes(fh_head* head, const float* scores, int32_t B, float tau, int32_t p_min,
+                             int32_t p_max, float T, int32_t* out_p, fh_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -6,6 +6,7 @@ end-to-end path from pinned host memory. There is no CPU fallback: if the
 library is missing, constructing a head raises ImportError.
 """
 from ._lib import FlashHeadError, load  # noqa: F401
-from .head import FlashHead, HostDecoder, bf16_from_bits, dense_head_noalloc  # noqa: F401
+from .head import FlashHead, HostDecoder, bf16_from_bits, dense_head_noalloc, speculative_verify  # noqa: F401
 
-__all__ = ["FlashHead", "FlashHeadError", "HostDecoder", "bf16_from_bits", "dense_head_noalloc", "load"]
+__all__ = ["FlashHead", "FlashHeadError", "HostDecoder", "bf16_from_bits", "dense_head_noalloc", "load",
+           "speculative_verify"]

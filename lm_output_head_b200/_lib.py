@@ -22,6 +22,7 @@ FH_ERR_TIMEOUT = 7
 
 FH_CENTROID_BF16 = 0
 FH_CENTROID_INT4_G32 = 1
+FH_CENTROID_INT8_G32 = 2
 FH_GREEDY = 0
 FH_SAMPLE_GUMBEL = 1
 
@@ -36,7 +37,8 @@ FH_QUERY_LAST_FULL = 5
 EXPORTED = (
     "fh_create", "fh_destroy", "fh_centroid_scores", "fh_select_clusters",
     "fh_candidate_logits", "fh_decode", "fh_dense_head", "fh_get_device_status",
-    "fh_status_string", "fh_set_spin_budget", "fh_query", "fh_dense_head_noalloc",
+    "fh_status_string", "fh_set_spin_budget", "fh_query", "fh_dense_head_noalloc", "fh_speculative_verify",
+    "fh_adaptive_probes",
     # include/fh_cluster.h
     "fh_cluster_create", "fh_cluster_destroy", "fh_cluster_normalize", "fh_cluster_seed",
     "fh_cluster_gather", "fh_cluster_similarities", "fh_cluster_assign", "fh_cluster_update",
@@ -98,6 +100,10 @@ def load() -> ctypes.CDLL:
     lib.fh_set_spin_budget.restype = ctypes.c_int
     lib.fh_query.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_int64)]
     lib.fh_query.restype = ctypes.c_int
+    lib.fh_speculative_verify.argtypes = [vp, vp, vp, i32, i32, vp, f32, vp, vp, vp, vp]
+    lib.fh_speculative_verify.restype = ctypes.c_int
+    lib.fh_adaptive_probes.argtypes = [vp, vp, i32, f32, i32, i32, f32, vp, vp]
+    lib.fh_adaptive_probes.restype = ctypes.c_int
     pi32 = ctypes.POINTER(ctypes.c_int32)
     lib.fh_cluster_create.argtypes = [i32, i32, i32, vp, ctypes.POINTER(vp)]
     lib.fh_cluster_destroy.argtypes = [vp]

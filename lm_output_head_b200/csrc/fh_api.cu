@@ -14,7 +14,7 @@ cudaError_t set_attrs_decode_b1(int max_smem);
 cudaError_t set_attrs_batched(int max_smem);
 cudaError_t set_attrs_dense(int max_smem);
 int dense_max_rows();
-cudaError_t occupancy_decode_b1(int int4, int nch, size_t smem, int* blocks);
+cudaError_t occupancy_decode_b1(int cfmt, int nch, size_t smem, int* blocks);
 size_t decode_b1_misc_bytes();
 size_t decode_b1_scratch_bytes(int c, int list_cap);
 cudaError_t occupancy_dense(int nch, size_t smem, int* blocks);
@@ -54,7 +54,7 @@ struct fh_head {
   int words = 0;
   int b1_grid = 0;
   int dense_grid = 0;
-  const uint8_t* crows = nullptr;      // centroid rows (bf16 borrowed, or packed INT4 in ws)
+  const uint8_t* crows = nullptr;      // centroid rows (bf16 borrowed, or packed INT4 / INT8 in ws)
   int crow_bytes = 0;
   int nch = 0;
   long long spin_budget = kDefaultSpinBudget;
@@ -133,7 +133,7 @@ fh_status launch_scores_rows(fh_head* h, const void* hidden, int32_t B, int mode
     P.off_ring = static_cast<int>(off_ring);
     P.off_h = static_cast<int>(off_ring + ring);
     const size_t smem = off_ring + ring + up(rows * row_bytes, 128);
-    cudaError_t e = launch_scores(P, h->num_sms, smem, D.fmt == FH_CENTROID_INT4_G32, h->nch, st);
+    cudaError_t e = launch_scores(P, h->num_sms, smem, D.fmt, h->nch, st);
     if (e != cudaSuccess) return cuda_fail(e);
   }
   return FH_OK;
@@ -179,7 +179,7 @@ fh_status launch_gemm_rows(fh_head* h, const void* hidden, int32_t B, int epi, i
                            float* out, cudaStream_t st) {
   const fh_head_desc& D = h->desc;
   const bool centroids = epi == 0;
-  const bool int4 = centroids && D.fmt == FH_CENTROID_INT4_G32;
+  const int cfmt = centroids ? D.fmt : kFmtBf16;  // packed INT4 / INT8 centroid rows, or bf16 rows
   const int rows = centroids ? D.c : D.v;
   const long long ldo = rows;
   for (int r0 = 0; r0 < B; r0 += 256) {
@@ -187,7 +187,7 @@ fh_status launch_gemm_rows(fh_head* h, const void* hidden, int32_t B, int epi, i
     P.rows = rows;
     P.d = D.d;
     P.nb = std::min(256, B - r0);
-    P.int4 = int4 ? 1 : 0;
+    P.cfmt = cfmt;
     P.epi = epi;
     P.mode = mode;
     P.T = T;
@@ -198,7 +198,7 @@ fh_status launch_gemm_rows(fh_head* h, const void* hidden, int32_t B, int epi, i
     P.u = u ? u + static_cast<size_t>(r0) * ldo : nullptr;
     P.best = h->best + r0;
     P.status = &h->sync->status;
-    const void* A = centroids ? (int4 ? nullptr : D.C) : D.E;
+    const void* A = centroids ? (cfmt != kFmtBf16 ? nullptr : D.C) : D.E;
     const void* H = static_cast<const uint16_t*>(hidden) + static_cast<size_t>(r0) * D.d;
     cudaError_t e = launch_gemm(P, A, H, h->num_sms, st);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -239,7 +239,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   if (!D.E || !aligned(D.E, 16) || !D.C2T || !aligned(D.C2T, 4)) return FH_ERR_INVALID_ARG;
   if (D.fmt == FH_CENTROID_BF16) {
     if (!D.C || !aligned(D.C, 16)) return FH_ERR_INVALID_ARG;
-  } else if (D.fmt == FH_CENTROID_INT4_G32) {
+  } else if (D.fmt == FH_CENTROID_INT4_G32 || D.fmt == FH_CENTROID_INT8_G32) {
     if (D.d % 32 || !D.C_q || !D.C_scales || !aligned(D.C_scales, 2)) return FH_ERR_INVALID_ARG;
   } else {
     return FH_ERR_INVALID_ARG;
@@ -265,6 +265,8 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   h->nch = nch_for(D.d);
   if (D.fmt == FH_CENTROID_INT4_G32) {
     h->crow_bytes = static_cast<int>(up(static_cast<size_t>(D.d) / 2 + static_cast<size_t>(D.d) / 16, 16));
+  } else if (D.fmt == FH_CENTROID_INT8_G32) {
+    h->crow_bytes = static_cast<int>(up(static_cast<size_t>(D.d) + static_cast<size_t>(D.d) / 16, 16));
   } else {
     h->crow_bytes = D.d * 2;
   }
@@ -300,7 +302,8 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   const int list_cap = static_cast<int>(std::min<size_t>(4 * mp, D.c));
   const size_t o_lkey = take(static_cast<size_t>(list_cap) * 4);
   const size_t o_lid = take(static_cast<size_t>(list_cap) * 4);
-  const size_t o_crow = D.fmt == FH_CENTROID_INT4_G32 ? take(static_cast<size_t>(D.c) * h->crow_bytes) : 0;
+  const bool packed = D.fmt != FH_CENTROID_BF16;
+  const size_t o_crow = packed ? take(static_cast<size_t>(D.c) * h->crow_bytes) : 0;
   h->ws_bytes = off;
 
   const char* cap = std::getenv("FH_TEST_WORKSPACE_LIMIT");
@@ -335,7 +338,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   h->b1_list_id = reinterpret_cast<int32_t*>(h->ws + o_lid);
   h->b1_list_cap = list_cap;
   h->words = words;
-  h->crows = D.fmt == FH_CENTROID_INT4_G32 ? h->ws + o_crow : static_cast<const uint8_t*>(D.C);
+  h->crows = packed ? h->ws + o_crow : static_cast<const uint8_t*>(D.C);
 
   fh_status status = FH_OK;
   do {
@@ -360,9 +363,10 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
     C2TCheckParams cp{D.C2T, h->c2t_counts, &h->sync->status, static_cast<long long>(D.v), D.v};
     e = launch_c2t_check(cp, st);
     if (e != cudaSuccess) { status = cuda_fail(e); break; }
-    if (D.fmt == FH_CENTROID_INT4_G32) {
-      RepackParams rp{D.C_q, static_cast<const uint16_t*>(D.C_scales), h->ws + o_crow, D.c, D.d, h->crow_bytes};
-      e = launch_repack_int4(rp, st);
+    if (packed) {
+      RepackParams rp{D.C_q, static_cast<const uint16_t*>(D.C_scales), h->ws + o_crow, D.c, D.d, h->crow_bytes,
+                      D.fmt == FH_CENTROID_INT8_G32 ? D.d : D.d / 2};
+      e = launch_repack(rp, st);
       if (e != cudaSuccess) { status = cuda_fail(e); break; }
     }
     int bad = 0;
@@ -396,7 +400,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
     o += std::max(static_cast<size_t>(kWarps) * h->b1_slot_bytes, decode_b1_scratch_bytes(D.c, h->b1_list_cap));
     h->b1_smem = o;
     int blocks = 0;
-    e = occupancy_decode_b1(D.fmt == FH_CENTROID_INT4_G32, h->nch, h->b1_smem, &blocks);
+    e = occupancy_decode_b1(D.fmt, h->nch, h->b1_smem, &blocks);
     (void)cudaGetLastError();
     const int per_sm = e == cudaSuccess ? std::min(blocks, 2) : 0;
     h->b1_grid = per_sm * h->num_sms;
@@ -572,7 +576,7 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
     P.off_slots = h->b1_off_slots;
     P.slot_bytes = h->b1_slot_bytes;
     P.spin_budget = h->spin_budget;
-    cudaError_t e = launch_decode_b1(P, h->b1_grid, h->b1_smem, D.fmt == FH_CENTROID_INT4_G32, h->nch, st);
+    cudaError_t e = launch_decode_b1(P, h->b1_grid, h->b1_smem, D.fmt, h->nch, st);
     return e == cudaSuccess ? FH_OK : cuda_fail(e);
   }
 
@@ -679,6 +683,34 @@ fh_status fh_dense_head(fh_head* h, const void* hidden, int32_t B, float* logits
     if (e != cudaSuccess) return cuda_fail(e);
   }
   return FH_OK;
+}
+
+fh_status fh_speculative_verify(fh_head* h, const float* logits, const int32_t* cand_tokens, int32_t n, int32_t B,
+                                const int32_t* draft, float T, const float* u_accept, const float* u_resample,
+                                int32_t* out_tokens, fh_stream_t stream) {
+  if (!h || !logits || !cand_tokens || !draft || !u_accept || !u_resample || !out_tokens) return FH_ERR_INVALID_ARG;
+  if (B < 1 || n < 1 || n > h->desc.v || !(T > 0.f && T < 3.0e38f)) return FH_ERR_INVALID_ARG;
+  cudaError_t e = launch_spec_verify(logits, h->desc.v, cand_tokens, n, B, draft, T, u_accept, u_resample, out_tokens,
+                                     &h->sync->status, reinterpret_cast<cudaStream_t>(stream));
+  if (e == cudaErrorInvalidValue) {
+    (void)cudaGetLastError();
+    return FH_ERR_UNSUPPORTED;
+  }
+  return e == cudaSuccess ? FH_OK : cuda_fail(e);
+}
+
+fh_status fh_adaptive_probes(fh_head* h, const float* scores, int32_t B, float tau, int32_t p_min, int32_t p_max,
+                             float T, int32_t* out_p, fh_stream_t stream) {
+  if (!h || !scores || !out_p || B < 1) return FH_ERR_INVALID_ARG;
+  if (!(tau > 0.f && tau <= 1.f) || p_min < 1 || p_min > p_max || p_max > h->desc.c) return FH_ERR_INVALID_ARG;
+  if (!(T > 0.f && T < 3.0e38f)) return FH_ERR_INVALID_ARG;
+  cudaError_t e = launch_adaptive_probes(scores, B, h->desc.c, tau, p_min, p_max, T, out_p,
+                                         reinterpret_cast<cudaStream_t>(stream));
+  if (e == cudaErrorInvalidValue) {
+    (void)cudaGetLastError();
+    return FH_ERR_UNSUPPORTED;
+  }
+  return e == cudaSuccess ? FH_OK : cuda_fail(e);
 }
 
 }  // extern "C"

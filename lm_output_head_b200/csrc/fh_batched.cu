@@ -25,7 +25,7 @@ namespace {
 // ----------------------------------------------------------------------------
 // stage 1 for a block of rows
 // ----------------------------------------------------------------------------
-template <int NCH, bool INT4>
+template <int NCH, int FMT>
 __global__ void __launch_bounds__(kThreads, 1) scores_kernel(const ScoresParams P) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -53,7 +53,47 @@ __global__ void __launch_bounds__(kThreads, 1) scores_kernel(const ScoresParams 
     P.out[o] = key;
   };
   bool ok;
-  if constexpr (INT4) {
+  if constexpr (FMT == kFmtInt8) {
+    // packed INT8 row: chunk m of lane l = the 8 codes of elements (l + 32 m) * 8 .. + 8
+    auto use = [&](int i, uint32_t slot) {
+      const int k = gw + i * W;
+      uint2 q[NCH];
+      float sc[NCH];
+#pragma unroll
+      for (int m = 0; m < NCH; ++m) {
+        const int e = (lane + 32 * m) * 8;
+        q[m] = make_uint2(0u, 0u);
+        sc[m] = 0.f;
+        if (e < d) {
+          q[m] = lds64(slot + static_cast<uint32_t>(e));
+          sc[m] = bf16f(lds16(slot + static_cast<uint32_t>(d + 2 * (e >> 5))));
+        }
+      }
+      for (int r = 0; r < R; ++r) {
+        const uint32_t hrow = sh_a + static_cast<uint32_t>(r * d * 2);
+        float acc = 0.f;
+#pragma unroll
+        for (int m = 0; m < NCH; ++m) {
+          const int e = (lane + 32 * m) * 8;
+          if (e < d) {
+            const uint4 hv = lds128(hrow + 2u * e);
+            float part = sbyte(q[m].x, 0) * bf16lo(hv.x);
+            part = fmaf(sbyte(q[m].x, 1), bf16hi(hv.x), part);
+            part = fmaf(sbyte(q[m].x, 2), bf16lo(hv.y), part);
+            part = fmaf(sbyte(q[m].x, 3), bf16hi(hv.y), part);
+            part = fmaf(sbyte(q[m].y, 0), bf16lo(hv.z), part);
+            part = fmaf(sbyte(q[m].y, 1), bf16hi(hv.z), part);
+            part = fmaf(sbyte(q[m].y, 2), bf16lo(hv.w), part);
+            part = fmaf(sbyte(q[m].y, 3), bf16hi(hv.w), part);
+            acc = fmaf(sc[m], part, acc);
+          }
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) emit(r, k, acc);
+      }
+    };
+    ok = warp_stream(n, P.nslot, ring_w, P.slot_bytes, bar_w, phase_bits, kWaitBudget, src, use);
+  } else if constexpr (FMT == kFmtInt4) {
     constexpr int NQ = (NCH + 1) / 2;
     auto use = [&](int i, uint32_t slot) {
       const int k = gw + i * W;
@@ -397,10 +437,11 @@ __global__ void __launch_bounds__(kThreads, 1) epilogue_kernel(const EpiloguePar
     default: return cudaErrorInvalidValue; \
   }
 
-cudaError_t launch_scores(const ScoresParams& P, int grid, size_t smem, int int4, int nch, cudaStream_t st) {
+cudaError_t launch_scores(const ScoresParams& P, int grid, size_t smem, int cfmt, int nch, cudaStream_t st) {
 #define FH_L(N)                                                                          \
-  if (int4) scores_kernel<N, true><<<grid, kThreads, smem, st>>>(P);                      \
-  else scores_kernel<N, false><<<grid, kThreads, smem, st>>>(P);                          \
+  if (cfmt == kFmtInt4) scores_kernel<N, kFmtInt4><<<grid, kThreads, smem, st>>>(P);      \
+  else if (cfmt == kFmtInt8) scores_kernel<N, kFmtInt8><<<grid, kThreads, smem, st>>>(P); \
+  else scores_kernel<N, kFmtBf16><<<grid, kThreads, smem, st>>>(P);                       \
   return cudaGetLastError();
   FH_DISPATCH_NCH(nch, FH_L)
 #undef FH_L
@@ -435,8 +476,9 @@ cudaError_t set_attrs_batched(int max_smem) {
     if (e == cudaSuccess) e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
   };
 #define FH_S(N)                                                   \
-  set(reinterpret_cast<const void*>(scores_kernel<N, true>));     \
-  set(reinterpret_cast<const void*>(scores_kernel<N, false>));    \
+  set(reinterpret_cast<const void*>(scores_kernel<N, kFmtBf16>)); \
+  set(reinterpret_cast<const void*>(scores_kernel<N, kFmtInt4>)); \
+  set(reinterpret_cast<const void*>(scores_kernel<N, kFmtInt8>)); \
   set(reinterpret_cast<const void*>(candidates_kernel<N>));
   FH_S(1) FH_S(2) FH_S(3) FH_S(4) FH_S(5) FH_S(6) FH_S(8) FH_S(10)
 #undef FH_S

@@ -14,7 +14,9 @@
 //    centres as the M operand in chunks of 256, the token rows streamed.
 //  - the balanced assignment in rounds of proposals: propose_kernel (every
 //    unassigned token picks its best cluster among those whose b-th held
-//    pair it beats), a CSR of the proposals by cluster, accept_kernel (one
+//    pair it beats, from a per-token shortlist of its 16 best clusters kept
+//    by the first round, else from its whole column), a CSR of the
+//    proposals by cluster, accept_kernel (one
 //    warp per cluster keeps the best b of its held tokens and proposers with
 //    a 32-lane bitonic merge). Under one strict order of all (token,
 //    cluster) pairs -- similarity desc, token asc, cluster asc -- the
@@ -43,6 +45,7 @@ constexpr int kSeedBlocks = 1024;  // row blocks of the seeding sums (one per pi
 constexpr int kMaxB = 32;          // a cluster's held list lives in one warp
 constexpr int kMaxDC = 8192;       // update_kernel keeps d / 256 chunks of 8 per thread
 constexpr int kUpdChunks = kMaxDC / (kCT * 8);
+constexpr int kShort = 16;         // per-token shortlist of its best clusters
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(a));
@@ -262,6 +265,9 @@ struct AssignParams {
   uint32_t* cur;        // [c]
   int32_t* list;        // [v] proposers grouped by cluster
   int32_t* unassigned;
+  float* sl_s;          // [kShort, v] every token's best clusters (similarity desc, cluster asc)
+  int32_t* sl_k;        //   INT_MAX past the end when c < kShort
+  int32_t* sl_pos;      // [v] first shortlist entry not yet ruled out
   int* status;
   int v, c, b;
 };
@@ -281,8 +287,67 @@ __global__ void __launch_bounds__(kCT) assign_init_kernel(AssignParams P) {
   if (i == 0) *P.unassigned = P.v;
 }
 
+// First round (every cluster has room): every token proposes to its best
+// cluster and keeps its kShort best (similarity desc, cluster asc) as a
+// shortlist, so that later rounds rarely read its whole column again.
+__global__ void __launch_bounds__(kCT) propose_first_kernel(AssignParams P) {
+  const int lane = threadIdx.x & 31;
+  const int nw = gridDim.x * (kCT / 32);
+  const int ngroups = (P.v + 31) / 32;
+  for (int g = blockIdx.x * (kCT / 32) + (threadIdx.x >> 5); g < ngroups; g += nw) {
+    const int t = g * 32 + lane;
+    const bool valid = t < P.v;
+    const int tc = valid ? t : P.v - 1;  // keep the loads in bounds
+    float ls[kShort];
+    int lk[kShort];
+#pragma unroll
+    for (int i = 0; i < kShort; ++i) {
+      ls[i] = -INFINITY;
+      lk[i] = INT_MAX;
+    }
+    for (int k = 0; k < P.c; ++k) {
+      const float s = __ldg(P.S + static_cast<size_t>(k) * P.v + tc);
+      if (s > ls[kShort - 1]) {  // k ascending: an equal similarity stays below the earlier cluster
+#pragma unroll
+        for (int i = kShort - 1; i > 0; --i) {
+          if (s > ls[i - 1]) {
+            ls[i] = ls[i - 1];
+            lk[i] = lk[i - 1];
+          } else if (s > ls[i]) {
+            ls[i] = s;
+            lk[i] = k;
+          }
+        }
+        if (s > ls[0]) {
+          ls[0] = s;
+          lk[0] = k;
+        }
+      }
+    }
+    if (valid) {
+#pragma unroll
+      for (int i = 0; i < kShort; ++i) {
+        P.sl_s[static_cast<size_t>(i) * P.v + t] = ls[i];
+        P.sl_k[static_cast<size_t>(i) * P.v + t] = lk[i];
+      }
+      P.sl_pos[t] = 0;
+      if (lk[0] == INT_MAX) {
+        record_error(P.status, FH_ERR_OUT_OF_RANGE);  // only non-finite similarities get here
+        P.prop_k[t] = -1;
+      } else {
+        P.prop_k[t] = lk[0];
+        P.prop_s[t] = ls[0];
+        atomicAdd(P.cnt + lk[0], 1u);
+      }
+    }
+  }
+}
+
 // Every unassigned token proposes to its best cluster (similarity desc,
-// cluster asc) among those that would not reject it at the round's start.
+// cluster asc) among those that would not reject it at the round's start:
+// the first shortlist entry still eligible (clusters only ever raise their
+// bar, so an entry ruled out once stays out, and every cluster outside the
+// shortlist ranks below all of it), else the best of its whole column.
 __global__ void __launch_bounds__(kCT) propose_kernel(AssignParams P) {
   const int lane = threadIdx.x & 31;
   const int nw = gridDim.x * (kCT / 32);
@@ -295,25 +360,46 @@ __global__ void __launch_bounds__(kCT) propose_kernel(AssignParams P) {
     const int tc = valid ? t : P.v - 1;  // keep the loads in bounds
     float bs = -INFINITY;
     int bk = -1;
-    int k = 0;
-    for (; k + 4 <= P.c; k += 4) {
-      float s[4];
-      int2 th[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        s[q] = __ldg(P.S + static_cast<size_t>(k + q) * P.v + tc);
-        th[q] = __ldg(P.thr + k + q);
+    if (active) {
+      int j = P.sl_pos[t];
+      for (; j < kShort; ++j) {
+        const int k = P.sl_k[static_cast<size_t>(j) * P.v + t];
+        if (k == INT_MAX) {
+          j = kShort;
+          break;
+        }
+        const float s = P.sl_s[static_cast<size_t>(j) * P.v + t];
+        const int2 th = __ldg(P.thr + k);
+        if (better(s, t, __int_as_float(th.x), th.y)) {
+          bs = s;
+          bk = k;
+          break;
+        }
       }
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const bool elig = better(s[q], t, __int_as_float(th[q].x), th[q].y);
-        if (elig && (bk < 0 || s[q] > bs)) { bs = s[q]; bk = k + q; }
-      }
+      P.sl_pos[t] = j;
     }
-    for (; k < P.c; ++k) {
-      const float s = __ldg(P.S + static_cast<size_t>(k) * P.v + tc);
-      const int2 th = __ldg(P.thr + k);
-      if (better(s, t, __int_as_float(th.x), th.y) && (bk < 0 || s > bs)) { bs = s; bk = k; }
+    const bool scan = active && bk < 0;  // shortlist exhausted: the whole column
+    if (__any_sync(0xFFFFFFFFu, scan)) {
+      int k = 0;
+      for (; k + 4 <= P.c; k += 4) {
+        float s[4];
+        int2 th[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          s[q] = __ldg(P.S + static_cast<size_t>(k + q) * P.v + tc);
+          th[q] = __ldg(P.thr + k + q);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const bool elig = better(s[q], t, __int_as_float(th[q].x), th[q].y);
+          if (scan && elig && (bk < 0 || s[q] > bs)) { bs = s[q]; bk = k + q; }
+        }
+      }
+      for (; k < P.c; ++k) {
+        const float s = __ldg(P.S + static_cast<size_t>(k) * P.v + tc);
+        const int2 th = __ldg(P.thr + k);
+        if (scan && better(s, t, __int_as_float(th.x), th.y) && (bk < 0 || s > bs)) { bs = s; bk = k; }
+      }
     }
     if (active) {
       if (bk < 0) {
@@ -589,7 +675,8 @@ fh_status run_assign(fh_cluster* cl, const float* S, int32_t* assign, int32_t* C
     if (++r > max_rounds) return FH_ERR_TIMEOUT;
     e = cudaMemsetAsync(P.cnt, 0, sizeof(uint32_t) * cl->c, st);
     if (e != cudaSuccess) return fail(e);
-    propose_kernel<<<gw, kCT, 0, st>>>(P);
+    if (r == 1) propose_first_kernel<<<gw, kCT, 0, st>>>(P);
+    else propose_kernel<<<gw, kCT, 0, st>>>(P);
     assign_scan_kernel<<<1, kPickThreads, 0, st>>>(P);
     assign_fill_kernel<<<gv, kCT, 0, st>>>(P);
     accept_kernel<<<gc, kCT, 0, st>>>(P);
@@ -704,6 +791,9 @@ fh_status fh_cluster_create(int32_t v, int32_t d, int32_t c, fh_stream_t stream,
   const size_t o_d2 = take(V * 4);
   const size_t o_part = take(kSeedBlocks * 8);
   const size_t o_taken = take(V);
+  const size_t o_sls = take(V * kShort * 4);
+  const size_t o_slk = take(V * kShort * 4);
+  const size_t o_slp = take(V * 4);
   cl->ws_bytes = off;
   e = cudaMalloc(&cl->ws, cl->ws_bytes);
   if (e != cudaSuccess) {
@@ -734,6 +824,9 @@ fh_status fh_cluster_create(int32_t v, int32_t d, int32_t c, fh_stream_t stream,
   A.cur = reinterpret_cast<uint32_t*>(w + o_cur);
   A.list = reinterpret_cast<int32_t*>(w + o_list);
   A.unassigned = words + 2;
+  A.sl_s = reinterpret_cast<float*>(w + o_sls);
+  A.sl_k = reinterpret_cast<int32_t*>(w + o_slk);
+  A.sl_pos = reinterpret_cast<int32_t*>(w + o_slp);
   A.status = cl->status;
   A.v = v; A.c = c; A.b = b;
   SeedParams& Sd = cl->Sd;

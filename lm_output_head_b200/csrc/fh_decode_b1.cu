@@ -6,7 +6,7 @@
 // The pages' pipeline (FlashHead write-up, section 2.2.2: h -> centroid_scores
 // -> top_p_clusters -> token_scores) runs as phases of one kernel:
 //
-//  1. centroid scores (section 1.2.2; INT4 centroids per section 1.2.4):
+//  1. centroid scores (section 1.2.2; INT4 or INT8 centroids per section 1.2.4):
 //     cluster k belongs to CTA k mod G (warp (k / G) mod 16), so every CTA
 //     owns c/G clusters. A warp's first row streams into registers, its
 //     second into a shared-memory slot by one bulk copy, both requested at
@@ -82,7 +82,7 @@ struct B1Misc {
   uint32_t bkey;
   int32_t bid;
   float edge_2p;
-  uint32_t nnote, base, nlist;
+  uint32_t nnote, base, prior_n;
   int32_t note_k[kNoteMax];
   uint32_t note_key[kNoteMax];
 };
@@ -102,8 +102,9 @@ __device__ __forceinline__ int region_bin(float key, float L, float S) {
   return x >= static_cast<float>(kB1Bins - 1) ? kB1Bins - 1 : static_cast<int>(x);
 }
 
-template <int NCH, bool INT4>
+template <int NCH, int FMT>
 __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P) {
+  constexpr bool INT4 = FMT == kFmtInt4, INT8 = FMT == kFmtInt8;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = gridDim.x;
@@ -115,7 +116,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   B1Misc* misc = reinterpret_cast<B1Misc*>(smem + P.off_misc);
   uint8_t* slots = smem + P.off_slots;  // per-warp row slots; the selection's scratch between phases
 
-  const uint32_t epoch = P.sync->epoch;  // calls on one head are stream-ordered
   FH_TL(0);
 
   // ---------------- phase 1: centroid scores ----------------
@@ -123,17 +123,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   const uint32_t wbar = smem_addr(&misc->wbar[warp]);
   const uint32_t slot = smem_addr(slots) + static_cast<uint32_t>(warp * P.slot_bytes);
   uint16_t* hraw = reinterpret_cast<uint16_t*>(hs + d / 2);
-  if (tid == 0) {
-    mbar_init(hbar, 1);
-    fence_mbar_init();
-    mbar_expect_tx(hbar, static_cast<uint32_t>(d * 2));
-    bulk_g2s(smem_addr(hraw), P.hidden, static_cast<uint32_t>(d * 2), hbar);
-    misc->nnote = 0u;
-  }
   const int cw = static_cast<int>(blockIdx.x) + G * warp;  // first cluster of this warp
   const int cstride = G * kWarps;
   const int n1 = cw < P.c ? (P.c - 1 - cw) / cstride + 1 : 0;  // <= 32 (host-checked)
   uint32_t wphase = 0;  // parity of this warp's slot barrier
+  // The centroid rows depend on no earlier kernel: the warp's first two start
+  // streaming before the wait for the preceding grid (programmatic dependent
+  // launch), which may still be finishing when this grid starts.
   if (lane == 0) {
     mbar_init(wbar, 1);
     fence_mbar_init();
@@ -145,9 +141,30 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   }
   uint4 w[NCH];
   uint32_t q[NCH], sc[NCH];
+  uint2 q8[NCH];
+  uint32_t sw8[int8_scale_words<NCH>()];
   if (n1 > 0) {
     if constexpr (INT4) row_load_int4<NCH>(P.Crows + static_cast<size_t>(cw) * P.crow_bytes, d, q, sc);
+    else if constexpr (INT8) row_load_int8<NCH>(P.Crows + static_cast<size_t>(cw) * P.crow_bytes, d, q8, sw8);
     else row_load_bf16<NCH>(reinterpret_cast<const uint16_t*>(P.Crows + static_cast<size_t>(cw) * P.crow_bytes), d, w);
+  }
+  // Phase 3 reads the chosen clusters' rows, scattered over all of Ecm: touch
+  // every 2 MB page of it once now (one L2 prefetch per page across the grid)
+  // so that their address translations are warm by then.
+  {
+    constexpr size_t kPage = size_t(2) << 20;
+    const size_t npages = (static_cast<size_t>(P.v) * d * 2 + kPage - 1) / kPage;
+    for (size_t pg = blockIdx.x + static_cast<size_t>(G) * tid; pg < npages; pg += static_cast<size_t>(G) * kThreads)
+      prefetch_l2(reinterpret_cast<const uint8_t*>(P.Ecm) + pg * kPage);
+  }
+  // h, the uniforms and the head's workspace state may come from the preceding grid
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (tid == 0) {
+    mbar_init(hbar, 1);
+    fence_mbar_init();
+    mbar_expect_tx(hbar, static_cast<uint32_t>(d * 2));
+    bulk_g2s(smem_addr(hraw), P.hidden, static_cast<uint32_t>(d * 2), hbar);
+    misc->nnote = 0u;
   }
   float ureg = 0.f;  // lane j holds u of item j
   if (gumbel && lane < n1) ureg = __ldg(P.u_clusters + cw + lane * cstride);
@@ -203,10 +220,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
       if (!mbar_wait_bounded(wbar, wphase, kWaitBudget) && lane == 0) record_error(&P.sync->status, FH_ERR_TIMEOUT);
       wphase ^= 1u;
       if constexpr (INT4) s = srow_dot_int4_hs<NCH>(slot, hs, d);
+      else if constexpr (INT8) s = srow_dot_int8_hs<NCH>(slot, hs, d);
       else s = srow_dot_bf16_hs<NCH>(slot, hs, d);
     } else if constexpr (INT4) {
       if (i > 0) row_load_int4<NCH>(P.Crows + static_cast<size_t>(k) * P.crow_bytes, d, q, sc);
       s = row_dot_int4_hs<NCH>(q, sc, hs, d);
+    } else if constexpr (INT8) {
+      if (i > 0) row_load_int8<NCH>(P.Crows + static_cast<size_t>(k) * P.crow_bytes, d, q8, sw8);
+      s = row_dot_int8_hs<NCH>(q8, sw8, hs, d);
     } else {
       if (i > 0) row_load_bf16<NCH>(reinterpret_cast<const uint16_t*>(P.Crows + static_cast<size_t>(k) * P.crow_bytes), d, w);
       s = row_dot_bf16_hs<NCH>(w, hs, d);
@@ -242,6 +263,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   }
   __syncthreads();
   if (tid == 0) {
+    misc->prior_n = P.sync->last_in_range;  // the list length the last call saw (read while waiting)
     red_release_add_u32(&P.sync->arrive, 1u);  // keys, counts and list entries of this CTA are published
     // wait (bounded, with backoff) until every CTA has arrived
     int okw = 1;
@@ -254,7 +276,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
       }
     }
     misc->claim = okw;
-    misc->nlist = __ldcg(&P.sync->list_count);
   }
   __syncthreads();
   FH_TL(3);
@@ -264,11 +285,45 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   // scratch (the slot area): the list's keys and ids, or all c keys; then the selection state
   const int p = P.p, c = P.c;
   const int r_2p = min(c, 2 * p);
-  const uint32_t nlist = misc->nlist;
-  const bool use_list = region && nlist >= static_cast<uint32_t>(p) && nlist <= static_cast<uint32_t>(P.list_cap);
-  const int nl = use_list ? static_cast<int>(nlist) : 0;
   uint32_t* skey = reinterpret_cast<uint32_t*>(slots);
   int32_t* sid = reinterpret_cast<int32_t*>(slots + up128(static_cast<size_t>(P.list_cap) * 4));
+  // The reads after the arrival go out together: the list length, this
+  // thread's histogram bins, and the list up to the length the last call saw
+  // (plus a margin); entries past that follow once the length is known.
+  uint32_t nlist = 0u;
+  uint4 hq = make_uint4(0u, 0u, 0u, 0u);
+  const uint32_t prior_n = misc->prior_n;
+  const int spec = min(P.list_cap, static_cast<int>(min(prior_n + prior_n / 4u + 64u, 0x7FFFFFFFu)));
+  auto load_list = [&](int from, int to) {
+    for (int base = from; base < to; base += 4 * kThreads) {
+      uint32_t kk[4];
+      int32_t ii[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = base + j * kThreads + tid;
+        if (i < to) {
+          kk[j] = __ldcg(P.list_key + i);
+          ii[j] = __ldcg(P.list_id + i);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = base + j * kThreads + tid;
+        if (i < to) {
+          skey[i] = kk[j];
+          sid[i] = ii[j];
+        }
+      }
+    }
+  };
+  if (ok && region) {
+    nlist = __ldcg(&P.sync->list_count);
+    hq = __ldcg(reinterpret_cast<const uint4*>(P.hist) + (kB1Bins / 4 - 1 - tid));
+    load_list(0, spec);
+  }
+  const bool use_list = region && nlist >= static_cast<uint32_t>(p) && nlist <= static_cast<uint32_t>(P.list_cap);
+  const int nl = use_list ? static_cast<int>(nlist) : 0;
+  if (ok && nl > spec) load_list(spec, nl);
   const uint32_t bs_off =
       static_cast<uint32_t>(P.off_slots) +
       static_cast<uint32_t>(std::max(2 * up128(static_cast<size_t>(P.list_cap) * 4), up128(static_cast<size_t>(c) * 4)));
@@ -280,11 +335,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   }
   if (ok) {
     if (use_list) {
-      const uint4 hq = __ldcg(reinterpret_cast<const uint4*>(P.hist) + (kB1Bins / 4 - 1 - tid));
-      for (int i = tid; i < nl; i += kThreads) {
-        skey[i] = __ldcg(P.list_key + i);
-        sid[i] = __ldcg(P.list_id + i);
-      }
       FH_TL(8);
       // bins from the top: thread t owns kB1Bins-1-4t (first) .. kB1Bins-4-4t
       const uint32_t hv[4] = {hq.w, hq.z, hq.y, hq.x};
@@ -424,6 +474,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     __syncthreads();
   }
   FH_TL(4);
+  // a dependent grid may launch now; its CTAs start as this grid's CTAs leave the SMs
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // ---------------- phase 3: candidate rows ----------------
   // row r is slot r % b of the (r / b)-th chosen cluster; rows
@@ -588,24 +640,41 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     P.sync->arrive = 0u;
     P.sync->ticket = 0u;
     P.sync->list_count = 0u;
-    P.sync->epoch = epoch + 1u;
+    P.sync->epoch = P.sync->epoch + 1u;  // calls on one head are stream-ordered
   }
 }
 
 template <int NCH>
-cudaError_t launch_nch(const B1Params& P, int grid, size_t smem, int int4, cudaStream_t st) {
+cudaError_t launch_nch(const B1Params& P, int grid, size_t smem, int cfmt, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (int4) return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, true>, P);
-  return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, false>, P);
+  // programmatic dependent launch with the cooperative attribute; if a driver
+  // refuses the pair, launch cooperatively alone from then on (the kernel's
+  // griddepcontrol instructions are no-ops without the attribute)
+  static bool pdl_ok = true;
+  cfg.numAttrs = pdl_ok ? 2 : 1;
+  auto go = [&]() {
+    if (cfmt == kFmtInt4) return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, kFmtInt4>, P);
+    if (cfmt == kFmtInt8) return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, kFmtInt8>, P);
+    return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, kFmtBf16>, P);
+  };
+  cudaError_t e = go();
+  if (e != cudaSuccess && cfg.numAttrs == 2 && e != cudaErrorLaunchOutOfResources) {
+    (void)cudaGetLastError();
+    pdl_ok = false;
+    cfg.numAttrs = 1;
+    e = go();
+  }
+  return e;
 }
 
 }  // namespace
@@ -626,24 +695,27 @@ extern "C" int fh_timeline_read(unsigned long long* host, int n) {
 }
 #endif
 
-cudaError_t launch_decode_b1(const B1Params& P, int grid, size_t smem, int int4, int nch, cudaStream_t st) {
+cudaError_t launch_decode_b1(const B1Params& P, int grid, size_t smem, int cfmt, int nch, cudaStream_t st) {
   switch (nch) {
-    case 1: return launch_nch<1>(P, grid, smem, int4, st);
-    case 2: return launch_nch<2>(P, grid, smem, int4, st);
-    case 3: return launch_nch<3>(P, grid, smem, int4, st);
-    case 4: return launch_nch<4>(P, grid, smem, int4, st);
-    case 5: return launch_nch<5>(P, grid, smem, int4, st);
-    case 6: return launch_nch<6>(P, grid, smem, int4, st);
-    case 8: return launch_nch<8>(P, grid, smem, int4, st);
-    case 10: return launch_nch<10>(P, grid, smem, int4, st);
+    case 1: return launch_nch<1>(P, grid, smem, cfmt, st);
+    case 2: return launch_nch<2>(P, grid, smem, cfmt, st);
+    case 3: return launch_nch<3>(P, grid, smem, cfmt, st);
+    case 4: return launch_nch<4>(P, grid, smem, cfmt, st);
+    case 5: return launch_nch<5>(P, grid, smem, cfmt, st);
+    case 6: return launch_nch<6>(P, grid, smem, cfmt, st);
+    case 8: return launch_nch<8>(P, grid, smem, cfmt, st);
+    case 10: return launch_nch<10>(P, grid, smem, cfmt, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
-cudaError_t occupancy_decode_b1(int int4, int nch, size_t smem, int* blocks) {
-#define FH_O(N)                                                                                      \
-  return int4 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, decode_b1_kernel<N, true>, kThreads, smem) \
-              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, decode_b1_kernel<N, false>, kThreads, smem);
+cudaError_t occupancy_decode_b1(int cfmt, int nch, size_t smem, int* blocks) {
+#define FH_O(N)                                                                                           \
+  return cfmt == kFmtInt4                                                                                 \
+             ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, decode_b1_kernel<N, kFmtInt4>, kThreads, smem) \
+         : cfmt == kFmtInt8                                                                               \
+             ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, decode_b1_kernel<N, kFmtInt8>, kThreads, smem) \
+             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, decode_b1_kernel<N, kFmtBf16>, kThreads, smem);
   switch (nch) {
     case 1: FH_O(1)
     case 2: FH_O(2)
@@ -662,9 +734,11 @@ cudaError_t set_attrs_decode_b1(int max_smem) {
   cudaError_t e = cudaSuccess;
 #define FH_SET(N)                                                                                         \
   if (e == cudaSuccess)                                                                                   \
-    e = cudaFuncSetAttribute(decode_b1_kernel<N, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem); \
+    e = cudaFuncSetAttribute(decode_b1_kernel<N, kFmtBf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem); \
   if (e == cudaSuccess)                                                                                   \
-    e = cudaFuncSetAttribute(decode_b1_kernel<N, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+    e = cudaFuncSetAttribute(decode_b1_kernel<N, kFmtInt4>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem); \
+  if (e == cudaSuccess)                                                                                   \
+    e = cudaFuncSetAttribute(decode_b1_kernel<N, kFmtInt8>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
   FH_SET(1) FH_SET(2) FH_SET(3) FH_SET(4) FH_SET(5) FH_SET(6) FH_SET(8) FH_SET(10)
 #undef FH_SET
   return e;

@@ -142,10 +142,10 @@ __global__ void c2t_verify_kernel(const C2TCheckParams P) {
     if (P.counts[t] != 1u) atomicExch(P.bad, 1);
 }
 
-// Packed INT4 row k: [d/2 code bytes][d/16 scale bytes][zero pad to rs].
-__global__ void repack_int4_kernel(const RepackParams P) {
+// Packed row k: [qb code bytes][d/16 scale bytes][zero pad to rs] (INT4: qb = d/2, INT8: qb = d).
+__global__ void repack_kernel(const RepackParams P) {
   const long long total = static_cast<long long>(P.c) * P.rs;
-  const int qb = P.d / 2, sb = P.d / 16;
+  const int qb = P.qb, sb = P.d / 16;
   const uint8_t* scales = reinterpret_cast<const uint8_t*>(P.C_scales);
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
@@ -188,8 +188,8 @@ cudaError_t launch_c2t_check(const C2TCheckParams& P, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_repack_int4(const RepackParams& P, cudaStream_t st) {
-  repack_int4_kernel<<<1024, 256, 0, st>>>(P);
+cudaError_t launch_repack(const RepackParams& P, cudaStream_t st) {
+  repack_kernel<<<1024, 256, 0, st>>>(P);
   return cudaGetLastError();
 }
 

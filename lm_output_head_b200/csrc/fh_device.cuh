@@ -157,6 +157,13 @@ __device__ __forceinline__ float nib(uint32_t w, int i) {
   return __uint_as_float(0x4B000000u | u) - 8388616.0f;
 }
 
+// Signed byte i (two's complement) of w as an exact float, by the same trick:
+// (byte ^ 0x80) maps -128..127 to 0..255 inside the mantissa of 2^23.
+__device__ __forceinline__ float sbyte(uint32_t w, int i) {
+  const uint32_t u = ((w >> (8 * i)) & 0xFFu) ^ 0x80u;
+  return __uint_as_float(0x4B000000u | u) - 8388736.0f;
+}
+
 // Dot of 8 bf16 (one 16-byte chunk) with 8 fp32 values.
 __device__ __forceinline__ float dot8(const uint4 w, const float* h, float acc) {
   acc = fmaf(bf16lo(w.x), h[0], acc);
@@ -826,6 +833,74 @@ __device__ __forceinline__ float row_dot_int4_hs(const uint32_t (&q)[NCH], const
   return warp_sum(acc);
 }
 
+// Packed INT8 row ([d code bytes][d/16 scale bytes]) in the bf16 chunk layout:
+// for chunk m, lane l holds the 8 codes of elements (l + 32 m) * 8 .. + 8 (one
+// 8-byte load) and the bf16 scale of their group of 32.
+__device__ __forceinline__ uint2 ldg_stream64(const void* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+
+// The row's bf16 scales travel as 32-bit words (word w = the scales of groups
+// 2w and 2w + 1), NW words per lane (lane l holds words l, l + 32, ...): one
+// register per 2048 elements instead of one per chunk. Chunk m of lane l
+// needs group (l >> 2) + 8 m, i.e. word (l >> 3) + 4 m, which sits in lane
+// ((l >> 3) + 4 m) % 32, register m / 8 -- the same register for the whole warp.
+template <int NCH>
+constexpr int int8_scale_words() { return (NCH + 7) / 8; }
+
+template <int NCH>
+__device__ __forceinline__ void row_load_int8(const uint8_t* row, int d, uint2 (&q)[NCH],
+                                              uint32_t (&scw)[int8_scale_words<NCH>()]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int m = 0; m < NCH; ++m) {
+    const int e = (lane + 32 * m) * 8;
+    q[m] = e < d ? ldg_stream64(row + e) : make_uint2(0u, 0u);
+  }
+  const int nw = (d / 32 + 1) / 2;  // scale words of the row
+#pragma unroll
+  for (int j = 0; j < int8_scale_words<NCH>(); ++j) {
+    const int wi = lane + 32 * j;
+    uint32_t v = 0u;
+    if (wi < nw) {
+      const unsigned short* sp = reinterpret_cast<const unsigned short*>(row + d) + 2 * wi;
+      v = __ldg(sp);
+      if (2 * wi + 1 < d / 32) v |= static_cast<uint32_t>(__ldg(sp + 1)) << 16;
+    }
+    scw[j] = v;
+  }
+}
+
+template <int NCH>
+__device__ __forceinline__ float row_dot_int8_hs(const uint2 (&q)[NCH], const uint32_t (&scw)[int8_scale_words<NCH>()],
+                                                 const float* hs, int d) {
+  const int lane = threadIdx.x & 31;
+  float acc = 0.f;
+#pragma unroll
+  for (int m = 0; m < NCH; ++m) {
+    const int wi = (lane >> 3) + 4 * m;
+    const uint32_t word = __shfl_sync(0xFFFFFFFFu, scw[m / 8], wi & 31);
+    const int e = (lane + 32 * m) * 8;
+    if (e < d) {
+      const float4 a = *reinterpret_cast<const float4*>(hs + e);
+      const float4 b = *reinterpret_cast<const float4*>(hs + e + 4);
+      float part = sbyte(q[m].x, 0) * a.x;
+      part = fmaf(sbyte(q[m].x, 1), a.y, part);
+      part = fmaf(sbyte(q[m].x, 2), a.z, part);
+      part = fmaf(sbyte(q[m].x, 3), a.w, part);
+      part = fmaf(sbyte(q[m].y, 0), b.x, part);
+      part = fmaf(sbyte(q[m].y, 1), b.y, part);
+      part = fmaf(sbyte(q[m].y, 2), b.z, part);
+      part = fmaf(sbyte(q[m].y, 3), b.w, part);
+      const uint32_t bits = ((lane >> 2) & 1) ? (word & 0xFFFF0000u) : (word << 16);  // group parity
+      acc = fmaf(__uint_as_float(bits), part, acc);
+    }
+  }
+  return warp_sum(acc);
+}
+
 // The same dots for a row held in shared memory (landed by a bulk copy).
 template <int NCH>
 __device__ __forceinline__ float srow_dot_bf16_hs(uint32_t row, const float* hs, int d) {
@@ -869,6 +944,32 @@ __device__ __forceinline__ float srow_dot_int4_hs(uint32_t row, const float* hs,
     }
   }
   return row_dot_int4_hs<NCH>(q, sc, hs, d);
+}
+
+template <int NCH>
+__device__ __forceinline__ float srow_dot_int8_hs(uint32_t row, const float* hs, int d) {
+  const int lane = threadIdx.x & 31;
+  float acc = 0.f;
+#pragma unroll
+  for (int m = 0; m < NCH; ++m) {
+    const int e = (lane + 32 * m) * 8;
+    if (e < d) {
+      const uint2 q = lds64(row + static_cast<uint32_t>(e));
+      const float scl = bf16f(lds16(row + static_cast<uint32_t>(d + 2 * (e >> 5))));
+      const float4 a = *reinterpret_cast<const float4*>(hs + e);
+      const float4 b = *reinterpret_cast<const float4*>(hs + e + 4);
+      float part = sbyte(q.x, 0) * a.x;
+      part = fmaf(sbyte(q.x, 1), a.y, part);
+      part = fmaf(sbyte(q.x, 2), a.z, part);
+      part = fmaf(sbyte(q.x, 3), a.w, part);
+      part = fmaf(sbyte(q.y, 0), b.x, part);
+      part = fmaf(sbyte(q.y, 1), b.y, part);
+      part = fmaf(sbyte(q.y, 2), b.z, part);
+      part = fmaf(sbyte(q.y, 3), b.w, part);
+      acc = fmaf(scl, part, acc);
+    }
+  }
+  return warp_sum(acc);
 }
 
 // Stage a bf16 vector of d elements (d % 8 == 0) into shared memory as fp32.

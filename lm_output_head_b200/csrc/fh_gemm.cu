@@ -13,10 +13,11 @@
 //   - warp 5 (one lane) loads H blocks, and the streamed rows when they are
 //     bf16, with TMA (cp.async.bulk.tensor, 128-byte swizzle, no multicast)
 //     into a ring of shared-memory stages of 64 K-elements;
-//   - INT4 centroids: warps 8..15 read the packed codes and bf16 scales and
-//     write code * scale into the stage as an exact pair of bf16 tiles
-//     hi + lo (hi = bf16(code * scale), lo = the rest, exact in bf16), in the
-//     same swizzled layout, so two MMAs give the exact products;
+//   - INT4 or INT8 centroids: warps 8..15 read the packed codes and bf16
+//     scales and write code * scale into the stage as an exact pair of bf16
+//     tiles hi + lo (hi = bf16(code * scale), lo = the rest, exact in bf16:
+//     code * scale has at most 7 + 8 significant bits), in the same swizzled
+//     layout, so two MMAs give the exact products;
 //   - warp 4 (one lane) issues tcgen05.mma kind::f16 (M 128, N tn, K 16; bf16
 //     in, fp32 accumulators in tensor memory, double-buffered when they fit so
 //     the epilogue of one tile overlaps the MMAs of the next) and commits stage
@@ -121,15 +122,16 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
 }
 
 
-template <bool B_INT4>
+template <int FMT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmR, const GemmParams P) {
+  constexpr bool B_Q = FMT != kFmtBf16;  // streamed rows dequantised in the kernel
   extern __shared__ __align__(1024) uint8_t gsm[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int S = P.stages, hm = P.hm, tn = P.tn, nbuf = P.nbuf;
   const uint32_t a_bytes = kTileM * kTileK * 2;                     // one 128-row block of H: 16 KB
   const uint32_t b_bytes = static_cast<uint32_t>(tn) * kTileK * 2;  // tn streamed rows x 128 B
-  const uint32_t stage_bytes = static_cast<uint32_t>(hm) * a_bytes + (B_INT4 ? 2u : 1u) * b_bytes;
+  const uint32_t stage_bytes = static_cast<uint32_t>(hm) * a_bytes + (B_Q ? 2u : 1u) * b_bytes;
   // stages start at the first 1024-byte boundary (the 128-byte swizzle repeats every 1024 bytes)
   const uint32_t raw = smem_addr(gsm);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -146,7 +148,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(bar(sm.full[s]), B_INT4 ? 1 + kDequantThreads : 1);
+      mbar_init(bar(sm.full[s]), B_Q ? 1 + kDequantThreads : 1);
       mbar_init(bar(sm.empty[s]), 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -186,9 +188,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ok = false;
             break;
           }
-          mbar_expect_tx(bar(sm.full[s]), static_cast<uint32_t>(hm) * a_bytes + (B_INT4 ? 0u : b_bytes));
+          mbar_expect_tx(bar(sm.full[s]), static_cast<uint32_t>(hm) * a_bytes + (B_Q ? 0u : b_bytes));
           for (int m = 0; m < hm; ++m) tma_load_2d(a_at(s, m), &tmH, ks * kTileK, m * kTileM, bar(sm.full[s]));
-          if (!B_INT4) tma_load_2d(b_hi(s), &tmR, ks * kTileK, t * tn, bar(sm.full[s]));
+          if (!B_Q) tma_load_2d(b_hi(s), &tmR, ks * kTileK, t * tn, bar(sm.full[s]));
         }
       }
       if (!ok) fail();
@@ -196,8 +198,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int j = std::max(0, g - S); j < g; ++j)
         wait_parity(bar(sm.full[j % S]), static_cast<uint32_t>(j / S) & 1u, abort_flag, kGemmBudget / 4);
     }
-  } else if (B_INT4 && warp >= 8) {
-    // ---------------- INT4 dequantisation of the streamed rows (hi + lo bf16) ----------------
+  } else if (B_Q && warp >= 8) {
+    // ---------------- INT4 / INT8 dequantisation of the streamed rows (hi + lo bf16) ----------------
     // thread pair (2r, 2r + 1) handles row r of the tile, 32 elements each; the
     // codes of a stage are loaded before its slot is free
     const int dt = tid - 8 * 32;  // 0 .. kDequantThreads-1
@@ -211,18 +213,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int e0 = ks * kTileK + 32 * half;  // this thread's 32 elements (one scale group)
         constexpr int kRowsPerPass = kDequantThreads / 2;
         const int nrow = tn / kRowsPerPass;  // 2 (tn 128) or 4 (tn 256)
-        uint4 q[4];
+        uint4 q[4], q2[4];  // q2: INT8 codes 16..31 of the group
         uint32_t scw[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           q[i] = make_uint4(0, 0, 0, 0);
+          q2[i] = make_uint4(0, 0, 0, 0);
           scw[i] = 0u;
           const int r = (dt >> 1) + i * kRowsPerPass;
           const int row = t * tn + r;
           if (i < nrow && row < P.rows && e0 < P.d) {
             const uint8_t* src = P.crows + static_cast<size_t>(row) * P.crow_bytes;
-            q[i] = *reinterpret_cast<const uint4*>(src + e0 / 2);
-            scw[i] = *reinterpret_cast<const unsigned short*>(src + P.d / 2 + 2 * (e0 / 32));
+            if constexpr (FMT == kFmtInt4) {
+              q[i] = *reinterpret_cast<const uint4*>(src + e0 / 2);
+              scw[i] = *reinterpret_cast<const unsigned short*>(src + P.d / 2 + 2 * (e0 / 32));
+            } else {
+              q[i] = *reinterpret_cast<const uint4*>(src + e0);
+              q2[i] = *reinterpret_cast<const uint4*>(src + e0 + 16);
+              scw[i] = *reinterpret_cast<const unsigned short*>(src + P.d + 2 * (e0 / 32));
+            }
           }
         }
         if (!wait_parity(bar(sm.empty[s]), ph ^ 1u, abort_flag, kGemmBudget)) {
@@ -234,7 +243,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (i >= nrow) break;
           const int r = (dt >> 1) + i * kRowsPerPass;
           const float scl = __uint_as_float(scw[i] << 16);
-          const uint32_t qw[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
+          const uint32_t qw[8] = {q[i].x, q[i].y, q[i].z, q[i].w, q2[i].x, q2[i].y, q2[i].z, q2[i].w};
           uint8_t* hi = gbase + (b_hi(s) - base) + r * 128;
           uint8_t* lo = gbase + (b_lo(s) - base) + r * 128;
 #pragma unroll
@@ -242,7 +251,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint32_t h[4], l[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float v0 = nib(qw[j], 2 * e) * scl, v1 = nib(qw[j], 2 * e + 1) * scl;
+              float v0, v1;
+              if constexpr (FMT == kFmtInt4) {
+                v0 = nib(qw[j], 2 * e) * scl;
+                v1 = nib(qw[j], 2 * e + 1) * scl;
+              } else {  // elements 8j + 2e, 8j + 2e + 1: word 2j + e/2, bytes 2(e&1), 2(e&1) + 1
+                const uint32_t wd = qw[2 * j + (e >> 1)];
+                v0 = sbyte(wd, 2 * (e & 1)) * scl;
+                v1 = sbyte(wd, 2 * (e & 1) + 1) * scl;
+              }
               const __nv_bfloat162 hb = __floats2bfloat162_rn(v0, v1);
               const float2 hf = __bfloat1622float2(hb);
               const __nv_bfloat162 lb = __floats2bfloat162_rn(v0 - hf.x, v1 - hf.y);  // exact rest
@@ -289,7 +306,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               const uint32_t dcol = tmem + static_cast<uint32_t>((buf * hm + m) * tn);
               const uint64_t ad = smem_desc_sw128(a_at(s, m) + 32u * k);
               mma_bf16(dcol, ad, bh, idesc, (ks | k) != 0);
-              if (B_INT4) mma_bf16(dcol, ad, bl, idesc, 1u);
+              if (B_Q) mma_bf16(dcol, ad, bl, idesc, 1u);
             }
           }
           mma_commit(bar(sm.empty[s]));  // the stage is free once these MMAs have read it
@@ -419,9 +436,9 @@ bool make_map(CUtensorMap* map, const void* ptr, int rows, int d, int box_rows) 
 
 }  // namespace
 
-// Stage plan: hm H blocks (16 KB each) + tn streamed rows (x2 for INT4 hi/lo) per stage.
-size_t gemm_smem_bytes(int hm, int tn, int int4, int* stages) {
-  const size_t st = static_cast<size_t>(hm) * kTileM * kTileK * 2 + (int4 ? 2 : 1) * static_cast<size_t>(tn) * kTileK * 2;
+// Stage plan: hm H blocks (16 KB each) + tn streamed rows (x2 for dequantised hi/lo) per stage.
+size_t gemm_smem_bytes(int hm, int tn, int dequant, int* stages) {
+  const size_t st = static_cast<size_t>(hm) * kTileM * kTileK * 2 + (dequant ? 2 : 1) * static_cast<size_t>(tn) * kTileK * 2;
   const size_t extra = sizeof(GemmSmem) + 1024;  // + alignment slack
   int s = 4;
   while (s > 2 && static_cast<size_t>(s) * st + extra > 227 * 1024) --s;
@@ -438,26 +455,29 @@ cudaError_t launch_gemm(const GemmParams& P0, const void* rows_bf16, const void*
   P.nbuf = P.hm * P.tn * 2 <= 512 ? 2 : 1;  // double-buffered accumulators when tensor memory allows
   P.tmem_cols = 32;
   while (P.tmem_cols < P.nbuf * P.hm * P.tn) P.tmem_cols *= 2;  // a power of two >= 32
-  const size_t smem = gemm_smem_bytes(P.hm, P.tn, P.int4, &P.stages);
+  const size_t smem = gemm_smem_bytes(P.hm, P.tn, P.cfmt != kFmtBf16, &P.stages);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   CUtensorMap mh{}, mr{};
   if (!make_map(&mh, H, P.nb, P.d, kTileM)) return cudaErrorInvalidValue;
-  if (P.int4) {
+  if (P.cfmt != kFmtBf16) {
     mr = mh;  // unused: the streamed rows are read and dequantised by the kernel
   } else if (!make_map(&mr, rows_bf16, P.rows, P.d, P.tn)) {
     return cudaErrorInvalidValue;
   }
   const int ntiles = (P.rows + P.tn - 1) / P.tn;
   const int grid = std::min(num_sms, ntiles);
-  if (P.int4) gemm_kernel<true><<<grid, kGemmThreads, smem, st>>>(mh, mr, P);
-  else gemm_kernel<false><<<grid, kGemmThreads, smem, st>>>(mh, mr, P);
+  if (P.cfmt == kFmtInt4) gemm_kernel<kFmtInt4><<<grid, kGemmThreads, smem, st>>>(mh, mr, P);
+  else if (P.cfmt == kFmtInt8) gemm_kernel<kFmtInt8><<<grid, kGemmThreads, smem, st>>>(mh, mr, P);
+  else gemm_kernel<kFmtBf16><<<grid, kGemmThreads, smem, st>>>(mh, mr, P);
   return cudaGetLastError();
 }
 
 cudaError_t set_attrs_gemm() {
-  cudaError_t e = cudaFuncSetAttribute(gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  cudaError_t e = cudaFuncSetAttribute(gemm_kernel<kFmtInt4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    e = cudaFuncSetAttribute(gemm_kernel<kFmtInt8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemm_kernel<kFmtBf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
   return e;
 }
 

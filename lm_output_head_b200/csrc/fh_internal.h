@@ -16,6 +16,11 @@ constexpr long long kWaitBudget = 4000000000LL;      // bulk-copy waits (~2 s)
 constexpr long long kDefaultSpinBudget = 2000000000LL;  // device-wide waits (~1 s)
 constexpr int kB1Bins = 2048;  // histogram bins of the fused B = 1 selection
 
+// Centroid row formats as the kernels see them (the same values as fh_centroid_format):
+// bf16 rows; packed INT4 g32 rows [d/2 codes][d/16 scale bytes]; packed INT8 g32 rows
+// [d codes][d/16 scale bytes] (packed rows padded to 16 bytes).
+constexpr int kFmtBf16 = 0, kFmtInt4 = 1, kFmtInt8 = 2;
+
 // Workspace words at the start of the workspace.
 struct SyncWords {
   int32_t status;
@@ -128,7 +133,7 @@ struct GemmParams {
   int rows, d;              // streamed operand: rows x d (centroid or token rows), K = d
   int nb;                   // hidden rows of this launch, 1..256 (two M blocks of 128)
   int hm, tn, nbuf, stages, tmem_cols;  // set by the launcher
-  int int4;                 // streamed operand given as packed INT4 rows (crows) instead of bf16
+  int cfmt;                 // streamed operand: kFmtBf16 rows through TMA, or packed INT4 / INT8 rows (crows)
   int epi;                  // 0: store scores / keys, 1: per-hidden-row argmax
   int mode;                 // epi 0: 0 raw scores, 1 Gumbel keys
   float T;
@@ -171,12 +176,13 @@ struct RepackParams {
   const uint16_t* C_scales;
   uint8_t* out;
   int c, d, rs;
+  int qb;                   // code bytes per row: d / 2 (INT4) or d (INT8)
 };
 
 // Launchers (defined in the .cu files). Each returns the CUDA error of the launch.
-cudaError_t launch_decode_b1(const B1Params& P, int grid, size_t smem, int int4, int nch,
+cudaError_t launch_decode_b1(const B1Params& P, int grid, size_t smem, int cfmt, int nch,
                              cudaStream_t st);
-cudaError_t launch_scores(const ScoresParams& P, int grid, size_t smem, int int4, int nch,
+cudaError_t launch_scores(const ScoresParams& P, int grid, size_t smem, int cfmt, int nch,
                           cudaStream_t st);
 cudaError_t launch_select(const SelectParams& P, int B, size_t smem, cudaStream_t st);
 cudaError_t launch_sort_ids(const SelectParams& P, int B, size_t smem, cudaStream_t st);
@@ -184,17 +190,24 @@ cudaError_t launch_candidates(const CandParams& P, int grid, size_t smem, int nc
 cudaError_t launch_epilogue(const EpilogueParams& P, int B, cudaStream_t st);
 cudaError_t launch_dense(const DenseParams& P, int grid, size_t smem, int nch, cudaStream_t st);
 cudaError_t launch_c2t_check(const C2TCheckParams& P, cudaStream_t st);
-cudaError_t launch_repack_int4(const RepackParams& P, cudaStream_t st);
+cudaError_t launch_repack(const RepackParams& P, cudaStream_t st);
 // Cluster-major copy of the token rows: out[k*b + j] = E[C2T[k][j]].
 cudaError_t launch_gather_cluster_major(const uint16_t* E, const int32_t* C2T, uint16_t* out, int v, int d,
                                         cudaStream_t st);
-// tcgen05 GEMM (B >= 64): streamed rows bf16 [rows, d] through TMA, or packed INT4 rows; H bf16 [nb, d].
+// tcgen05 GEMM (B >= 64): streamed rows bf16 [rows, d] through TMA, or packed INT4 / INT8 rows; H bf16 [nb, d].
 cudaError_t launch_gemm(const GemmParams& P, const void* rows_bf16, const void* H, int num_sms, cudaStream_t st);
 cudaError_t set_attrs_gemm();
 // De-duplicated candidate logits of a batch (b == 16): CSR of the selections by cluster, then one
 // pass per distinct cluster on the tensor cores.
 cudaError_t launch_group(const GroupParams& P, int num_sms, cudaStream_t st);
 cudaError_t set_attrs_group();
+// Speculative verification of draft tokens against dense logits (one CTA per row).
+cudaError_t launch_spec_verify(const float* logits, int v, const int32_t* cand, int n, int B, const int32_t* draft,
+                               float T, const float* u_accept, const float* u_resample, int32_t* out, int* status,
+                               cudaStream_t st);
+// Adaptive probe count per row of centroid scores (one CTA per row).
+cudaError_t launch_adaptive_probes(const float* scores, int B, int c, float tau, int p_min, int p_max, float T,
+                                   int32_t* out_p, cudaStream_t st);
 
 // Opt-in shared memory attribute for every instantiation (called once per device).
 cudaError_t set_kernel_attributes(int max_smem);

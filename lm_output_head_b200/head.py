@@ -51,8 +51,9 @@ def bf16_from_bits(bits: np.ndarray, device="cuda") -> torch.Tensor:
 class FlashHead:
     """A FlashHead retrieval head bound to device tensors (borrowed, kept alive here).
 
-    ``E`` bf16 [v, d]; ``C2T`` int32 [c, b]; centroids either ``C`` bf16 [c, d]
-    or ``C_q`` uint8 [c, d/2] with ``C_scales`` bf16 [c, d/32].
+    ``E`` bf16 [v, d]; ``C2T`` int32 [c, b]; centroids either ``C`` bf16 [c, d],
+    or ``C_q`` with ``C_scales`` bf16 [c, d/32]: uint8 [c, d/2] packed INT4
+    codes, or int8 [c, d] INT8 codes (the dtype picks the format).
     """
 
     def __init__(self, E: torch.Tensor, C2T: torch.Tensor, *, C: Optional[torch.Tensor] = None,
@@ -68,11 +69,11 @@ class FlashHead:
             C = _dev(C, "C", _BF16, 2)
             fmt = _lib.FH_CENTROID_BF16
         elif C_q is not None and C_scales is not None:
-            C_q = _dev(C_q, "C_q", (torch.uint8,), 2)
+            C_q = _dev(C_q, "C_q", (torch.uint8, torch.int8), 2)
             C_scales = _dev(C_scales, "C_scales", _BF16, 2)
-            fmt = _lib.FH_CENTROID_INT4_G32
+            fmt = _lib.FH_CENTROID_INT8_G32 if C_q.dtype == torch.int8 else _lib.FH_CENTROID_INT4_G32
         else:
-            raise ValueError("give C (bf16) or C_q and C_scales (INT4)")
+            raise ValueError("give C (bf16) or C_q and C_scales (INT4 uint8 / INT8 int8 codes)")
         self.E, self.C2T, self.C, self.C_q, self.C_scales = E, C2T, C, C_q, C_scales
         self.v, self.d, self.c, self.b = v, d, c, b
         self.fmt = fmt
@@ -165,6 +166,17 @@ class FlashHead:
                                              _ptr(logits), _stream(stream)), "fh_candidate_logits")
         return toks, logits
 
+    def adaptive_probes(self, scores: torch.Tensor, tau: float, p_min: int, p_max: int, *, T: float = 1.0,
+                        stream=None) -> torch.Tensor:
+        """Probes per row: the smallest p in [p_min, p_max] whose top-p clusters hold a fraction tau
+        of softmax(scores / T)."""
+        scores = _dev(scores, "scores", (torch.float32,), 2)
+        B = scores.shape[0]
+        out = torch.empty(B, dtype=torch.int32, device=self.device)
+        _check(self._lib.fh_adaptive_probes(self._h, _ptr(scores), B, float(tau), int(p_min), int(p_max), float(T),
+                                            _ptr(out), _stream(stream)), "fh_adaptive_probes")
+        return out
+
     def decode(self, hidden: torch.Tensor, p: int, *, mode: str = "greedy", T: float = 1.0,
                u_clusters: Optional[torch.Tensor] = None, u_token: Optional[torch.Tensor] = None,
                out_tokens: Optional[torch.Tensor] = None, out_cluster_ids: Optional[torch.Tensor] = None,
@@ -189,6 +201,21 @@ class FlashHead:
         _check(self._lib.fh_dense_head(self._h, _ptr(hidden), B, _ptr(logits), _ptr(out_argmax),
                                        _stream(stream)), "fh_dense_head")
         return (out_argmax, logits) if want_logits else out_argmax
+
+
+def speculative_verify(head: FlashHead, logits: torch.Tensor, cand_tokens: torch.Tensor, draft: torch.Tensor,
+                       T: float, u_accept: torch.Tensor, u_resample: torch.Tensor, stream=None) -> torch.Tensor:
+    """Check FlashHead drafts against the dense logits (``fh_speculative_verify``)."""
+    logits = _dev(logits, "logits", (torch.float32,), 2)
+    cand_tokens = _dev(cand_tokens, "cand_tokens", (torch.int32,), 2)
+    B, n = cand_tokens.shape
+    if logits.shape != (B, head.v):
+        raise ValueError("logits must be [B, v]")
+    out = torch.empty(B, dtype=torch.int32, device=logits.device)
+    _check(head._lib.fh_speculative_verify(head._h, _ptr(logits), _ptr(cand_tokens), int(n), int(B), _ptr(draft),
+                                           float(T), _ptr(u_accept), _ptr(u_resample), _ptr(out), _stream(stream)),
+           "fh_speculative_verify")
+    return out
 
 
 def dense_head_noalloc(E: torch.Tensor, hidden: torch.Tensor, out_argmax: torch.Tensor, *,

@@ -100,18 +100,21 @@ def run_case(cfg_id, B, repeats):
     print(json.dumps(rec), flush=True)
 
 
-def run_b1(cfg_id, steps):
+def run_b1(cfg_id, steps, int8=False):
     """One hidden state per step through the fused kernel, steps issued back to
     back and rotated over enough head copies that every step reads its
-    centroid and token rows from HBM (the protocol of bench.py)."""
+    centroid and token rows from HBM (the protocol of bench.py). With int8,
+    the head's centroids are quantised to INT8 group-32 codes."""
     import ctypes
     import torch
     import synth
     import lm_output_head_b200 as fh
     cfg, head, hid, _ = synth.make_config(cfg_id)
     dev = torch.device("cuda", 0)
-    int4 = head.C_q is not None
-    cbytes = head.C_q.nbytes + head.C_scales.nbytes if int4 else head.C.nbytes
+    if int8:
+        head.C_q, head.C_scales = synth.quantize_int8_g32(head.C)
+    int4 = head.C_q is not None and not int8
+    cbytes = head.C_q.nbytes + head.C_scales.nbytes if head.C_q is not None else head.C.nbytes
     abytes = cbytes + cfg.p * cfg.b * cfg.d * 2 + cfg.p * cfg.b * 4 + cfg.d * 2 + 4
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     n_copies = max(3, -(-4 * l2 // abytes) + 1)
@@ -120,7 +123,7 @@ def run_b1(cfg_id, steps):
     heads = []
     for i in range(n_copies):
         E, T = (E0, T0) if i == 0 else (E0.clone(), T0.clone())
-        if int4:
+        if head.C_q is not None:
             heads.append(fh.FlashHead(E, T, C_q=torch.from_numpy(head.C_q).to(dev),
                                       C_scales=fh.bf16_from_bits(head.C_scales, dev), max_batch=1,
                                       max_probes=cfg.p))
@@ -156,7 +159,7 @@ def run_b1(cfg_id, steps):
         h.close()
     print(json.dumps({
         "workload": f"config {cfg_id}: v{cfg.v} d{cfg.d} c{cfg.c} b{cfg.b} p{cfg.p} "
-                    f"{'INT4' if int4 else 'bf16'} centroids, B=1 greedy, fused kernel",
+                    f"{'INT8' if int8 else 'INT4' if int4 else 'bf16'} centroids, B=1 greedy, fused kernel",
         "us_per_token": round(us, 3), "tokens_per_s": round(1e6 / us, 1), "algorithmic_bytes": int(abytes),
         "achieved_GBps": round(abytes / us / 1e3, 1), "frac_of_hbm_peak": round(abytes / us / 1e3 / peak, 4),
         "peak_kind": kind, "head_copies": n_copies, "device_status": status}), flush=True)
@@ -166,13 +169,16 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--repeats", type=int, default=20)
     ap.add_argument("--cases", default="4:256,3:32,2:16,2:4,2:1",
-                    help="comma-separated config:batch pairs (batch 1: the fused kernel, back to back)")
+                    help="comma-separated config:batch pairs (batch 1: the fused kernel, back to back; "
+                         "config 'NQ8' = config N with INT8 centroids, batch 1 only)")
     ap.add_argument("--b1-steps", type=int, default=1000)
     args = ap.parse_args()
     for case in args.cases.split(","):
-        cfg_id, B = (int(x) for x in case.split(":"))
+        cs, bs = case.split(":")
+        int8 = cs.endswith("Q8")
+        cfg_id, B = int(cs[:-2] if int8 else cs), int(bs)
         if B == 1:
-            run_b1(cfg_id, args.b1_steps)
+            run_b1(cfg_id, args.b1_steps, int8=int8)
         else:
             run_case(cfg_id, B, args.repeats)
 

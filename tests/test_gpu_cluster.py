@@ -207,3 +207,83 @@ def test_create_rejects_bad_shapes(fh):
     assert lib.fh_cluster_create(100, 256, 3, None, ctypes.byref(h)) == _lib.FH_ERR_INVALID_ARG
     assert lib.fh_cluster_create(4096, 250, 64, None, ctypes.byref(h)) == _lib.FH_ERR_INVALID_ARG
     assert lib.fh_cluster_create(4096, 256, 64, None, ctypes.byref(h)) == _lib.FH_ERR_UNSUPPORTED  # b = 64
+
+
+def test_assign_at_the_llama_shape_has_no_blocking_pair(fh):
+    """v 128256, c 8016, d 2048 from k-means++ seeds: the assignment is balanced and,
+    on the same fp32 similarities, no token prefers a cluster whose weakest member
+    it beats -- the property that makes it the global greedy (unique under the
+    order similarity desc, token asc, cluster asc)."""
+    from lm_output_head_b200.cluster import ClusterBuilder
+    cfg, head, _, _ = synth.make_config(1, n_states=1)
+    v, d, c, b = head.v, head.d, head.c, head.b
+    cbl = ClusterBuilder(v, d, c)
+    try:
+        En = cbl.normalize(fh.bf16_from_bits(head.E, "cuda"))
+        u = np.random.default_rng(21).uniform(size=c).astype(np.float32)
+        ids = cbl.seed(En, torch.from_numpy(u).cuda())
+        assert cbl.device_status() == 0
+        idh = ids.cpu().numpy()
+        assert idh[0] == min(int(math.floor(float(u[0]) * v)), v - 1) and len(set(idh.tolist())) == c
+        S = cbl.similarities(En, cbl.gather(En, ids))
+        a, m, rounds = cbl.assign(S)
+        assert cbl.device_status() == 0
+        mh = m.cpu().numpy()
+        assert oracle.check_c2t(mh, v) and np.all(np.diff(mh, axis=1) > 0)
+        a = a.long()
+        t_all = torch.arange(v, device="cuda")
+        sa = S[a, t_all]                                    # every token's similarity to its cluster
+        ms = S.gather(1, m.long())                          # [c, b] members' similarities
+        # weakest member of every cluster: lowest similarity, then highest token id
+        ws = ms.min(dim=1).values
+        wt = torch.where(ms == ws[:, None], m.long(), torch.full_like(m.long(), -1)).max(dim=1).values
+        blocking = 0
+        for k0 in range(0, c, 512):
+            k1 = min(c, k0 + 512)
+            Sc = S[k0:k1]
+            kk = torch.arange(k0, k1, device="cuda")[:, None]
+            pref = (Sc > sa[None, :]) | ((Sc == sa[None, :]) & (kk < a[None, :]))
+            beats = (Sc > ws[k0:k1, None]) | ((Sc == ws[k0:k1, None]) & (t_all[None, :] < wt[k0:k1, None]))
+            blocking += int((pref & beats & (kk != a[None, :])).sum().item())
+        assert blocking == 0
+        assert rounds >= 1
+    finally:
+        cbl.close()
+
+
+def test_built_clusters_serve_as_a_head(fh):
+    """Cluster a planted vocabulary on the GPU, build a FlashHead from the result (E, C_out,
+    C2T_out) and decode: the tokens match the oracle's two-stage head on the same arrays."""
+    from lm_output_head_b200.cluster import ClusterBuilder
+    from tests import parity
+    bits, truth = _planted(15, noise=0.3)
+    rng = np.random.default_rng(16)
+    u = rng.uniform(size=C).astype(np.float32)
+    cbl = ClusterBuilder(V, D, C)
+    try:
+        E = fh.bf16_from_bits(bits, "cuda")
+        Cout, m, it = cbl.build(E, u_init=torch.from_numpy(u).cuda(), max_iter=100)
+        assert cbl.device_status() == 0
+    finally:
+        cbl.close()
+    head = synth.Head(v=V, d=D, c=C, b=B, E=bits, C=_bits(Cout), C2T=m.cpu().numpy())
+    assert oracle.check_c2t(head.C2T, V)
+    dh = fh.FlashHead(E, m, C=Cout, max_batch=4, max_probes=8)
+    try:
+        Hx = synth.to_bf16_bits((rng.standard_normal((8, D)) * 0.5).astype(np.float32))
+        rep = parity.Report()
+        for r in range(8):
+            tok = int(dh.decode(torch.from_numpy(Hx[r:r + 1].view(np.int16)).view(torch.bfloat16).cuda(), 8).item())
+            ids = torch.empty((1, 8), dtype=torch.int32, device="cuda")
+            dh.decode(torch.from_numpy(Hx[r:r + 1].view(np.int16)).view(torch.bfloat16).cuda(), 8,
+                      out_cluster_ids=ids)
+            Cw = oracle.centroid_matrix(head)
+            S = oracle.centroid_scores(Cw, Hx[r:r + 1])[0]
+            hw = oracle.widen_bf16(Hx[r])
+            rep.add(parity.check_cluster_set(ids.cpu().numpy()[0], S, 8, parity.loose_bound(Cw, hw),
+                                             parity.tight_bound(Cw, hw)))
+            rep.add(parity.check_greedy_token(head, Hx[r], ids.cpu().numpy()[0], tok))
+        assert rep.tight_mismatch == 0, rep
+        assert dh.device_status() == 0
+    finally:
+        dh.close()
