@@ -22,8 +22,11 @@ memory, SM clocks sampled during the timed region, and the fp64 oracle timed
 on the host cores.
 
 ``--impl reference`` times the fp64 CPU oracle on the same workload instead.
-Under torchrun every rank runs its own replica (the head does not shard:
-independent hidden states), timing is the max over ranks.
+``--gpus N`` runs N replicas, one process per GPU: under torchrun (WORLD_SIZE
+set) every rank is one replica; without it the script starts the N ranks
+itself through torch.distributed.run. The head does not shard (independent
+hidden states), so there is no data-path collective; timing is the maximum
+over ranks of each rank's device-timed total.
 """
 from __future__ import annotations
 
@@ -197,6 +200,7 @@ def oracle_threads():
 
 
 def time_oracle(head, hid, p, budget_s, max_states):
+    """The oracle as it stands, one hidden state per call, BLAS on its default threads."""
     import oracle
     n = 0
     t0 = time.perf_counter()
@@ -205,6 +209,70 @@ def time_oracle(head, hid, p, budget_s, max_states):
         n += 1
     dt = time.perf_counter() - t0
     return n, dt
+
+
+def oracle_pool_threads():
+    return max(1, min(os.cpu_count() or 1, 32))
+
+
+def time_oracle_rows(head, H, p, budget_s, threads):
+    """The oracle as it stands over hidden-state rows: ``threads`` workers, each
+    decoding its own rows one call at a time with single-threaded BLAS (numpy
+    releases the GIL inside its array operations). Returns (states, seconds)."""
+    import concurrent.futures as cf
+    from threadpoolctl import threadpool_limits
+    import oracle
+    n_states = H.shape[0]
+    t_end = [0.0]
+
+    def worker(w):
+        done = 0
+        i = w
+        while time.perf_counter() < t_end[0] and i < n_states:
+            oracle.decode(head, H[i:i + 1], p)
+            done += 1
+            i += threads
+        return done
+
+    with threadpool_limits(1):
+        t0 = time.perf_counter()
+        t_end[0] = t0 + budget_s
+        if threads == 1:
+            n = worker(0)
+        else:
+            with cf.ThreadPoolExecutor(threads) as ex:
+                n = sum(ex.map(worker, range(threads)))
+        dt = time.perf_counter() - t0
+    return n, dt
+
+
+def time_oracle_dense(head, H, budget_s):
+    """The oracle's dense head (z = E h over all v, argmax), one state per call, default BLAS threads."""
+    import oracle
+    n = 0
+    t0 = time.perf_counter()
+    while n < H.shape[0] and (n == 0 or (time.perf_counter() - t0) < budget_s):
+        oracle.dense_head(head.E, H[n:n + 1])
+        n += 1
+    return n, time.perf_counter() - t0
+
+
+def cpu_baseline(head, hid, p, budget_s):
+    """The fp64 oracle on the host cores, a bounded sample of the workload:
+    single-threaded, all cores (one worker per core over the hidden-state
+    rows), and the oracle's dense head. About ``budget_s`` seconds in all."""
+    threads = oracle_pool_threads()
+    n1, t1 = time_oracle_rows(head, hid.H, p, 0.3 * budget_s, 1)
+    na, ta = time_oracle_rows(head, hid.H, p, 0.45 * budget_s, threads)
+    nd, td = time_oracle_dense(head, hid.H, 0.25 * budget_s)
+    return {"value": round(na / ta, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"fp64 numpy oracle on hidden states of the same workload: {na} states over "
+                      f"{threads} worker threads in {ta:.1f} s (all cores); {n1} states single-threaded "
+                      f"in {t1:.1f} s; {nd} dense-head states in {td:.1f} s",
+            "all_cores_us_per_token": round(ta / na * 1e6, 1),
+            "single_thread_us_per_token": round(t1 / n1 * 1e6, 1),
+            "dense_oracle_us_per_token": round(td / nd * 1e6, 1),
+            "host_cpus": os.cpu_count()}
 
 
 # ---------------------------------------------------------------------------
@@ -429,11 +497,7 @@ def run_ours(args):
         "clocks": clocks,
     }
     if not args.no_cpu_baseline and world == 1:
-        n, dt = time_oracle(head, hid, cfg.p, args.cpu_seconds, n_states)
-        rec["cpu_baseline"] = {"value": round(n / dt, 3), "unit": "tokens/s", "cores": oracle_threads(),
-                               "kind": "oracle",
-                               "sample": f"{n} hidden states of the same workload, fp64 numpy oracle, "
-                                         f"{dt:.1f} s"}
+        rec["cpu_baseline"] = cpu_baseline(head, hid, cfg.p, args.cpu_seconds)
     print(json.dumps(rec), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
@@ -452,7 +516,8 @@ def run_reference(args):
     for i in range(min(args.warmup, 1)):
         oracle.decode(head, hid.H[i:i + 1], cfg.p)
     budget = args.cpu_seconds
-    n, dt = time_oracle(head, hid, cfg.p, budget, min(args.steps, hid.H.shape[0]))
+    threads = oracle_pool_threads()
+    n, dt = time_oracle_rows(head, hid.H[:min(args.steps, hid.H.shape[0])], cfg.p, budget, threads)
     value = n / dt
     rec = {
         "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
@@ -461,13 +526,66 @@ def run_reference(args):
         "data": "synthetic (seeded planted-cluster head)",
         "config": {"workload": WORKLOAD, "global_batch": 1, "parallelism": "host cores"},
         "impl": "reference",
-        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": oracle_threads(),
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads,
                          "kind": "oracle",
-                         "sample": f"{n} of the {args.steps} requested steps (one hidden state each) "
-                                   f"within a {budget:.0f} s budget"},
+                         "sample": f"{n} of the {args.steps} requested steps (one hidden state each) over "
+                                   f"{threads} worker threads within a {budget:.0f} s budget"},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(rec), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# launching N replicas, and a host-only run of the replica layer
+# ---------------------------------------------------------------------------
+def free_port():
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def relaunch(n, argv):
+    """Start ``n`` ranks of this script (one process per GPU) under
+    torch.distributed.run on this node; rank 0 prints the JSON line."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={free_port()}", os.path.abspath(__file__), *argv]
+    env = dict(os.environ, OMP_NUM_THREADS=os.environ.get("OMP_NUM_THREADS", "1"))
+    return subprocess.call(cmd, env=env)
+
+
+def run_host_selftest(args):
+    """The replica layer without a GPU: every rank times K host steps (a small
+    fp32 matrix product) after W warm-up steps between barriers, the maximum
+    over ranks goes through an all_reduce on gloo, and rank 0 prints the line
+    with the whole-job throughput. Exercises the launcher and the timing logic."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    world, rank, _ = dist_setup()
+    if world > 1:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    x = np.random.default_rng(rank).random((128, 128), dtype=np.float32)
+    for _ in range(args.warmup):
+        x = (x @ x) / 128.0
+    if world > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        x = (x @ x) / 128.0
+    total_ms = (time.perf_counter() - t0) * 1e3
+    total_ms = max_over_ranks(total_ms, world, "cpu")
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        print(json.dumps({"metric": "host self-test steps/s", "value": job_throughput(total_ms, args.steps, world),
+                          "unit": "steps/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                          "ms_per_step": total_ms / args.steps, "host_selftest": True}), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    del torch
 
 
 def main():
@@ -482,10 +600,16 @@ def main():
                     help="head copies the steps rotate over (default: enough to exceed 4 x L2)")
     ap.add_argument("--only-decode", action="store_true",
                     help="time the decode loop only (for profiling runs)")
+    ap.add_argument("--host-selftest", action="store_true",
+                    help="run the replica layer on host steps with gloo (no GPU): a check of the launcher")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(relaunch(args.gpus, sys.argv[1:]))
+    if args.host_selftest:
+        run_host_selftest(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -66,3 +66,19 @@ def test_two_gloo_replicas():
         assert value == pytest.approx(2 * 100 / 0.020)  # both ranks' tokens over that time
     assert res[0][4] == 0 and res[1][4] == 37 * 2    # rank 1 starts 37 rows later
     assert res[1][5] is None                         # rank 1 returned from the reference arm
+
+
+def test_bench_launches_its_own_ranks():
+    # `bench.py --gpus 2` without an outside launcher starts two ranks itself;
+    # the host self-test runs the replica layer on gloo and rank 0 alone prints
+    import json
+    import subprocess
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--host-selftest",
+                        "--steps", "20", "--warmup", "3"], capture_output=True, text=True, timeout=240, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    rec = json.loads(lines[0])
+    assert rec["n_gpus"] == 2 and rec["host_selftest"] and rec["steps"] == 20
+    assert rec["value"] == pytest.approx(2 * 20 / (rec["ms_per_step"] * 20 / 1e3))
