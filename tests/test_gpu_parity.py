@@ -455,17 +455,12 @@ def test_decode_gumbel_qwen_b32(fh):
 # ---------------------------------------------------------------------------
 # dense head
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("cfg_id,B", [(0, 1), (0, 33), (0, 65), (1, 1), (1, 4), (3, 2), (4, 64)])
-def test_dense_head(fh, cfg_id, B):
-    """B >= 64 runs the tcgen05 tile GEMM with the fused column argmax."""
-    cfg, head, hid, _, dh = get_cfg(cfg_id, fh) if cfg_id else get_cfg(0, fh, n_states=65, max_batch=65,
-                                                                       max_probes=256)
+def _dense_check(cfg, head, hid, dh, B):
     H = hid.H[:B]
     am, z = dh.dense_head(hid_dev(H), want_logits=True)
     am, z = am.cpu().numpy(), z.cpu().numpy()
     assert dh.device_status() == 0
     zr, amr = oracle.dense_head(head.E, H)
-    Ew = None
     for r in range(B):
         hw = oracle.widen_bf16(H[r])
         sample = np.arange(cfg.v) if cfg.v <= 8192 else np.random.default_rng(r).choice(cfg.v, 4096, False)
@@ -479,6 +474,31 @@ def test_dense_head(fh, cfg_id, B):
     # argmax only (no logits written)
     am2 = dh.dense_head(hid_dev(H)).cpu().numpy()
     assert np.array_equal(am2, am)
+
+
+@pytest.mark.parametrize("cfg_id,B", [(0, 1), (0, 33), (0, 65), (1, 1), (1, 4), (3, 2), (4, 64)])
+def test_dense_head(fh, cfg_id, B):
+    """B >= 64 runs the tcgen05 tile GEMM with the fused column argmax."""
+    cfg, head, hid, _, dh = get_cfg(cfg_id, fh) if cfg_id else get_cfg(0, fh, n_states=65, max_batch=65,
+                                                                       max_probes=256)
+    _dense_check(cfg, head, hid, dh, B)
+
+
+@pytest.mark.parametrize("cfg_id,B", [(0, 128), (0, 129), (0, 256), (4, 129), (4, 256)])
+def test_dense_head_two_row_blocks(fh, cfg_id, B):
+    """B > 128: the tcgen05 GEMM holds two 128-row blocks of hidden states per
+    launch, and the fused argmax epilogue keeps a running maximum for each; B = 129
+    leaves a one-row second block, B = 128 exactly one full block."""
+    if cfg_id == 0:
+        key = ("dense256", 0)
+        if key not in _HEADS:
+            cfg, head, hid, uni = synth.make_config(0, n_states=256)
+            _HEADS[key] = (cfg, head, hid, uni, _to_dev(head, 256, 256, fh))
+        cfg, head, hid, _, dh = _HEADS[key]
+    else:
+        cfg, head, hid, _, dh = get_cfg(cfg_id, fh)
+    assert hid.H.shape[0] >= B
+    _dense_check(cfg, head, hid, dh, B)
 
 
 # ---------------------------------------------------------------------------
