@@ -70,6 +70,11 @@ typedef enum {
 } fh_centroid_format;
 
 typedef enum {
+  FH_C2T_INT32 = 0,         /* C2T: int32 [c, b] */
+  FH_C2T_UINT16 = 1         /* C2T: uint16 [c, b], v <= 65536 */
+} fh_c2t_format;
+
+typedef enum {
   FH_GREEDY = 0,            /* top-p clusters by score, argmax token */
   FH_SAMPLE_GUMBEL = 1      /* Gumbel-top-p clusters at T, softmax(z/T) token */
 } fh_mode;
@@ -89,10 +94,14 @@ typedef enum {
  *               byte per element (the W8A16 row of the write-up's parameter
  *               table, section 5.2).
  *  C_scales     device bf16 [c, d/32] (INT4 and INT8 formats): value = code * scale.
- *  C2T          device int32 [c, b].
+ *  C2T          device int32 [c, b] (4-byte aligned), or, with c2t_format
+ *               FH_C2T_UINT16 and v <= 65536, device uint16 [c, b] (2-byte
+ *               aligned): the compact map of the write-up's section 2.2.1,
+ *               half the bytes; every token id is read through it as is.
  *  fmt          fh_centroid_format.
  *  max_batch    largest B any call will pass (>= 1).
  *  max_probes   largest p any call will pass (1 <= max_probes <= c).
+ *  c2t_format   fh_c2t_format (0, the int32 map, when the field is left zero).
  */
 typedef struct {
   int32_t v, d, c, b;
@@ -100,10 +109,11 @@ typedef struct {
   const void* C;
   const uint8_t* C_q;
   const void* C_scales;
-  const int32_t* C2T;
+  const void* C2T;
   int32_t fmt;
   int32_t max_batch;
   int32_t max_probes;
+  int32_t c2t_format;
 } fh_head_desc;
 
 typedef struct fh_head fh_head;
@@ -213,6 +223,9 @@ fh_status fh_dense_head(fh_head* head, const void* hidden, int32_t B, float* log
  * attributes: make it before any stream capture begins. All calls on a
  * device share the scratch: launches that can overlap in time (unordered
  * streams, concurrent host threads) race and corrupt each other's results.
+ * Cost: every group of up to 8 hidden rows is one pass over E, so a call with
+ * B > 8 reads E about ceil(B / 8) times (fh_dense_head reads it once from
+ * B = 64 on, on the tensor cores).
  */
 #define FH_NOALLOC_MAX_ROWS 64
 fh_status fh_dense_head_noalloc(const void* E, int32_t v, int32_t d, const void* hidden, int32_t B,
@@ -234,6 +247,7 @@ const char* fh_status_string(fh_status status);
  * exercise that path).
  */
 fh_status fh_set_spin_budget(fh_head* head, int64_t cycles);
+
 
 /*
  * Introspection: FH_QUERY_WORKSPACE_BYTES, FH_QUERY_LAST_UNION (number of

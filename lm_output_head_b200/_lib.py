@@ -45,6 +45,9 @@ EXPORTED = (
     "fh_cluster_build", "fh_cluster_get_device_status",
 )
 
+FH_C2T_INT32 = 0
+FH_C2T_UINT16 = 1
+
 FH_NOALLOC_MAX_ROWS = 64
 
 
@@ -54,6 +57,7 @@ class HeadDesc(ctypes.Structure):
         ("E", ctypes.c_void_p), ("C", ctypes.c_void_p), ("C_q", ctypes.c_void_p),
         ("C_scales", ctypes.c_void_p), ("C2T", ctypes.c_void_p),
         ("fmt", ctypes.c_int32), ("max_batch", ctypes.c_int32), ("max_probes", ctypes.c_int32),
+        ("c2t_format", ctypes.c_int32),
     ]
 
 

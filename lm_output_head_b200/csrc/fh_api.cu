@@ -51,6 +51,7 @@ struct fh_head {
   uint32_t* b1_list_key = nullptr;     // [b1_list_cap]
   int32_t* b1_list_id = nullptr;       // [b1_list_cap]
   int b1_list_cap = 0;
+  C2TView c2t{};                       // the caller's C2T, int32 or uint16
   int words = 0;
   int b1_grid = 0;
   int dense_grid = 0;
@@ -236,7 +237,10 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   if (static_cast<long long>(D.c) * D.b != D.v) return FH_ERR_INVALID_ARG;
   if (D.d % 8) return FH_ERR_INVALID_ARG;
   if (D.max_batch < 1 || D.max_probes < 1 || D.max_probes > D.c) return FH_ERR_INVALID_ARG;
-  if (!D.E || !aligned(D.E, 16) || !D.C2T || !aligned(D.C2T, 4)) return FH_ERR_INVALID_ARG;
+  if (D.c2t_format != FH_C2T_INT32 && D.c2t_format != FH_C2T_UINT16) return FH_ERR_INVALID_ARG;
+  const bool c2t16 = D.c2t_format == FH_C2T_UINT16;
+  if (c2t16 && D.v > 65536) return FH_ERR_INVALID_ARG;  // token ids 0..v-1 must fit in 16 bits
+  if (!D.E || !aligned(D.E, 16) || !D.C2T || !aligned(D.C2T, c2t16 ? 2 : 4)) return FH_ERR_INVALID_ARG;
   if (D.fmt == FH_CENTROID_BF16) {
     if (!D.C || !aligned(D.C, 16)) return FH_ERR_INVALID_ARG;
   } else if (D.fmt == FH_CENTROID_INT4_G32 || D.fmt == FH_CENTROID_INT8_G32) {
@@ -258,6 +262,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   fh_head* h = new (std::nothrow) fh_head();
   if (!h) return FH_ERR_OOM;
   h->desc = D;
+  h->c2t = C2TView::make(D.C2T, c2t16);
   h->device = dev;
   h->num_sms = prop.multiProcessorCount;
   // leave room for the kernels' static shared memory
@@ -297,6 +302,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   const int words = (D.c + 31) / 32;
   const size_t o_keys1 = take(static_cast<size_t>(D.c) * 4);
   const size_t o_zbuf = take(static_cast<size_t>(D.v) * 4);
+  // candidate list of the fused decode: up to 4 p entries (the region aims at ~2 p keys)
   const size_t o_hist1 = take(static_cast<size_t>(kB1Bins) * 4);
   // candidate list of the fused decode: up to 4 p entries (the region aims at ~2 p keys)
   const int list_cap = static_cast<int>(std::min<size_t>(4 * mp, D.c));
@@ -360,7 +366,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
     }
     e = cudaMemsetAsync(h->ws, 0, h->ws_bytes, st);
     if (e != cudaSuccess) { status = cuda_fail(e); break; }
-    C2TCheckParams cp{D.C2T, h->c2t_counts, &h->sync->status, static_cast<long long>(D.v), D.v};
+    C2TCheckParams cp{h->c2t, h->c2t_counts, &h->sync->status, static_cast<long long>(D.v), D.v};
     e = launch_c2t_check(cp, st);
     if (e != cudaSuccess) { status = cuda_fail(e); break; }
     if (packed) {
@@ -375,7 +381,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
     if (e != cudaSuccess) { status = cuda_fail(e); break; }
     if (bad) { status = FH_ERR_INVALID_C2T; break; }
     // token rows in cluster-major order (C2T is a permutation: every read is in range)
-    e = launch_gather_cluster_major(static_cast<const uint16_t*>(D.E), D.C2T, h->Ecm, D.v, D.d, st);
+    e = launch_gather_cluster_major(static_cast<const uint16_t*>(D.E), h->c2t, h->Ecm, D.v, D.d, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) { status = cuda_fail(e); break; }
   } while (false);
@@ -490,7 +496,7 @@ fh_status fh_select_clusters(fh_head* h, const float* scores, int32_t B, int32_t
   SelectParams P{};
   P.in = scores;
   P.u_clusters = mode == FH_SAMPLE_GUMBEL ? u_clusters : nullptr;
-  P.C2T = h->desc.C2T;
+  P.C2T = h->c2t;
   P.sel = cluster_ids;
   P.status = &h->sync->status;
   P.c = h->desc.c;
@@ -513,7 +519,7 @@ fh_status fh_candidate_logits(fh_head* h, const void* hidden, int32_t B, int32_t
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   SelectParams P{};
   P.ids_in = cluster_ids;
-  P.C2T = h->desc.C2T;
+  P.C2T = h->c2t;
   P.sel = h->sel;
   P.cand_tok = h->cand_tok;
   P.row_ok = h->row_ok;
@@ -547,7 +553,7 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
     P.E = static_cast<const uint16_t*>(D.E);
     P.Ecm = h->Ecm;
     P.Crows = h->crows;
-    P.C2T = D.C2T;
+    P.C2T = h->c2t;
     P.hidden = static_cast<const uint16_t*>(hidden);
     P.u_clusters = gumbel ? u_clusters : nullptr;
     P.u_token = gumbel ? u_token : nullptr;
@@ -587,7 +593,7 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
   if (s != FH_OK) return s;
   SelectParams SP{};
   SP.in = h->keys;
-  SP.C2T = D.C2T;
+  SP.C2T = h->c2t;
   SP.sel = h->sel;
   SP.cand_tok = h->cand_tok;
   SP.status = &h->sync->status;
@@ -603,7 +609,7 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
     // de-duplicated across the batch: every chosen cluster's token rows are read once
     GroupParams GP{};
     GP.sel = h->sel;
-    GP.C2T = D.C2T;
+    GP.C2T = h->c2t;
     GP.Ecm = h->Ecm;
     GP.H = static_cast<const uint16_t*>(hidden);
     GP.cnt = h->g_cnt;

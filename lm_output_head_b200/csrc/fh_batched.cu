@@ -181,7 +181,7 @@ __device__ void write_candidates(const SelectParams& P, const int32_t* ssel, int
   const int nc = P.p * P.b;
   int32_t* out = P.cand_tok + static_cast<size_t>(row) * nc;
   for (int r = threadIdx.x; r < nc; r += kThreads)
-    out[r] = __ldg(P.C2T + static_cast<size_t>(ssel[r / P.b]) * P.b + r % P.b);
+    out[r] = P.C2T.at(static_cast<size_t>(ssel[r / P.b]) * P.b + r % P.b);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelectParams P) {

@@ -50,22 +50,6 @@
 namespace fh {
 namespace {
 
-#ifdef FH_TIMELINE
-// Development aid (off in the library build): globaltimer stamps per CTA.
-__device__ unsigned long long g_tl[1024 * 16 + 8];
-__device__ __forceinline__ void tl_mark(int i) {
-  if (threadIdx.x == 0) {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    g_tl[blockIdx.x * 16 + i] = t;
-  }
-}
-#define FH_TL(i) tl_mark(i)
-#define FH_TLV(i, v) (g_tl[blockIdx.x * 16 + (i)] = (v))
-#else
-#define FH_TL(i)
-#define FH_TLV(i, v)
-#endif
 
 static_assert(kB1Bins == 4 * kThreads, "each thread scans four histogram bins");
 
@@ -82,7 +66,7 @@ struct B1Misc {
   uint32_t bkey;
   int32_t bid;
   float edge_2p;
-  uint32_t nnote, base, prior_n;
+  uint32_t nnote, base, nlist;
   int32_t note_k[kNoteMax];
   uint32_t note_key[kNoteMax];
 };
@@ -116,7 +100,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   B1Misc* misc = reinterpret_cast<B1Misc*>(smem + P.off_misc);
   uint8_t* slots = smem + P.off_slots;  // per-warp row slots; the selection's scratch between phases
 
-  FH_TL(0);
 
   // ---------------- phase 1: centroid scores ----------------
   const uint32_t hbar = smem_addr(&misc->hbar);
@@ -127,9 +110,15 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   const int cstride = G * kWarps;
   const int n1 = cw < P.c ? (P.c - 1 - cw) / cstride + 1 : 0;  // <= 32 (host-checked)
   uint32_t wphase = 0;  // parity of this warp's slot barrier
-  // The centroid rows depend on no earlier kernel: the warp's first two start
-  // streaming before the wait for the preceding grid (programmatic dependent
-  // launch), which may still be finishing when this grid starts.
+  // h is requested first, then every warp's first two centroid rows: one into
+  // registers, one into its slot by a bulk copy
+  if (tid == 0) {
+    mbar_init(hbar, 1);
+    fence_mbar_init();
+    mbar_expect_tx(hbar, static_cast<uint32_t>(d * 2));
+    bulk_g2s(smem_addr(hraw), P.hidden, static_cast<uint32_t>(d * 2), hbar);
+    misc->nnote = 0u;
+  }
   if (lane == 0) {
     mbar_init(wbar, 1);
     fence_mbar_init();
@@ -147,24 +136,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     if constexpr (INT4) row_load_int4<NCH>(P.Crows + static_cast<size_t>(cw) * P.crow_bytes, d, q, sc);
     else if constexpr (INT8) row_load_int8<NCH>(P.Crows + static_cast<size_t>(cw) * P.crow_bytes, d, q8, sw8);
     else row_load_bf16<NCH>(reinterpret_cast<const uint16_t*>(P.Crows + static_cast<size_t>(cw) * P.crow_bytes), d, w);
-  }
-  // Phase 3 reads the chosen clusters' rows, scattered over all of Ecm: touch
-  // every 2 MB page of it once now (one L2 prefetch per page across the grid)
-  // so that their address translations are warm by then.
-  {
-    constexpr size_t kPage = size_t(2) << 20;
-    const size_t npages = (static_cast<size_t>(P.v) * d * 2 + kPage - 1) / kPage;
-    for (size_t pg = blockIdx.x + static_cast<size_t>(G) * tid; pg < npages; pg += static_cast<size_t>(G) * kThreads)
-      prefetch_l2(reinterpret_cast<const uint8_t*>(P.Ecm) + pg * kPage);
-  }
-  // h, the uniforms and the head's workspace state may come from the preceding grid
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (tid == 0) {
-    mbar_init(hbar, 1);
-    fence_mbar_init();
-    mbar_expect_tx(hbar, static_cast<uint32_t>(d * 2));
-    bulk_g2s(smem_addr(hraw), P.hidden, static_cast<uint32_t>(d * 2), hbar);
-    misc->nnote = 0u;
   }
   float ureg = 0.f;  // lane j holds u of item j
   if (gumbel && lane < n1) ureg = __ldg(P.u_clusters + cw + lane * cstride);
@@ -199,7 +170,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     hnorm = sqrtf(tot);
     __syncthreads();
   }
-  FH_TL(1);
   // the predicted region [L, U): from the last call's rank-2p key up to its
   // rank-p key plus twice their distance (identical arithmetic in every CTA)
   const float unit = gumbel ? 1.f : hnorm;
@@ -249,7 +219,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     }
   }
   __syncthreads();
-  FH_TL(2);
   // append this CTA's region keys to the candidate list
   const int nnote = min(static_cast<int>(misc->nnote), kNoteMax);
   if (tid == 0) misc->base = nnote ? atomicAdd(&P.sync->list_count, static_cast<uint32_t>(nnote)) : 0u;
@@ -263,7 +232,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   }
   __syncthreads();
   if (tid == 0) {
-    misc->prior_n = P.sync->last_in_range;  // the list length the last call saw (read while waiting)
     red_release_add_u32(&P.sync->arrive, 1u);  // keys, counts and list entries of this CTA are published
     // wait (bounded, with backoff) until every CTA has arrived
     int okw = 1;
@@ -276,9 +244,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
       }
     }
     misc->claim = okw;
+    misc->nlist = __ldcg(&P.sync->list_count);
   }
   __syncthreads();
-  FH_TL(3);
   bool ok = misc->claim != 0;
 
   // ---------------- phase 2: the boundary of the top p ----------------
@@ -287,43 +255,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   const int r_2p = min(c, 2 * p);
   uint32_t* skey = reinterpret_cast<uint32_t*>(slots);
   int32_t* sid = reinterpret_cast<int32_t*>(slots + up128(static_cast<size_t>(P.list_cap) * 4));
-  // The reads after the arrival go out together: the list length, this
-  // thread's histogram bins, and the list up to the length the last call saw
-  // (plus a margin); entries past that follow once the length is known.
-  uint32_t nlist = 0u;
-  uint4 hq = make_uint4(0u, 0u, 0u, 0u);
-  const uint32_t prior_n = misc->prior_n;
-  const int spec = min(P.list_cap, static_cast<int>(min(prior_n + prior_n / 4u + 64u, 0x7FFFFFFFu)));
-  auto load_list = [&](int from, int to) {
-    for (int base = from; base < to; base += 4 * kThreads) {
-      uint32_t kk[4];
-      int32_t ii[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int i = base + j * kThreads + tid;
-        if (i < to) {
-          kk[j] = __ldcg(P.list_key + i);
-          ii[j] = __ldcg(P.list_id + i);
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int i = base + j * kThreads + tid;
-        if (i < to) {
-          skey[i] = kk[j];
-          sid[i] = ii[j];
-        }
-      }
-    }
-  };
-  if (ok && region) {
-    nlist = __ldcg(&P.sync->list_count);
-    hq = __ldcg(reinterpret_cast<const uint4*>(P.hist) + (kB1Bins / 4 - 1 - tid));
-    load_list(0, spec);
-  }
+  const uint32_t nlist = misc->nlist;
   const bool use_list = region && nlist >= static_cast<uint32_t>(p) && nlist <= static_cast<uint32_t>(P.list_cap);
   const int nl = use_list ? static_cast<int>(nlist) : 0;
-  if (ok && nl > spec) load_list(spec, nl);
   const uint32_t bs_off =
       static_cast<uint32_t>(P.off_slots) +
       static_cast<uint32_t>(std::max(2 * up128(static_cast<size_t>(P.list_cap) * 4), up128(static_cast<size_t>(c) * 4)));
@@ -335,7 +269,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   }
   if (ok) {
     if (use_list) {
-      FH_TL(8);
+      const uint4 hq = __ldcg(reinterpret_cast<const uint4*>(P.hist) + (kB1Bins / 4 - 1 - tid));
+      for (int i = tid; i < nl; i += kThreads) {
+        skey[i] = __ldcg(P.list_key + i);
+        sid[i] = __ldcg(P.list_id + i);
+      }
       // bins from the top: thread t owns kB1Bins-1-4t (first) .. kB1Bins-4-4t
       const uint32_t hv[4] = {hq.w, hq.z, hq.y, hq.x};
       uint32_t total;
@@ -359,7 +297,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
         run += hv[j];
       }
       __syncthreads();
-      FH_TL(9);
       // the list holds every key the histogram counted; a crowded boundary bin takes the general path
       full = misc->m1 > static_cast<uint32_t>(kBoundEntries) || misc->total != nlist;
       if (!full) {
@@ -376,7 +313,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
           }
         }
         __syncthreads();
-        FH_TL(10);
         const uint32_t m1 = min(bs.nc, static_cast<uint32_t>(kBoundEntries));  // == misc->m1
         const uint32_t need = static_cast<uint32_t>(p) - misc->above;
         for (uint32_t a = tid; a < m1; a += kThreads) {
@@ -398,12 +334,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
           if (m1 != misc->m1) misc->m1 = 0xFFFFFFFFu;  // inconsistent counts: take the general path
         }
         __syncthreads();
-        FH_TL(11);
         full = misc->m1 == 0xFFFFFFFFu;
       }
     }
     if (full) {
       // the general exact selector over all c keys
+      __syncthreads();  // every thread is done with the list scratch before the keys overwrite it
       for (int i = tid; i < c / 4; i += kThreads)
         reinterpret_cast<uint4*>(skey)[i] = __ldcg(reinterpret_cast<const uint4*>(P.keys) + i);
       for (int i = (c / 4) * 4 + tid; i < c; i += kThreads) skey[i] = __ldcg(P.keys + i);
@@ -473,9 +409,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     fence_proxy_async_smem();  // the slots were generic scratch; bulk copies follow
     __syncthreads();
   }
-  FH_TL(4);
-  // a dependent grid may launch now; its CTAs start as this grid's CTAs leave the SMs
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // ---------------- phase 3: candidate rows ----------------
   // row r is slot r % b of the (r / b)-th chosen cluster; rows
@@ -500,8 +433,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     uint4 e[NCH];
     row_load_bf16<NCH>(P.Ecm + q0 * d, d, e);
     int t = 0;
-    if (lane == 0) t = __ldg(P.C2T + q0);
-    else if (lane == 1 && two) t = __ldg(P.C2T + q1);
+    if (lane == 0) t = P.C2T.at(q0);
+    else if (lane == 1 && two) t = P.C2T.at(q1);
     const int t0 = __shfl_sync(0xFFFFFFFFu, t, 0);
     const int t1 = two ? __shfl_sync(0xFFFFFFFFu, t, 1) : 0;
     const float z0 = row_dot_bf16_hs<NCH>(e, hs, d);
@@ -528,7 +461,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   best = warp_max_u64(best);
   if (lane == 0) misc->wbest[warp] = best;
   __syncthreads();
-  FH_TL(5);
 
   // ---------------- exit: the last CTA writes the token ----------------
   if (tid == 0) {
@@ -539,7 +471,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     misc->last = atom_acq_rel_add_u32(&P.sync->ticket, 1u) == static_cast<uint32_t>(G - 1);
   }
   __syncthreads();
-  FH_TL(6);
   if (!misc->last) return;
 
   const unsigned long long bw = __ldcg(P.best);
@@ -602,19 +533,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     __syncthreads();
     if (tid == 0) {
       const int idx = misc->claim != INT_MAX ? misc->claim : misc->lastpos;
-      P.out_tokens[0] = __ldg(P.C2T + static_cast<size_t>(ssel[idx / b]) * b + idx % b);
+      P.out_tokens[0] = P.C2T.at(static_cast<size_t>(ssel[idx / b]) * b + idx % b);
     }
   }
-#ifdef FH_TIMELINE
-  if (tid == 0) {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    g_tl[1024 * 16] = t;
-    g_tl[1024 * 16 + 1] = blockIdx.x;
-    g_tl[1024 * 16 + 2] = misc->full;
-    g_tl[1024 * 16 + 3] = misc->total;
-  }
-#endif
   // clear the histogram for the next call (every CTA has read it)
   if (region) reinterpret_cast<uint4*>(P.hist)[tid] = make_uint4(0, 0, 0, 0);
   if (tid == 0) {
@@ -651,30 +572,14 @@ cudaError_t launch_nch(const B1Params& P, int grid, size_t smem, int cfmt, cudaS
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  // programmatic dependent launch with the cooperative attribute; if a driver
-  // refuses the pair, launch cooperatively alone from then on (the kernel's
-  // griddepcontrol instructions are no-ops without the attribute)
-  static bool pdl_ok = true;
-  cfg.numAttrs = pdl_ok ? 2 : 1;
-  auto go = [&]() {
-    if (cfmt == kFmtInt4) return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, kFmtInt4>, P);
-    if (cfmt == kFmtInt8) return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, kFmtInt8>, P);
-    return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, kFmtBf16>, P);
-  };
-  cudaError_t e = go();
-  if (e != cudaSuccess && cfg.numAttrs == 2 && e != cudaErrorLaunchOutOfResources) {
-    (void)cudaGetLastError();
-    pdl_ok = false;
-    cfg.numAttrs = 1;
-    e = go();
-  }
-  return e;
+  cfg.numAttrs = 1;
+  if (cfmt == kFmtInt4) return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, kFmtInt4>, P);
+  if (cfmt == kFmtInt8) return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, kFmtInt8>, P);
+  return cudaLaunchKernelEx(&cfg, decode_b1_kernel<NCH, kFmtBf16>, P);
 }
 
 }  // namespace
@@ -689,11 +594,6 @@ size_t decode_b1_scratch_bytes(int c, int list_cap) {
   return keys + std::max(sizeof(BoundSmem), sizeof(SelectSmem));
 }
 
-#ifdef FH_TIMELINE
-extern "C" int fh_timeline_read(unsigned long long* host, int n) {
-  return static_cast<int>(cudaMemcpyFromSymbol(host, g_tl, static_cast<size_t>(n) * 8));
-}
-#endif
 
 cudaError_t launch_decode_b1(const B1Params& P, int grid, size_t smem, int cfmt, int nch, cudaStream_t st) {
   switch (nch) {

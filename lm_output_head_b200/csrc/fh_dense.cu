@@ -131,7 +131,7 @@ namespace {
 __global__ void c2t_count_kernel(const C2TCheckParams P) {
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < P.n;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int t = P.C2T[i];
+    const int t = P.C2T.at(static_cast<size_t>(i));
     if (t < 0 || t >= P.v) atomicExch(P.bad, 1);
     else atomicAdd(P.counts + t, 1u);
   }
@@ -160,21 +160,21 @@ __global__ void repack_kernel(const RepackParams P) {
 
 // Cluster-major copy of E: row r = k*b + j holds E[C2T[k][j]] (C2T already
 // verified to be a permutation of 0..v-1), 16 bytes per thread step.
-__global__ void gather_cluster_major_kernel(const uint16_t* E, const int32_t* C2T, uint16_t* out, int v, int d) {
+__global__ void gather_cluster_major_kernel(const uint16_t* E, const C2TView C2T, uint16_t* out, int v, int d) {
   const int chunks = d / 8;
   const long long total = static_cast<long long>(v) * chunks;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long r = i / chunks;
     const int q = static_cast<int>(i - r * chunks);
-    const int t = __ldg(C2T + r);
+    const int t = C2T.at(static_cast<size_t>(r));
     reinterpret_cast<uint4*>(out + r * d)[q] = __ldg(reinterpret_cast<const uint4*>(E + static_cast<size_t>(t) * d) + q);
   }
 }
 
 }  // namespace
 
-cudaError_t launch_gather_cluster_major(const uint16_t* E, const int32_t* C2T, uint16_t* out, int v, int d,
+cudaError_t launch_gather_cluster_major(const uint16_t* E, C2TView C2T, uint16_t* out, int v, int d,
                                         cudaStream_t st) {
   gather_cluster_major_kernel<<<2048, 256, 0, st>>>(E, C2T, out, v, d);
   return cudaGetLastError();

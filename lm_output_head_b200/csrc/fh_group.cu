@@ -167,8 +167,8 @@ __global__ void __launch_bounds__(kGroupWarps * 32, 1) group_kernel(const GroupP
     const int k = P.ulist[ui];
     const int r0 = static_cast<int>(P.off[k]), r1 = static_cast<int>(P.off[k + 1]);
     const uint16_t* ek = P.Ecm + static_cast<size_t>(k) * b * d;  // the cluster's 16 rows, contiguous
-    const int tok_a = __ldg(P.C2T + static_cast<size_t>(k) * b + g);
-    const int tok_b = __ldg(P.C2T + static_cast<size_t>(k) * b + g + 8);
+    const int tok_a = P.C2T.at(static_cast<size_t>(k) * b + g);
+    const int tok_b = P.C2T.at(static_cast<size_t>(k) * b + g + 8);
     for (int rb = r0; rb < r1; rb += 8 * kChunks) {
       const int nrows = min(8 * kChunks, r1 - rb);
       const int nch = (nrows + 7) / 8;

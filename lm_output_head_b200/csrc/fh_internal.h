@@ -14,17 +14,35 @@ namespace fh {
 constexpr int kMaxD = 2560;
 constexpr long long kWaitBudget = 4000000000LL;      // bulk-copy waits (~2 s)
 constexpr long long kDefaultSpinBudget = 2000000000LL;  // device-wide waits (~1 s)
-constexpr int kB1Bins = 2048;  // histogram bins of the fused B = 1 selection
+constexpr int kB1Bins = 2048;  // histogram bins of the fused B = 1 selection's predicted region
 
 // Centroid row formats as the kernels see them (the same values as fh_centroid_format):
 // bf16 rows; packed INT4 g32 rows [d/2 codes][d/16 scale bytes]; packed INT8 g32 rows
 // [d codes][d/16 scale bytes] (packed rows padded to 16 bytes).
 constexpr int kFmtBf16 = 0, kFmtInt4 = 1, kFmtInt8 = 2;
 
+// The caller's cluster-to-token map C2T [c, b] (write-up section 1.2.1):
+// int32 entries, or uint16 entries when v <= 65536 (the compact map). One
+// word: the map's address, with bit 0 set for uint16 entries (every map is at
+// least 2-byte aligned), so a kernel holds it in one register pair.
+struct C2TView {
+  uintptr_t bits;
+  static C2TView make(const void* ptr, bool u16) {
+    return C2TView{reinterpret_cast<uintptr_t>(ptr) | (u16 ? 1u : 0u)};
+  }
+#ifdef __CUDACC__
+  __device__ __forceinline__ int32_t at(size_t q) const {
+    const uintptr_t a = bits & ~static_cast<uintptr_t>(1);
+    return (bits & 1u) ? static_cast<int32_t>(__ldg(reinterpret_cast<const unsigned short*>(a) + q))
+                       : __ldg(reinterpret_cast<const int32_t*>(a) + q);
+  }
+#endif
+};
+
 // Workspace words at the start of the workspace.
 struct SyncWords {
   int32_t status;
-  uint32_t arrive;        // grid barrier arrivals
+  uint32_t arrive;        // batched decode: grid barrier arrivals (unused by the fused call)
   uint32_t ticket;        // kernel exit tickets (last CTA finalises)
   uint32_t union_count;   // distinct clusters of the last batched decode
   uint32_t epoch;         // fused B = 1 calls so far
@@ -32,6 +50,8 @@ struct SyncWords {
   float prior_p[2];       // fused call: keys of rank p and 2p in the last call of each mode
   float prior_2p[2];      //   [greedy: key / |h|, sampling: key]
   uint32_t prior_ok[2];   // the predictions of a mode hold values
+  float prior_T[2];       // the temperature and probe count they were taken at
+  int32_t prior_pc[2];
   uint32_t last_in_range; // keys the last fused call counted in its histogram
   uint32_t list_count;    // fused call: entries appended to the candidate list
 };
@@ -39,8 +59,8 @@ struct SyncWords {
 struct B1Params {
   const uint16_t* E;
   const uint16_t* Ecm;    // cluster-major token rows: row k*b + j = E[C2T[k][j]]
-  const uint8_t* Crows;   // bf16 rows (d*2 bytes) or packed INT4 rows (crow_bytes)
-  const int32_t* C2T;
+  const uint8_t* Crows;   // bf16 rows (d*2 bytes) or packed INT4 / INT8 rows (crow_bytes)
+  C2TView C2T;
   const uint16_t* hidden;
   const float* u_clusters;
   const float* u_token;
@@ -48,8 +68,8 @@ struct B1Params {
   int32_t* out_cluster_ids;
   float* out_max_logit;
   uint32_t* keys;         // workspace [c]: order-preserving keys of the clusters
-  float* z_buf;           // workspace [c*b]: logit of slot k*b + j of the chosen clusters (sampling)
-  uint32_t* hist;         // workspace [kB1Bins]: counts of keys per bin near the predicted boundary
+  float* z_buf;           // workspace [c*b]: logit of slot k*b + j of the scored clusters (sampling)
+  uint32_t* hist;         // workspace [kB1Bins]: counts of keys per bin of the predicted region
   uint32_t* list_key;     // workspace [list_cap]: keys in the predicted region (candidate list)
   int32_t* list_id;       // workspace [list_cap]: their cluster ids
   int list_cap;
@@ -81,7 +101,7 @@ struct SelectParams {
   const float* in;         // [B, c] scores or keys
   const float* u_clusters; // [B, c] when perturb
   const int32_t* ids_in;   // [B, p] explicit ids (sort mode) or null
-  const int32_t* C2T;
+  C2TView C2T;
   int32_t* sel;            // [B, p] ascending
   int32_t* cand_tok;       // [B, p*b] canonical token ids, or null
   int32_t* row_ok;         // [B] (sort mode) or null
@@ -148,7 +168,7 @@ struct GemmParams {
 
 struct GroupParams {
   const int32_t* sel;       // [B, p] chosen clusters per row, ascending
-  const int32_t* C2T;       // [c, b]
+  C2TView C2T;              // [c, b]
   const uint16_t* Ecm;      // [v, d] cluster-major token rows: row k*b + j = E[C2T[k][j]]
   const uint16_t* H;        // [B, d]
   uint32_t* cnt;            // [c] workspace: rows per cluster
@@ -164,7 +184,7 @@ struct GroupParams {
 };
 
 struct C2TCheckParams {
-  const int32_t* C2T;
+  C2TView C2T;
   uint32_t* counts;         // [v]
   int* bad;
   long long n;
@@ -192,7 +212,7 @@ cudaError_t launch_dense(const DenseParams& P, int grid, size_t smem, int nch, c
 cudaError_t launch_c2t_check(const C2TCheckParams& P, cudaStream_t st);
 cudaError_t launch_repack(const RepackParams& P, cudaStream_t st);
 // Cluster-major copy of the token rows: out[k*b + j] = E[C2T[k][j]].
-cudaError_t launch_gather_cluster_major(const uint16_t* E, const int32_t* C2T, uint16_t* out, int v, int d,
+cudaError_t launch_gather_cluster_major(const uint16_t* E, C2TView C2T, uint16_t* out, int v, int d,
                                         cudaStream_t st);
 // tcgen05 GEMM (B >= 64): streamed rows bf16 [rows, d] through TMA, or packed INT4 / INT8 rows; H bf16 [nb, d].
 cudaError_t launch_gemm(const GemmParams& P, const void* rows_bf16, const void* H, int num_sms, cudaStream_t st);

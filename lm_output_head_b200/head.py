@@ -51,7 +51,8 @@ def bf16_from_bits(bits: np.ndarray, device="cuda") -> torch.Tensor:
 class FlashHead:
     """A FlashHead retrieval head bound to device tensors (borrowed, kept alive here).
 
-    ``E`` bf16 [v, d]; ``C2T`` int32 [c, b]; centroids either ``C`` bf16 [c, d],
+    ``E`` bf16 [v, d]; ``C2T`` int32 [c, b], or uint16 [c, b] (int16 bits are
+    read as uint16) for v <= 65536; centroids either ``C`` bf16 [c, d],
     or ``C_q`` with ``C_scales`` bf16 [c, d/32]: uint8 [c, d/2] packed INT4
     codes, or int8 [c, d] INT8 codes (the dtype picks the format).
     """
@@ -62,7 +63,8 @@ class FlashHead:
         self._lib = _lib.load()
         self._h = None
         E = _dev(E, "E", _BF16, 2)
-        C2T = _dev(C2T, "C2T", (torch.int32,), 2)
+        C2T = _dev(C2T, "C2T", (torch.int32, torch.uint16, torch.int16), 2)
+        c2t_format = _lib.FH_C2T_INT32 if C2T.dtype == torch.int32 else _lib.FH_C2T_UINT16
         v, d = E.shape
         c, b = C2T.shape
         if C is not None:
@@ -84,7 +86,7 @@ class FlashHead:
                              C_q=C_q.data_ptr() if C_q is not None else None,
                              C_scales=C_scales.data_ptr() if C_scales is not None else None,
                              C2T=C2T.data_ptr(), fmt=fmt, max_batch=self.max_batch,
-                             max_probes=self.max_probes)
+                             max_probes=self.max_probes, c2t_format=c2t_format)
         h = ctypes.c_void_p()
         with torch.cuda.device(E.device):
             _check(self._lib.fh_create(ctypes.byref(desc), _stream(), ctypes.byref(h)), "fh_create")
