@@ -51,6 +51,7 @@ struct fh_head {
   uint32_t* b1_list_key = nullptr;     // [b1_list_cap]
   int32_t* b1_list_id = nullptr;       // [b1_list_cap]
   int b1_list_cap = 0;
+  B1Hot* b1_hot = nullptr;             // the fused call's shared counters
   C2TView c2t{};                       // the caller's C2T, int32 or uint16
   int words = 0;
   int b1_grid = 0;
@@ -302,12 +303,13 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   const int words = (D.c + 31) / 32;
   const size_t o_keys1 = take(static_cast<size_t>(D.c) * 4);
   const size_t o_zbuf = take(static_cast<size_t>(D.v) * 4);
-  // candidate list of the fused decode: up to 4 p entries (the region aims at ~2 p keys)
+  // predicted-region histogram of the fused decode
   const size_t o_hist1 = take(static_cast<size_t>(kB1Bins) * 4);
   // candidate list of the fused decode: up to 4 p entries (the region aims at ~2 p keys)
   const int list_cap = static_cast<int>(std::min<size_t>(4 * mp, D.c));
   const size_t o_lkey = take(static_cast<size_t>(list_cap) * 4);
   const size_t o_lid = take(static_cast<size_t>(list_cap) * 4);
+  const size_t o_hot = take(sizeof(B1Hot));
   const bool packed = D.fmt != FH_CENTROID_BF16;
   const size_t o_crow = packed ? take(static_cast<size_t>(D.c) * h->crow_bytes) : 0;
   h->ws_bytes = off;
@@ -343,6 +345,7 @@ fh_status fh_create(const fh_head_desc* desc, fh_stream_t stream, fh_head** out)
   h->b1_list_key = reinterpret_cast<uint32_t*>(h->ws + o_lkey);
   h->b1_list_id = reinterpret_cast<int32_t*>(h->ws + o_lid);
   h->b1_list_cap = list_cap;
+  h->b1_hot = reinterpret_cast<B1Hot*>(h->ws + o_hot);
   h->words = words;
   h->crows = packed ? h->ws + o_crow : static_cast<const uint8_t*>(D.C);
 
@@ -566,7 +569,7 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
     P.list_key = h->b1_list_key;
     P.list_id = h->b1_list_id;
     P.list_cap = h->b1_list_cap;
-    P.best = h->best;
+    P.hot = h->b1_hot;
     P.sync = h->sync;
     P.v = D.v;
     P.d = D.d;

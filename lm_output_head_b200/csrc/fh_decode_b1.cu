@@ -221,7 +221,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   __syncthreads();
   // append this CTA's region keys to the candidate list
   const int nnote = min(static_cast<int>(misc->nnote), kNoteMax);
-  if (tid == 0) misc->base = nnote ? atomicAdd(&P.sync->list_count, static_cast<uint32_t>(nnote)) : 0u;
+  if (tid == 0)
+    misc->base = nnote ? static_cast<uint32_t>(atomicAdd(&P.hot->arrive_list, static_cast<unsigned long long>(nnote)))
+                       : 0u;
   __syncthreads();
   for (int i = tid; i < nnote; i += kThreads) {
     const uint32_t at = misc->base + static_cast<uint32_t>(i);
@@ -232,11 +234,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   }
   __syncthreads();
   if (tid == 0) {
-    red_release_add_u32(&P.sync->arrive, 1u);  // keys, counts and list entries of this CTA are published
+    red_release_add_u64(&P.hot->arrive_list, 1ull << 32);  // keys, counts and list entries of this CTA are published
     // wait (bounded, with backoff) until every CTA has arrived
     int okw = 1;
     const long long t0 = clock64();
-    while (ld_acquire_u32(&P.sync->arrive) < static_cast<uint32_t>(G)) {
+    unsigned long long av;
+    while (((av = ld_acquire_u64(&P.hot->arrive_list)) >> 32) < static_cast<unsigned long long>(G)) {
       __nanosleep(32);
       if (clock64() - t0 > P.spin_budget) {
         okw = 0;
@@ -244,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
       }
     }
     misc->claim = okw;
-    misc->nlist = __ldcg(&P.sync->list_count);
+    misc->nlist = static_cast<uint32_t>(av);
   }
   __syncthreads();
   bool ok = misc->claim != 0;
@@ -299,6 +302,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
       __syncthreads();
       // the list holds every key the histogram counted; a crowded boundary bin takes the general path
       full = misc->m1 > static_cast<uint32_t>(kBoundEntries) || misc->total != nlist;
+      if (!full) {
+        // the clusters above the boundary bin are certain: start reading their
+        // token rows into L2 now, under the rest of the selection
+        const int t1 = static_cast<int>(misc->t1);
+        for (int i = static_cast<int>(blockIdx.x) + G * tid; i < nl; i += G * kThreads) {
+          const int k = sid[i];
+          if (k >= 0 && k < c && region_bin(key2f(skey[i]), L, S) > t1)
+            bulk_prefetch_l2(P.Ecm + static_cast<size_t>(k) * b * d, static_cast<uint32_t>(b * d * 2));
+        }
+      }
       if (!full) {
         // gather the boundary bin's entries (their bins agree with phase 1), rank them exactly
         const int t1 = static_cast<int>(misc->t1);
@@ -466,14 +479,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
   if (tid == 0) {
     unsigned long long m = 0ull;
     for (int i = 0; i < kWarps; ++i) m = misc->wbest[i] > m ? misc->wbest[i] : m;
-    if (m) atomicMax(P.best, m);
+    if (m) atomicMax(&P.hot->best, m);
     // acq_rel: this CTA's maximum and logits are published; the last CTA sees everyone's
-    misc->last = atom_acq_rel_add_u32(&P.sync->ticket, 1u) == static_cast<uint32_t>(G - 1);
+    misc->last = atom_acq_rel_add_u32(&P.hot->ticket, 1u) == static_cast<uint32_t>(G - 1);
   }
   __syncthreads();
   if (!misc->last) return;
 
-  const unsigned long long bw = __ldcg(P.best);
+  const unsigned long long bw = __ldcg(&P.hot->best);
   if (tid == 0) {
     if (!gumbel) P.out_tokens[0] = best_token(bw);
     if (P.out_max_logit) P.out_max_logit[0] = best_logit(bw);
@@ -557,10 +570,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
       P.sync->last_in_range = region ? misc->total : 0u;
       P.sync->last_full = misc->full;
     }
-    *P.best = 0ull;
-    P.sync->arrive = 0u;
-    P.sync->ticket = 0u;
-    P.sync->list_count = 0u;
+    P.hot->best = 0ull;
+    P.hot->arrive_list = 0ull;
+    P.hot->ticket = 0u;
     P.sync->epoch = P.sync->epoch + 1u;  // calls on one head are stream-ordered
   }
 }

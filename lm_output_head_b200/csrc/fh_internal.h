@@ -53,7 +53,17 @@ struct SyncWords {
   float prior_T[2];       // the temperature and probe count they were taken at
   int32_t prior_pc[2];
   uint32_t last_in_range; // keys the last fused call counted in its histogram
-  uint32_t list_count;    // fused call: entries appended to the candidate list
+};
+
+// Counters that every CTA of a fused B = 1 call updates or polls, each on a
+// 128-byte line of its own (workspace; zero between calls). The arrival count
+// and the candidate list's length share one 64-bit word: a CTA reserves its
+// list entries (low half) before it arrives (high half), so the poll that sees
+// the last arrival also reads the final length.
+struct B1Hot {
+  alignas(128) unsigned long long arrive_list;  // CTAs arrived << 32 | list entries reserved
+  alignas(128) uint32_t ticket;          // exit tickets (the last CTA finalises)
+  alignas(128) unsigned long long best;  // packed (logit, token) maximum over the candidates
 };
 
 struct B1Params {
@@ -73,7 +83,7 @@ struct B1Params {
   uint32_t* list_key;     // workspace [list_cap]: keys in the predicted region (candidate list)
   int32_t* list_id;       // workspace [list_cap]: their cluster ids
   int list_cap;
-  unsigned long long* best;
+  B1Hot* hot;
   SyncWords* sync;
   int v, d, c, b, p;
   int crow_bytes;
