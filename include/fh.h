@@ -307,6 +307,20 @@ fh_status fh_speculative_verify(fh_head* head, const float* logits, const int32_
 fh_status fh_adaptive_probes(fh_head* head, const float* scores, int32_t B, float tau, int32_t p_min,
                              int32_t p_max, float T, int32_t* out_p, fh_stream_t stream);
 
+/*
+ * Hot-cluster residency (write-up section 2.2.1: the token rows of frequently
+ * used clusters kept in fast on-chip memory). Requests into L2 the token rows
+ * of the given clusters (their b x d bf16 block in the head's cluster-major
+ * copy of E) and their C2T rows, on `stream`, and returns without waiting: a
+ * serving loop passes the clusters it expects the next decode to choose. It
+ * only warms a cache; no result of any call depends on it.
+ *  cluster_ids  device int32 [n], each in [0, c); an id out of range is skipped
+ *               and FH_ERR_OUT_OF_RANGE is recorded in the device status.
+ * n >= 0 (0: nothing is launched). FH_ERR_INVALID_ARG for a null head, n < 0,
+ * or a null cluster_ids with n > 0.
+ */
+fh_status fh_prefetch_clusters(fh_head* head, const int32_t* cluster_ids, int32_t n, fh_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -38,7 +38,7 @@ EXPORTED = (
     "fh_create", "fh_destroy", "fh_centroid_scores", "fh_select_clusters",
     "fh_candidate_logits", "fh_decode", "fh_dense_head", "fh_get_device_status",
     "fh_status_string", "fh_set_spin_budget", "fh_query", "fh_dense_head_noalloc", "fh_speculative_verify",
-    "fh_adaptive_probes",
+    "fh_adaptive_probes", "fh_prefetch_clusters",
     # include/fh_cluster.h
     "fh_cluster_create", "fh_cluster_destroy", "fh_cluster_normalize", "fh_cluster_seed",
     "fh_cluster_gather", "fh_cluster_similarities", "fh_cluster_assign", "fh_cluster_update",
@@ -108,6 +108,8 @@ def load() -> ctypes.CDLL:
     lib.fh_speculative_verify.restype = ctypes.c_int
     lib.fh_adaptive_probes.argtypes = [vp, vp, i32, f32, i32, i32, f32, vp, vp]
     lib.fh_adaptive_probes.restype = ctypes.c_int
+    lib.fh_prefetch_clusters.argtypes = [vp, vp, i32, vp]
+    lib.fh_prefetch_clusters.restype = ctypes.c_int
     pi32 = ctypes.POINTER(ctypes.c_int32)
     lib.fh_cluster_create.argtypes = [i32, i32, i32, vp, ctypes.POINTER(vp)]
     lib.fh_cluster_destroy.argtypes = [vp]

@@ -722,4 +722,11 @@ fh_status fh_adaptive_probes(fh_head* h, const float* scores, int32_t B, float t
   return e == cudaSuccess ? FH_OK : cuda_fail(e);
 }
 
+fh_status fh_prefetch_clusters(fh_head* h, const int32_t* cluster_ids, int32_t n, fh_stream_t stream) {
+  if (!h || n < 0 || (n > 0 && !cluster_ids)) return FH_ERR_INVALID_ARG;
+  cudaError_t e = launch_prefetch_clusters(h->Ecm, h->c2t, h->desc.c, h->desc.b, h->desc.d, cluster_ids, n,
+                                           &h->sync->status, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FH_OK : cuda_fail(e);
+}
+
 }  // extern "C"

@@ -210,6 +210,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
       const int bn = region ? region_bin(key, L, S) : -1;
       if (bn >= 0) {
         red_relaxed_add_u32(P.hist + bn, 1u);
+        // in the region's upper half, i.e. above the predicted rank-p key by half
+        // the predicted gap to rank 2p: almost surely chosen, so its token rows
+        // start towards L2 now (the post-barrier prefetch covers the rest)
+        if (bn >= kB1Bins / 2 && k < P.c)
+          bulk_prefetch_l2(P.Ecm + static_cast<size_t>(k) * P.b * P.d, static_cast<uint32_t>(P.b * P.d * 2));
         const uint32_t at = atomicAdd(&misc->nnote, 1u);
         if (at < static_cast<uint32_t>(kNoteMax)) {
           misc->note_k[at] = k;
@@ -573,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_b1_kernel(const B1Params P
     P.hot->best = 0ull;
     P.hot->arrive_list = 0ull;
     P.hot->ticket = 0u;
-    P.sync->epoch = P.sync->epoch + 1u;  // calls on one head are stream-ordered
+    red_relaxed_add_u32(&P.sync->epoch, 1u);  // a count of calls; nothing waits for it
   }
 }
 

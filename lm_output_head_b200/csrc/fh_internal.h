@@ -36,6 +36,10 @@ struct C2TView {
     return (bits & 1u) ? static_cast<int32_t>(__ldg(reinterpret_cast<const unsigned short*>(a) + q))
                        : __ldg(reinterpret_cast<const int32_t*>(a) + q);
   }
+  __device__ __forceinline__ const void* ptr() const {
+    return reinterpret_cast<const void*>(bits & ~static_cast<uintptr_t>(1));
+  }
+  __device__ __forceinline__ size_t elem_bytes() const { return (bits & 1u) ? 2u : 4u; }
 #endif
 };
 
@@ -238,6 +242,10 @@ cudaError_t launch_spec_verify(const float* logits, int v, const int32_t* cand, 
 // Adaptive probe count per row of centroid scores (one CTA per row).
 cudaError_t launch_adaptive_probes(const float* scores, int B, int c, float tau, int p_min, int p_max, float T,
                                    int32_t* out_p, cudaStream_t st);
+
+// L2 prefetch of the token rows (cluster-major copy) and C2T rows of n clusters.
+cudaError_t launch_prefetch_clusters(const uint16_t* Ecm, C2TView C2T, int c, int b, int d, const int32_t* ids, int n,
+                                     int* status, cudaStream_t st);
 
 // Opt-in shared memory attribute for every instantiation (called once per device).
 cudaError_t set_kernel_attributes(int max_smem);

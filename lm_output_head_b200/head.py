@@ -179,6 +179,12 @@ class FlashHead:
                                             _ptr(out), _stream(stream)), "fh_adaptive_probes")
         return out
 
+    def prefetch_clusters(self, cluster_ids: torch.Tensor, stream=None):
+        """Start reading the token rows of these clusters into L2 (``fh_prefetch_clusters``)."""
+        cluster_ids = _dev(cluster_ids, "cluster_ids", (torch.int32,), 1)
+        _check(self._lib.fh_prefetch_clusters(self._h, _ptr(cluster_ids), int(cluster_ids.shape[0]),
+                                              _stream(stream)), "fh_prefetch_clusters")
+
     def decode(self, hidden: torch.Tensor, p: int, *, mode: str = "greedy", T: float = 1.0,
                u_clusters: Optional[torch.Tensor] = None, u_token: Optional[torch.Tensor] = None,
                out_tokens: Optional[torch.Tensor] = None, out_cluster_ids: Optional[torch.Tensor] = None,

@@ -12,6 +12,7 @@ timed repeats, each on a cold L2 (a buffer twice the L2 written and read back
 before it, outside the events); one JSON line per case.
 
     python -m lm_output_head_b200.microbench.batched_head [--repeats N] [--cases 4:256,3:32,2:16,2:4,2:1]
+    python -m lm_output_head_b200.microbench.batched_head --residency 4:256 [--repeats N]
 """
 from __future__ import annotations
 
@@ -174,6 +175,73 @@ def run_b1(cfg_id, steps, int8=False):
         "peak_kind": kind, "head_copies": n_copies, "device_status": status}), flush=True)
 
 
+def run_residency(cfg_id, B, repeats):
+    """Hot-cluster residency on a batch whose planted clusters recur (write-up
+    section 2.2.1). Three protocols, each call after a cold-L2 flush: (a) the
+    decode alone; (b) the recurring clusters' token rows requested into L2 by
+    fh_prefetch_clusters and landed before the events (an ideal resident
+    cache: the most any residency scheme can save); (c) the same request issued
+    inside the events just before the decode (no cache kept across steps)."""
+    import numpy as np
+    import torch
+    import synth
+    import lm_output_head_b200 as fh
+    cfg, head, hid, _ = synth.make_config(cfg_id, n_states=max(B, 64))
+    dev = "cuda"
+    E = fh.bf16_from_bits(head.E, dev)
+    C2T = torch.from_numpy(head.C2T).to(dev)
+    if head.C_q is not None:
+        dh = fh.FlashHead(E, C2T, C_q=torch.from_numpy(head.C_q).to(dev),
+                          C_scales=fh.bf16_from_bits(head.C_scales, dev), max_batch=B, max_probes=cfg.p)
+    else:
+        dh = fh.FlashHead(E, C2T, C=fh.bf16_from_bits(head.C, dev), max_batch=B, max_probes=cfg.p)
+    H = fh.bf16_from_bits(hid.H[:B], dev)
+    planted = hid.planted[:B]
+    hot_np = np.unique(planted[planted >= 0]).astype(np.int32)
+    hot = torch.from_numpy(hot_np).to(dev)
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    tok = torch.empty(B, dtype=torch.int32, device=dev)
+
+    def once(pre, inside):
+        flush.fill_(1)
+        flush.view(torch.int64).sum()
+        if pre:
+            dh.prefetch_clusters(hot)
+            torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        if inside:
+            dh.prefetch_clusters(hot)
+        dh.decode(H, cfg.p, out_tokens=tok)
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) * 1e3
+
+    for _ in range(3):
+        once(False, False)
+    res = {"cold": [], "hot_resident": [], "hot_requested_in_step": []}
+    for _ in range(repeats):  # interleaved, so drift affects all three alike
+        res["cold"].append(once(False, False))
+        res["hot_resident"].append(once(True, False))
+        res["hot_requested_in_step"].append(once(False, True))
+    union = dh.query(1)
+    med = {k: round(statistics.median(v), 2) for k, v in res.items()}
+    hot_bytes = len(hot_np) * (cfg.b * cfg.d * 2 + cfg.b * 4)
+    rec = {"workload": f"config {cfg_id}: v{cfg.v} d{cfg.d} c{cfg.c} b{cfg.b} p{cfg.p}, B={B}, "
+                       f"{len(hot_np)} recurring planted clusters",
+           "decode_us_median": med, "hot_clusters": len(hot_np), "hot_token_row_bytes": int(hot_bytes),
+           "union_clusters": union,
+           "union_token_row_bytes": int(union * (cfg.b * cfg.d * 2 + cfg.b * 4)),
+           "saving_if_resident_us": round(med["cold"] - med["hot_resident"], 2),
+           "saving_if_resident_frac": round((med["cold"] - med["hot_resident"]) / med["cold"], 4),
+           "protocol": f"{repeats} interleaved repeats of each protocol, 2 x L2 written and read back before "
+                       "every call, medians", "device_status": dh.device_status()}
+    dh.close()
+    print(json.dumps(rec), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--repeats", type=int, default=20)
@@ -181,7 +249,13 @@ def main():
                     help="comma-separated config:batch pairs (batch 1: the fused kernel, back to back; "
                          "config 'NQ8' = config N with INT8 centroids, batch 1 only)")
     ap.add_argument("--b1-steps", type=int, default=1000)
+    ap.add_argument("--residency", default=None, metavar="CONFIG:BATCH",
+                    help="instead of the cases: the hot-cluster residency experiment on this config and batch")
     args = ap.parse_args()
+    if args.residency:
+        cs, bs = args.residency.split(":")
+        run_residency(int(cs), int(bs), args.repeats)
+        return
     for case in args.cases.split(","):
         cs, bs = case.split(":")
         int8 = cs.endswith("Q8")
