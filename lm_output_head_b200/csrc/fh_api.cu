@@ -170,9 +170,17 @@ fh_status launch_candidates_rows(fh_head* h, const void* hidden, int32_t B, int3
   return e == cudaSuccess ? FH_OK : cuda_fail(e);
 }
 
-// Batches of at least this many hidden rows score centroids (and run the
-// dense head) on the tensor cores; smaller ones stream rows on CUDA cores.
+// Batches of at least this many hidden rows run the dense head on the tensor
+// cores; smaller ones stream E on CUDA cores.
 constexpr int kGemmMinBatch = 64;
+
+// Centroid scores move to the tensor cores at a smaller batch: the CUDA-core
+// kernel's time grows with B (one FMA per element and row) while the GEMM's is
+// flat below 128 rows. Crossovers measured on B200 with a cold L2 (c 8016-9496,
+// d 2048-2560): bf16 centroids 45 vs 34 us at B = 8; INT4 / INT8 centroids,
+// dequantised to hi + lo pairs for the MMA, 32-36 vs 46 us at B = 8 and 54-58
+// vs 46 us at B = 16.
+int scores_gemm_min_batch(int fmt) { return fmt == FH_CENTROID_BF16 ? 8 : 16; }
 
 // tcgen05 GEMM over blocks of up to 256 hidden rows. epi 0: out[r][k] =
 // scores (mode 0) or Gumbel keys (mode 1) of A = the centroids; epi 1: packed
@@ -484,7 +492,7 @@ fh_status fh_centroid_scores(fh_head* h, const void* hidden, int32_t B, float* s
   fh_status s = check_call(h, hidden, B);
   if (s != FH_OK) return s;
   if (!scores || !aligned(scores, 4)) return FH_ERR_INVALID_ARG;
-  if (B >= kGemmMinBatch)
+  if (B >= scores_gemm_min_batch(h->desc.fmt))
     return launch_gemm_rows(h, hidden, B, 0, 0, 1.f, nullptr, scores, reinterpret_cast<cudaStream_t>(stream));
   return launch_scores_rows(h, hidden, B, 0, 1.f, nullptr, scores, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -590,7 +598,7 @@ fh_status fh_decode(fh_head* h, const void* hidden, int32_t B, int32_t p, int32_
   }
 
   // batched path: keys -> per-row select -> candidates -> epilogue
-  s = B >= kGemmMinBatch
+  s = B >= scores_gemm_min_batch(D.fmt)
           ? launch_gemm_rows(h, hidden, B, 0, gumbel ? 1 : 0, gumbel ? T : 1.f, u_clusters, h->keys, st)
           : launch_scores_rows(h, hidden, B, gumbel ? 1 : 0, gumbel ? T : 1.f, u_clusters, h->keys, st);
   if (s != FH_OK) return s;
