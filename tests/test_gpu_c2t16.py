@@ -4,7 +4,7 @@ v <= 65536) through the C ABI (needs a B200).
 A head built on the uint16 map must give exactly the outputs of the same head
 on the int32 map -- cluster sets, tokens, logits and token ids -- on every
 path that reads the map (the fused B = 1 decode, the batched decode with its
-de-duplicated tensor-core gather and the B >= 64 GEMM, Gumbel sampling,
+de-duplicated tensor-core gather and the centroid GEMM, Gumbel sampling,
 explicit candidate logits), and those outputs hold against the fp64 oracle.
 fh_create checks the uint16 map like the int32 one and refuses it past
 v = 65536.

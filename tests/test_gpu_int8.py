@@ -2,7 +2,7 @@
 
 Every kernel that reads centroid rows has an INT8 form: the fused
 single-token decode (register-streamed and bulk-copied rows), the batched
-score kernel (B < 64) and the tcgen05 GEMM (B >= 64, codes * scale written as
+score kernel (B < 16) and the tcgen05 GEMM (B >= 16, codes * scale written as
 exact hi + lo bf16 pairs). Cases: the tiny planted head (several tiles,
 ragged tails), d = 288 (a ragged lane stride), and the Llama-3.2-1B-shaped
 head at one token per call.

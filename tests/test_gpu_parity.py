@@ -143,11 +143,12 @@ def test_workspace_limit_gives_oom(fh, monkeypatch):
 # ---------------------------------------------------------------------------
 # stage 1: centroid scores
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("cfg_id,B", [(0, 1), (0, 32), (0, 64), (0, 65), (1, 1), (2, 1), (2, 4), (2, 16), (3, 32),
-                                      (4, 256)])
+@pytest.mark.parametrize("cfg_id,B", [(0, 1), (0, 7), (0, 8), (0, 32), (0, 64), (0, 65), (1, 1), (2, 1), (2, 4),
+                                      (2, 15), (2, 16), (3, 32), (4, 256)])
 def test_centroid_scores(fh, cfg_id, B):
-    """B >= 64 runs the tcgen05 tile GEMM (bf16, or INT4 dequantised as exact hi + lo
-    bf16 pairs); smaller batches stream centroid rows on CUDA cores."""
+    """From B = 8 (bf16) or B = 16 (INT4) the tcgen05 tile GEMM scores the centroids
+    (INT4 dequantised as exact hi + lo bf16 pairs); smaller batches stream centroid
+    rows on CUDA cores. Both sides of each threshold are covered."""
     cfg, head, hid, _, dh = get_cfg(cfg_id, fh)
     H = hid.H[:B]
     s = dh.centroid_scores(hid_dev(H)).cpu().numpy()
