@@ -95,7 +95,7 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int, period_ms: int = 50):
+    def __init__(self, gpu_index: int, period_ms: int = 20):
         self.gpu_index = gpu_index
         self.period_ms = period_ms
         self.samples = []
@@ -532,7 +532,7 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                      "frac_of_8TBps": round(achieved / 8000.0, 4),
-                     "algorithmic_bytes": abytes, "kernel": "decode_b1_kernel<8,false>",
+                     "algorithmic_bytes": abytes, "kernel": "decode_b1_kernel<8,0>",
                      "traffic": measured_traffic("decode_b1_llama1b")},
         "selection": {"candidate_list_mean": round(statistics.mean(n for n, _ in sel_stats), 1),
                       "from_all_keys": sum(1 for _, f in sel_stats if f),
