@@ -1,11 +1,14 @@
-"""The allocation-free dense head (fh_dense_head_noalloc) against fh_dense_head,
+"""The allocation-free dense head (fh_dense_head_noalloc) against fh_dense_head
+and against the fp64 oracle's dense head (FlashHead write-up, section 1.1),
 through the C ABI. Its own file, collected last; it passes alone too."""
 import ctypes
 
 import numpy as np
 import pytest
 
+import oracle
 import synth
+from tests import parity
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -44,6 +47,27 @@ def test_matches_dense_head_on_two_calls_in_a_row(env, B):
         torch.cuda.synchronize()
         assert torch.equal(am, ref_am)
         torch.testing.assert_close(z, ref_z, rtol=1e-6, atol=1e-6)
+
+
+@pytest.mark.parametrize("B", [3, 9])
+def test_matches_the_oracle(env, B):
+    # every logit within the fp32 accumulation bound of the oracle's; the argmax equal
+    # to the oracle's unless the two candidates' logits lie within that bound
+    m, lib, cfg, E, H, dh = env
+    _, head, hid, _ = synth.make_config(0, n_states=70)
+    am = torch.full((B,), -1, dtype=torch.int32, device="cuda")
+    z = torch.full((B, cfg.v), float("nan"), dtype=torch.float32, device="cuda")
+    assert _call(lib, E, H, B, z, am) == 0
+    torch.cuda.synchronize()
+    am, z = am.cpu().numpy(), z.cpu().numpy()
+    zr, amr = oracle.dense_head(head.E, hid.H[:B])
+    Ew = oracle.widen_bf16(head.E)
+    for r in range(B):
+        hw = oracle.widen_bf16(hid.H[r])
+        parity.check_values(z[r], zr[r], Ew, hw, f"noalloc dense row {r}")
+        if am[r] != amr[r]:
+            gap = zr[r, amr[r]] - zr[r, am[r]]
+            assert gap <= parity.loose_bound(oracle.widen_bf16(head.E[[am[r], amr[r]]]), hw).sum()
 
 
 def test_argmax_only_and_python_wrapper(env):
