@@ -548,6 +548,9 @@ def run_ours(args):
                 "h2d_bytes_per_step": hd.h2d_bytes, "d2h_bytes_per_step": hd.d2h_bytes},
         "gpu_launches": args.steps,
         "clocks": clocks,
+        "diagnostics": {"intra_cluster_cosine": round(float(synth.intra_cluster_cosine(head)), 4),
+                        "note": "mean cosine between token rows and their centroid over 256 clusters "
+                                "(the pages' clustering health check asks for > 0.6)"},
     }
     if not args.no_cpu_baseline and world == 1:
         rec["cpu_baseline"] = cpu_baseline(head, hid, cfg.p, args.cpu_seconds)
